@@ -1,0 +1,52 @@
+"""The allocator model against the demo program of P3 §三 (main) and its own rules."""
+import json
+import os
+
+import pytest
+
+from oracle.block_pool import BlockPoolModel, ManagerModel, OutOfBlocks, RefcountError
+from pins import GOLDEN
+
+
+def test_demo_program():
+    with open(os.path.join(GOLDEN, "allocator_demo.json")) as f:
+        demo = json.load(f)
+    m = ManagerModel(demo["num_blocks"], demo["block_size"])
+    for st in demo["steps"]:
+        if st["op"] == "allocate_for_request":
+            assert m.allocate_for_request(st["rid"], st["prompt_len"]) == st["returns"]
+            assert m.tables[st["rid"]] == st["table"]
+        elif st["op"] == "append_slot":
+            assert m.append_slot(st["rid"], st["current_len"]) == st["returns"]
+            assert m.tables[st["rid"]] == st["table"]
+        elif st["op"] == "share_prefix_blocks":
+            m.share_prefix_blocks(st["src"], st["dst"], st["shared_len"])
+            assert m.tables[st["dst"]] == st["table"]
+        elif st["op"] == "free_request":
+            m.free_request(st["rid"])
+        for b, r in st.get("refcounts", {}).items():
+            assert m.pool.ref[int(b)] == r, (st, b)
+        if "free_tail" in st:
+            tail = st["free_tail"]
+            assert list(m.pool.free_queue)[-len(tail):] == tail
+    assert m.pool.num_free() == demo["final_num_free"]
+    assert m.pool.usage_ratio() == demo["final_usage"]
+
+
+def test_all_or_nothing_and_errors():
+    p = BlockPoolModel(4, initial_order=[2, 0, 3, 1])
+    assert p.allocate_n(3) == [2, 0, 3]
+    with pytest.raises(OutOfBlocks):
+        p.allocate_n(2)
+    assert p.num_free() == 1 and p.usage_ratio() == 0.75
+    p.free(0)
+    with pytest.raises(RefcountError):
+        p.free(0)                      # double free is an error here, not a silent no-op
+    with pytest.raises(RefcountError):
+        p.add_ref(0)
+    t = p.fork([2, 3])
+    assert t == [2, 3] and p.ref[2] == 2 and p.ref[3] == 2
+    p.free(2)
+    assert p.ref[2] == 1 and 2 not in p.free_queue   # back to the queue only at zero
+    p.free(2)
+    assert list(p.free_queue) == [1, 0, 2]
