@@ -1,0 +1,498 @@
+#!/usr/bin/env python3
+"""Benchmark of the paged decode step on B200: tokens/s and KV-cache GB/s.
+
+One step = the whole hot path for one decode step of one layer over a batch:
+K1 (pa_reshape_and_cache: each sequence's new K/V into its slot), then K2 (+K3)
+(pa_decode: attention over every sequence's paged context, split partitions
+merged).  The slot resolution a1 (host allocator) is timed separately and
+reported as ``a1_us``.  One new token per sequence per step: tokens/s =
+num_seqs / step time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama7b]
+    python bench.py --impl reference ...      # the fp64 CPU oracle on host cores
+
+Under torchrun (N > 1) every rank runs an independent replica of the workload on
+its own GPU (the decode path has no exchange step), time is the max over ranks,
+and the value is the sum of all ranks' tokens over that time (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attention tokens/s and KV-cache HBM GB/s (fraction of ~8 TB/s) on 1 B200"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "paged_decode_llama7b.md")
+DECODE_SOURCE = os.path.join(ROOT, "paged_kv_cache_374_b200", "csrc", "paged_decode.cu")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--workload", default="llama7b")
+    p.add_argument("--impl", default="native", choices=["native", "reference"])
+    p.add_argument("--partition-tokens", type=int, default=0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-clocks", action="store_true")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(units_now: int):
+    """DRAM bytes per launch of K2 from the committed ncu summary, scaled to this
+    launch's tokens; None when the summary is missing or the kernel source has
+    changed since the counters were taken."""
+    try:
+        fields = {}
+        with open(PROFILE_SUMMARY) as f:
+            for line in f:
+                if line.startswith("- ") and ": " in line:
+                    k, v = line[2:].split(": ", 1)
+                    fields[k.strip()] = v.strip().strip("`")
+        if fields.get("source_sha256_16") != source_digest(DECODE_SOURCE):
+            return None
+        per_token = float(fields["dram_bytes_per_launch"]) / float(fields["tokens_per_launch"])
+        return per_token * units_now
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.lines = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", self.gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, fl in enumerate(flags) if fl.lower() == "active"})
+        sm = [r[0] for r in rows]
+        loaded = [x for x in sm if x >= 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def gpu_uuid(torch, device):
+    try:
+        u = str(torch.cuda.get_device_properties(device).uuid)
+        return u if u.startswith("GPU-") else f"GPU-{u}"
+    except Exception:
+        return str(device.index or 0)
+
+
+# --------------------------------------------------------------- workload
+
+def build_step(name, device, partition_tokens):
+    """Tables from the library's allocator, one step's slots via a1, tensors on
+    the device.  Returns a dict of everything the timed loop needs."""
+    import torch
+    from paged_kv_cache_374_b200 import binding as pa
+    from paged_kv_cache_374_b200 import workloads as wk
+
+    wl = wk.make_workload(name)
+    spec = wl.spec
+    bs = spec.block_size
+    alloc = pa.BlockAllocator(wl.num_blocks, wl.pool_order)
+    s = spec.num_seqs
+    stored = (wl.context_lens - 1).astype(np.int32)
+    tables = np.full((s, wl.max_blocks_per_seq), -1, dtype=np.int32)
+    have = np.zeros(s, dtype=np.int64)
+    if spec.prefix_tokens:
+        npre = pa.pa_num_required_blocks(spec.prefix_tokens, bs)
+        prefix = alloc.alloc_n(npre)
+        for i in range(s):
+            tables[i, :npre] = alloc.fork(prefix)
+        have[:] = npre
+    for i in range(s):
+        n = pa.pa_num_required_blocks(int(stored[i]), bs) - int(have[i])
+        tables[i, have[i]:have[i] + n] = alloc.alloc_n(n)
+    lens = stored.copy()
+    t0 = time.perf_counter()
+    slots = alloc.append_slots(tables, lens, bs)
+    a1_us = (time.perf_counter() - t0) * 1e6
+    t = wk.make_tensors(wl, device=device)
+    ws_bytes = pa.pa_decode_workspace_size(s, spec.num_heads, spec.num_kv_heads, spec.head_dim, bs,
+                                           wl.max_blocks_per_seq, partition_tokens)
+    d = dict(
+        wl=wl, spec=spec, alloc=alloc, tables_h=tables, lens_h=lens, slots_h=slots, a1_us=a1_us,
+        tables=torch.from_numpy(tables).to(device), lens=torch.from_numpy(lens).to(device),
+        slots=torch.from_numpy(slots).to(device), out=torch.empty_like(t["q"]),
+        workspace=torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device), ws_bytes=ws_bytes,
+        partition_tokens=partition_tokens, **t)
+    return d
+
+
+def algorithmic_bytes(st):
+    """Bytes K2+K3 must move per step: every sequence's K and V rows once (shared
+    prefix blocks once), q in and out back, the table entries read, the lengths,
+    and the partials written by K2 and read by K3."""
+    spec, wl = st["spec"], st["wl"]
+    lens = st["lens_h"].astype(np.int64)
+    e = 2
+    hk, d, h, s, bs = spec.num_kv_heads, spec.head_dim, spec.num_heads, spec.num_seqs, spec.block_size
+    row = 2 * hk * d * e  # K and V of one token, all kv heads
+    if spec.prefix_tokens:
+        unique_tokens = spec.prefix_tokens + int(np.sum(lens - spec.prefix_tokens))
+    else:
+        unique_tokens = int(np.sum(lens))
+    logical_tokens = int(np.sum(lens))
+    from paged_kv_cache_374_b200 import binding as pa
+    ptok = st["partition_tokens"] or pa.pa_decode_partition_tokens(s, h, hk, d, bs, wl.max_blocks_per_seq)
+    nparts = np.where(lens > ptok, -(-lens // ptok), 0)
+    partials = int(np.sum(nparts)) * h * (d + 2) * 4 * 2
+    meta = int(np.sum(-(-lens // bs))) * 4 + 4 * s
+    qo = 2 * s * h * d * e
+    return {"unique": unique_tokens * row + qo + meta + partials,
+            "logical": logical_tokens * row + qo + meta + partials,
+            "unique_tokens": unique_tokens, "k1": 2 * s * hk * d * e * 2 + 8 * s}
+
+
+def static_config(wl, args, world):
+    spec = wl.spec
+    lens = wl.context_lens.astype(np.int64)
+    kv = int(np.sum(lens)) * 2 * spec.num_kv_heads * spec.head_dim * 2
+    return {
+        "workload": f"{spec.name}: {spec.description}",
+        "num_seqs": spec.num_seqs, "num_heads": spec.num_heads, "num_kv_heads": spec.num_kv_heads,
+        "head_dim": spec.head_dim, "block_size": spec.block_size, "seed": spec.seed,
+        "mean_context": float(np.mean(lens)),
+        "partition_tokens": args.partition_tokens or "auto",
+        "l2": "no flush: the paged cache read per step (%.2f GB) is far larger than the 126 MB L2" % (kv / 1e9),
+        "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+    }
+
+
+# --------------------------------------------------------------- native arm
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_374_b200 import binding as pa
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+    st = build_step(args.workload, device, args.partition_tokens)
+    spec = st["spec"]
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        pa.pa_reshape_and_cache(st["k"], st["v"], st["slots"], st["k_cache"], st["v_cache"], stream=stream)
+        pa.pa_decode(st["q"], st["k_cache"], st["v_cache"], st["tables"], st["lens"], spec.scale,
+                     spec.num_kv_heads, st["out"], workspace=st["workspace"],
+                     partition_tokens=st["partition_tokens"], stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    barrier()
+
+    # timed region: K steps, with per-kernel events on the launching stream
+    k1_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    k2_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(gpu_uuid(torch, device)) if not args.no_clocks else None
+    if sampler:
+        sampler.__enter__()
+    barrier()
+    start.record(stream)
+    for i in range(args.steps):
+        k1_ev[i][0].record(stream)
+        pa.pa_reshape_and_cache(st["k"], st["v"], st["slots"], st["k_cache"], st["v_cache"], stream=stream)
+        k1_ev[i][1].record(stream)
+        k2_ev[i][0].record(stream)
+        pa.pa_decode(st["q"], st["k_cache"], st["v_cache"], st["tables"], st["lens"], spec.scale,
+                     spec.num_kv_heads, st["out"], workspace=st["workspace"],
+                     partition_tokens=st["partition_tokens"], stream=stream)
+        k2_ev[i][1].record(stream)
+    stop.record(stream)
+    barrier()
+    if sampler:
+        sampler.__exit__(None, None, None)
+    elapsed_ms = start.elapsed_time(stop)
+    k1_ms = statistics.mean(a.elapsed_time(b) for a, b in k1_ev)
+    k2_ms = statistics.mean(a.elapsed_time(b) for a, b in k2_ev)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # e2e through the binding: per step, H2D of the step's inputs from pinned
+    # host memory, K1, K2(+K3), D2H of the output
+    host = {k: st[k].cpu().pin_memory() for k in ("q", "k", "v", "slots", "tables", "lens")}
+    out_h = torch.empty(st["out"].shape, dtype=st["out"].dtype).pin_memory()
+    dev_in = {k: torch.empty_like(st[k]) for k in host}
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step():
+        for k, v in host.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        pa.pa_reshape_and_cache(dev_in["k"], dev_in["v"], dev_in["slots"], st["k_cache"], st["v_cache"],
+                                stream=stream)
+        pa.pa_decode(dev_in["q"], st["k_cache"], st["v_cache"], dev_in["tables"], dev_in["lens"], spec.scale,
+                     spec.num_kv_heads, st["out"], workspace=st["workspace"],
+                     partition_tokens=st["partition_tokens"], stream=stream)
+        out_h.copy_(st["out"], non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 500))
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    ab = algorithmic_bytes(st)
+    ms_per_step = elapsed_ms / args.steps
+    tokens_per_step = spec.num_seqs
+    value = world * tokens_per_step / (ms_per_step / 1e3)
+    peak, peak_kind = measured_hbm_peak()
+    achieved = ab["unique"] / (k2_ms / 1e3) / 1e9
+    nparts_max = -(-int(st["wl"].max_blocks_per_seq * spec.block_size) // (
+        st["partition_tokens"] or pa.pa_decode_partition_tokens(spec.num_seqs, spec.num_heads, spec.num_kv_heads,
+                                                                 spec.head_dim, spec.block_size,
+                                                                 st["wl"].max_blocks_per_seq)))
+    launches_per_step = 2 + (1 if nparts_max > 1 else 0)
+    result = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": spec.dtype,
+        "data": "synthetic",
+        "config": static_config(st["wl"], args, world),
+        "detail": {
+            "kv_gbs": round(achieved, 1), "frac_of_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+            "kv_bytes_per_step": ab["unique"], "logical_kv_bytes_per_step": ab["logical"],
+            "k1_us": round(k1_ms * 1e3, 2), "k2k3_us": round(k2_ms * 1e3, 2), "a1_us": round(st["a1_us"], 1),
+            "e2e_ms_per_step": round(e2e_ms, 4),
+        },
+        "roofline": {
+            "kernel": "paged_decode_mha_kernel + paged_decode_merge_kernel (timed together: one pa_decode call)",
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+            "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "traffic": profiled_traffic(ab["unique_tokens"]),
+        },
+        "e2e": {"value": round(world * tokens_per_step / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * launches_per_step,
+        "clocks": sampler.summary() if sampler else None,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args.workload, budget_s=12.0)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ------------------------------------------------------------ oracle timing
+
+def oracle_sample(name, max_pairs=None):
+    """Host inputs for the first sequences of a workload (same lengths as the full
+    workload's first sequences), drawn on the CPU."""
+    import torch
+    from paged_kv_cache_374_b200 import workloads as wk
+    from oracle.block_pool import BlockPoolModel
+    import oracle as oracle_pkg
+
+    full = wk.make_workload(name)
+    n = min(full.spec.num_seqs, 4)
+    wl = wk.make_workload(name, num_seqs=n)
+    spec = wl.spec
+    bs = spec.block_size
+    pool = BlockPoolModel(wl.num_blocks, wl.pool_order)
+    tables = np.full((n, wl.max_blocks_per_seq), -1, dtype=np.int32)
+    for i in range(n):
+        k = -(-int(wl.context_lens[i]) // bs)
+        tables[i, :k] = pool.allocate_n(k)
+    t = wk.make_tensors(wl, device="cpu")
+    to_bits = lambda x: x.contiguous().view(torch.int16).numpy().view(np.uint16)
+    q, kc, vc = to_bits(t["q"]), to_bits(t["k_cache"]), to_bits(t["v_cache"])
+    o = oracle_pkg.get()
+    dt = 0 if spec.dtype == "f16" else 1
+    lens = wl.context_lens.copy()
+    slots = o.slot_mapping(tables, lens, bs)
+    kn, vn = to_bits(t["k"]), to_bits(t["v"])
+    return dict(o=o, q=q, kc=kc, vc=vc, tables=tables, lens=lens, slots=slots, k=kn, v=vn, spec=spec, dt=dt)
+
+
+def time_oracle_pairs(smp, pairs, nthreads):
+    o = smp["o"]
+    t0 = time.perf_counter()
+    o.reshape_and_cache(smp["k"], smp["v"], smp["slots"], smp["kc"], smp["vc"])
+    o.decode(smp["q"], smp["kc"], smp["vc"], smp["tables"], smp["lens"], smp["spec"].scale, smp["dt"],
+             pairs=pairs, nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(name, budget_s=12.0):
+    """The oracle as it stands on this host's cores, on a bounded sample: as many
+    (sequence, head) pairs of the workload's first sequences as fit about
+    `budget_s` of wall time; tokens/s counts num_heads pairs as one token."""
+    smp = oracle_sample(name)
+    spec = smp["spec"]
+    nthreads = os.cpu_count() or 1
+    all_pairs = np.array([(s, h) for s in range(len(smp["lens"])) for h in range(spec.num_heads)], dtype=np.int32)
+    probe = all_pairs[:nthreads]
+    t = time_oracle_pairs(smp, probe, nthreads)
+    per_pair = t / len(probe) * nthreads
+    n = int(min(len(all_pairs), max(nthreads, budget_s * nthreads / max(per_pair, 1e-6))))
+    pairs = all_pairs[:n]
+    t = time_oracle_pairs(smp, pairs, nthreads)
+    tokens = n / spec.num_heads
+    return {"value": round(tokens / t, 3), "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+            "sample": f"{n} (sequence, head) pairs of the first {len(smp['lens'])} sequences of {name} "
+                      f"(mean context {float(np.mean(smp['lens'])):.0f}), K1 + fp64 decode, {t:.1f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    smp = oracle_sample(args.workload)
+    spec = smp["spec"]
+    nthreads = os.cpu_count() or 1
+    all_pairs = np.array([(s, h) for s in range(len(smp["lens"])) for h in range(spec.num_heads)], dtype=np.int32)
+    probe = all_pairs[:nthreads]
+    per_pair = time_oracle_pairs(smp, probe, nthreads) / len(probe) * nthreads
+    # size each step so that warmup + steps take about two minutes in all
+    per_step_s = 120.0 / max(1, args.steps + args.warmup)
+    n = int(min(len(all_pairs), max(1, per_step_s * nthreads / max(per_pair, 1e-9))))
+    pairs = all_pairs[:n]
+    for _ in range(args.warmup):
+        time_oracle_pairs(smp, pairs, nthreads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time_oracle_pairs(smp, pairs, nthreads)
+    total = time.perf_counter() - t0
+    tokens = args.steps * n / spec.num_heads
+    value = tokens / total
+    sample = (f"each step: {n} (sequence, head) pairs of the first {len(smp['lens'])} sequences of "
+              f"{args.workload}, K1 + fp64 decode")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": static_config(__import__("paged_kv_cache_374_b200.workloads", fromlist=["x"]).make_workload(
+            args.workload), args, world),
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,208 @@
+/*
+ * pa.h -- C ABI of the B200 paged decode-attention library (libpa.so).
+ *
+ * The library implements the data-parallel hot path of PagedAttention decoding:
+ * the KV cache lives in fixed-size physical blocks of block_size tokens, and each
+ * sequence reaches its tokens through a block table that maps logical block j to
+ * a physical block id.
+ *
+ * Pages cited by title and section:
+ *   P1  "大模型部署中的PagedAttention：KV Cache显存管理突破" (blog.csdn.net)
+ *   P2  "大模型推理优化：KV Cache与PagedAttention技术详解" (intelliparadigm.com)
+ *   P3  "LLM 推理中的 PageAttention 实现原理：虚拟内存管理在 KV Cache 中的创新应用"
+ *       (dpshk.com)
+ *
+ * Conventions for every call
+ *   - Return value: a pa_status code (PA_OK == 0).  Host-side argument checks run
+ *     before anything is launched; on an error nothing is launched or changed.
+ *   - Device pointers are owned by the caller and must stay valid until the work
+ *     queued on `stream` has finished.  Calls are asynchronous on `stream` (a
+ *     cudaStream_t passed as void*; NULL is the legacy default stream) and
+ *     allocate no device or pinned memory.
+ *   - dtype is PA_F16 or PA_BF16 and is the same for q, k, v, the caches and out.
+ *   - Every tensor is contiguous, row-major, in the layout stated, and every
+ *     device pointer is 16-byte aligned.
+ *   - Cache layout: k_cache and v_cache are [num_blocks][block_size][num_kv_heads]
+ *     [head_dim].  Token slot = phys * block_size + offset, so element (slot, h, i)
+ *     sits at (slot * num_kv_heads + h) * head_dim + i.  (The pages fix blocks of
+ *     block_size tokens, P1 §1 and P3 §一, a per-block tensor of (block_size,
+ *     d_model), P1 §2, and a cache of [seq_len, num_heads, head_dim], P2 §2.1; the
+ *     order inside a block is this library's choice.)
+ *   - Bad indices found on the device never fault: the access is skipped and, if
+ *     err_word (a device int32, may be NULL) is given, a PA_DEVERR_* bit is OR-ed
+ *     into it.  The caller clears it.
+ *   - The block allocator is host-only and single-threaded: callers serialise
+ *     access to one allocator (the pages' listing holds a mutex around it, P3 §三).
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer, short workspace, bad id */
+    PA_ERR_UNSUPPORTED = 2,   /* no kernel for this head_dim / block_size / dtype / group */
+    PA_ERR_OUT_OF_BLOCKS = 3, /* the allocator has too few free blocks; nothing was allocated */
+    PA_ERR_REFCOUNT = 4,      /* free or add_ref of a block whose reference count is 0 */
+    PA_ERR_CUDA = 5           /* a CUDA runtime call or kernel launch failed */
+} pa_status;
+
+enum { PA_F16 = 0, PA_BF16 = 1 };
+
+/* Bits OR-ed into *err_word by the kernels. */
+enum {
+    PA_DEVERR_SLOT_RANGE = 1,    /* slot_mapping entry >= num_blocks * block_size (write skipped) */
+    PA_DEVERR_TABLE_RANGE = 2,   /* block_tables entry outside [0, num_blocks) (output row is NaN) */
+    PA_DEVERR_LEN_RANGE = 4,     /* context_len < 0 or > max_blocks_per_seq * block_size (row NaN) */
+    PA_DEVERR_TIMEOUT = 8        /* an in-kernel wait gave up (the output is not valid) */
+};
+
+/* Human-readable name of a pa_status value (static storage). */
+const char* pa_status_string(int status);
+
+/* ------------------------------------------------------------------------ K1 */
+
+/*
+ * pa_reshape_and_cache -- write each new token's K and V rows into their slots.
+ *
+ * Step 3 of a decode step (P2 §2.1: the current token's K/V is added to the
+ * cache before attention runs over all t tokens); the slot of a token is
+ * table[pos / block_size] * block_size + pos % block_size (P3 §三,
+ * BlockTable::get_physical_location).
+ *
+ *   k, v          [num_tokens][num_kv_heads][head_dim], dtype, device
+ *   slot_mapping  [num_tokens] int64, device; a negative entry means "no token"
+ *                 (skipped in silence), an entry >= num_blocks * block_size is
+ *                 skipped and sets PA_DEVERR_SLOT_RANGE
+ *   k_cache, v_cache  [num_blocks][block_size][num_kv_heads][head_dim], device
+ *
+ * For every i < num_tokens with a valid slot and every h < num_kv_heads:
+ *   k_cache[slot_i][h][:] = k[i][h][:], v_cache[slot_i][h][:] = v[i][h][:],
+ * a bit-exact copy.  Slots must be distinct (a repeated slot gets one of the rows).
+ * head_dim must be a multiple of 8.
+ */
+int pa_reshape_and_cache(const void* k, const void* v, const int64_t* slot_mapping, void* k_cache,
+                         void* v_cache, int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, int dtype, int32_t* err_word, void* stream);
+
+/* ------------------------------------------------------------------- K2 + K3 */
+
+/*
+ * Context partition used by pa_decode when partition_tokens == 0: the token span
+ * of one unit of work.  A sequence longer than this is split across CTAs and the
+ * partial results are merged by a second kernel.  Always a multiple of 64.
+ */
+int pa_decode_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq);
+
+/*
+ * Bytes of device workspace pa_decode needs for these sizes (0 when no sequence
+ * can span more than one partition).  partition_tokens: 0 = the default above,
+ * otherwise a positive multiple of 64.  Returns 0 for invalid sizes as well.
+ */
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                int max_blocks_per_seq, int partition_tokens);
+
+/*
+ * pa_decode -- single-query (decode) attention over the paged cache.
+ *
+ * For every sequence s and query head h, with g = num_heads / num_kv_heads and
+ * h_kv = h / g (g consecutive query heads share one K/V head), L = context_lens[s]
+ * tokens in logical order t = 0..L-1, token t at physical block
+ * block_tables[s][t / block_size], offset t % block_size (P3 §三):
+ *     x_t = scale * sum_i q[s][h][i] * K[t][h_kv][i]
+ *     out[s][h][:] = sum_t exp(x_t - M) V[t][h_kv][:] / sum_t exp(x_t - M),  M = max_t x_t
+ * i.e. softmax(q K^T * scale) V as one softmax over all L tokens (P1 §1, first
+ * formula; the per-block sum printed beside it is not normalised and is not what
+ * is computed).  scale is applied as given (1/sqrt(head_dim) is the usual value).
+ * Arithmetic is fp32; the result is rounded once to dtype (round to nearest even).
+ *
+ *   q             [num_seqs][num_heads][head_dim], dtype, device
+ *   k_cache, v_cache  cache layout above, device
+ *   block_tables  [num_seqs][max_blocks_per_seq] int32, device; entries past
+ *                 ceil(L / block_size) are never read
+ *   context_lens  [num_seqs] int32, device; L includes this step's new token;
+ *                 L == 0 gives a row of zeros
+ *   out           [num_seqs][num_heads][head_dim], dtype, device
+ *   partition_tokens  0 = default; else a positive multiple of 64
+ *   workspace     device scratch of pa_decode_workspace_size(...) bytes (may be
+ *                 NULL when that is 0); its contents on entry do not matter
+ *
+ * Supported: head_dim in {64, 128}; block_size in {16, 32, 64}; num_heads a
+ * multiple of num_kv_heads; any num_seqs >= 0.  Otherwise PA_ERR_UNSUPPORTED or
+ * PA_ERR_INVALID_ARG.
+ */
+int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+              const int32_t* context_lens, float scale, int num_kv_heads, void* out, int num_seqs,
+              int num_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+              int dtype, int partition_tokens, void* workspace, size_t workspace_bytes, int32_t* err_word,
+              void* stream);
+
+/* ---------------------------------------------------------- host allocator */
+
+/*
+ * Refcounted block allocator over num_blocks physical block ids, after the block
+ * pool of P3 §三 (BlockPool, BlockTable, PageAttentionManager) and the beam-search
+ * fork of P3 §四:
+ *   - free ids wait in a FIFO queue: allocation takes the front and sets the
+ *     reference count to 1; a block whose count drops to 0 goes to the back;
+ *   - add_ref / fork add one reference per block (prefix sharing, beam fork);
+ *   - multi-block allocation is all-or-nothing.
+ * Unlike the listing's saturating free, freeing or add_ref-ing a block whose
+ * count is 0 is an error (PA_ERR_REFCOUNT) so that double frees surface.
+ * Every call that fails leaves the allocator unchanged.
+ */
+typedef struct pa_allocator pa_allocator;
+
+/* initial_order: NULL for 0..num_blocks-1, else a permutation giving the initial
+ * order of the free queue.  Returns NULL on a bad argument or out of memory. */
+pa_allocator* pa_allocator_create(int num_blocks, const int32_t* initial_order);
+void pa_allocator_destroy(pa_allocator* a);
+
+/* BlockTable::num_required_blocks (P3 §三): ceil(num_tokens / block_size); -1 on bad input. */
+int pa_num_required_blocks(int num_tokens, int block_size);
+
+int pa_alloc(pa_allocator* a, int32_t* out_id);                     /* one block */
+int pa_alloc_n(pa_allocator* a, int n, int32_t* out_ids);           /* n blocks, all or nothing */
+int pa_free(pa_allocator* a, int32_t id);                           /* drop one reference */
+int pa_free_n(pa_allocator* a, int n, const int32_t* ids);          /* drop one reference each (free_request) */
+int pa_add_ref(pa_allocator* a, int32_t id);                        /* one more reference */
+/* dst[i] = src[i] with one more reference each: a beam fork or a shared prefix
+ * (P3 §三 share_prefix_blocks; P3 §四, beam search).  dst may equal src. */
+int pa_fork(pa_allocator* a, const int32_t* src, int n, int32_t* dst);
+int pa_refcount(const pa_allocator* a, int32_t id);                 /* -1 for an id out of range */
+int pa_num_free(const pa_allocator* a);
+int pa_num_blocks(const pa_allocator* a);
+double pa_usage(const pa_allocator* a);                             /* allocated / total (usage_ratio) */
+
+/*
+ * pa_append_slots -- slot resolution for one decode step (host; step a1).
+ *
+ * For each sequence s, n = context_lens[s] tokens are stored before this step.
+ * The new token goes to position n: when n % block_size == 0 a block is
+ * allocated first and written to block_tables[s][n / block_size]
+ * (PageAttentionManager::append_slot, P3 §三).  Then
+ *     slot_mapping[s] = block_tables[s][n / block_size] * block_size + n % block_size
+ * and context_lens[s] becomes n + 1, the length pa_decode takes.
+ *
+ *   block_tables  host int32 [num_seqs][max_blocks_per_seq], in/out
+ *   context_lens  host int32 [num_seqs], in/out
+ *   slot_mapping  host int64 [num_seqs], out
+ * All or nothing: PA_ERR_OUT_OF_BLOCKS (too few free blocks for every sequence on
+ * a boundary) or PA_ERR_INVALID_ARG (a table full, an id out of range) leaves all
+ * three arrays and the allocator unchanged.
+ */
+int pa_append_slots(pa_allocator* a, int32_t* block_tables, int max_blocks_per_seq, int32_t* context_lens,
+                    int num_seqs, int block_size, int64_t* slot_mapping);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

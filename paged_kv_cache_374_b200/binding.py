@@ -1,0 +1,302 @@
+"""Thin Python binding over libpa.so's C ABI (include/pa.h), same names.
+
+Argument marshalling only: torch tensors become device pointers and sizes, numpy
+arrays become host pointers, status codes become ``PAError``.  Every step of the
+path runs in the library's kernels; there is no fallback, and importing this
+module fails loudly when the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_PKG, "libpa.so")
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_OUT_OF_BLOCKS, PA_ERR_REFCOUNT, PA_ERR_CUDA = range(6)
+PA_F16, PA_BF16 = 0, 1
+PA_DEVERR_SLOT_RANGE, PA_DEVERR_TABLE_RANGE, PA_DEVERR_LEN_RANGE, PA_DEVERR_TIMEOUT = 1, 2, 4, 8
+
+if not os.path.exists(LIBRARY):
+    raise ImportError(f"{LIBRARY} is missing: build it with `python -m paged_kv_cache_374_b200.build` "
+                      "(the library has no CPU fallback)")
+
+_lib = ctypes.CDLL(LIBRARY)
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+def _sig(name, restype, *argtypes):
+    f = getattr(_lib, name)
+    f.restype = restype
+    f.argtypes = list(argtypes)
+    return f
+
+
+_sig("pa_status_string", ctypes.c_char_p, _i32)
+_sig("pa_reshape_and_cache", _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp)
+_sig("pa_decode_partition_tokens", _i32, _i32, _i32, _i32, _i32, _i32, _i32)
+_sig("pa_decode_workspace_size", ctypes.c_size_t, _i32, _i32, _i32, _i32, _i32, _i32, _i32)
+_sig("pa_decode", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+     _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
+_sig("pa_allocator_create", _vp, _i32, _i32p)
+_sig("pa_allocator_destroy", None, _vp)
+_sig("pa_num_required_blocks", _i32, _i32, _i32)
+_sig("pa_alloc", _i32, _vp, _i32p)
+_sig("pa_alloc_n", _i32, _vp, _i32, _i32p)
+_sig("pa_free", _i32, _vp, ctypes.c_int32)
+_sig("pa_free_n", _i32, _vp, _i32, _i32p)
+_sig("pa_add_ref", _i32, _vp, ctypes.c_int32)
+_sig("pa_fork", _i32, _vp, _i32p, _i32, _i32p)
+_sig("pa_refcount", _i32, _vp, ctypes.c_int32)
+_sig("pa_num_free", _i32, _vp)
+_sig("pa_num_blocks", _i32, _vp)
+_sig("pa_usage", ctypes.c_double, _vp)
+_sig("pa_append_slots", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32, _i64p)
+
+
+class PAError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        name = _lib.pa_status_string(status).decode()
+        super().__init__(f"{what}: {name}" if what else name)
+
+
+def _check(status: int, what: str):
+    if status != PA_OK:
+        raise PAError(status, what)
+
+
+def pa_status_string(status: int) -> str:
+    return _lib.pa_status_string(status).decode()
+
+
+# ----------------------------------------------------------------- tensors
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float16:
+        return PA_F16
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: float16 or bfloat16")
+
+
+def _dev(t, name, dtype=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, like):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(like.device)
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def pa_reshape_and_cache(k, v, slot_mapping, k_cache, v_cache, err_word=None, stream=None) -> None:
+    """K1.  k, v [N, Hk, d]; slot_mapping int64 [N]; caches [NB, B, Hk, d] (CUDA)."""
+    import torch
+    n, hk, d = k.shape
+    nb, bs, hk2, d2 = k_cache.shape
+    if v.shape != k.shape or v_cache.shape != k_cache.shape or (hk2, d2) != (hk, d):
+        raise ValueError("shape mismatch")
+    if slot_mapping.shape != (n,):
+        raise ValueError("slot_mapping must be [num_tokens]")
+    dt = _dtype_code(k)
+    for t in (v, k_cache, v_cache):
+        if t.dtype != k.dtype:
+            raise TypeError("k, v and the caches must share one dtype")
+    st = _lib.pa_reshape_and_cache(_dev(k, "k"), _dev(v, "v"), _dev(slot_mapping, "slot_mapping", torch.int64),
+                                   _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), n, hk, d, bs, nb, dt,
+                                   _dev(err_word, "err_word", torch.int32), _stream(stream, k))
+    _check(st, "pa_reshape_and_cache")
+
+
+def pa_decode_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq) -> int:
+    return _lib.pa_decode_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                           max_blocks_per_seq)
+
+
+def pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                             partition_tokens=0) -> int:
+    return _lib.pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                         max_blocks_per_seq, partition_tokens)
+
+
+def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out, workspace=None,
+              partition_tokens=0, err_word=None, stream=None):
+    """K2 + K3.  q/out [S, H, d]; caches [NB, B, Hk, d]; block_tables int32 [S, MB];
+    context_lens int32 [S]; workspace: a CUDA uint8 tensor of at least
+    pa_decode_workspace_size(...) bytes, or None to have one made here (torch).
+    Returns ``out``."""
+    import torch
+    s, h, d = q.shape
+    nb, bs, hk, d2 = k_cache.shape
+    if hk != num_kv_heads or d2 != d or v_cache.shape != k_cache.shape or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [S, MB] and context_lens [S]")
+    mb = block_tables.shape[1]
+    dt = _dtype_code(q)
+    for t in (k_cache, v_cache, out):
+        if t.dtype != q.dtype:
+            raise TypeError("q, the caches and out must share one dtype")
+    need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = _lib.pa_decode(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                        _dev(block_tables, "block_tables", torch.int32),
+                        _dev(context_lens, "context_lens", torch.int32), float(scale), hk, _dev(out, "out"),
+                        s, h, d, bs, nb, mb, dt, int(partition_tokens), ws_ptr, ws_bytes,
+                        _dev(err_word, "err_word", torch.int32), _stream(stream, q))
+    _check(st, "pa_decode")
+    return out
+
+
+# --------------------------------------------------------------- allocator
+
+def _np_i32(a, name):
+    a = np.asarray(a)
+    if a.dtype != np.int32 or not a.flags.c_contiguous:
+        raise TypeError(f"{name} must be a C-contiguous int32 array")
+    return a
+
+
+def pa_allocator_create(num_blocks: int, initial_order=None) -> int:
+    order = None
+    if initial_order is not None:
+        order = np.ascontiguousarray(initial_order, dtype=np.int32)
+        if order.shape != (num_blocks,):
+            raise ValueError("initial_order must have num_blocks entries")
+    h = _lib.pa_allocator_create(num_blocks, order.ctypes.data_as(_i32p) if order is not None else None)
+    if not h:
+        raise PAError(PA_ERR_INVALID_ARG, "pa_allocator_create")
+    return h
+
+
+def pa_allocator_destroy(handle) -> None:
+    _lib.pa_allocator_destroy(handle)
+
+
+def pa_num_required_blocks(num_tokens: int, block_size: int) -> int:
+    return _lib.pa_num_required_blocks(num_tokens, block_size)
+
+
+def pa_alloc(handle) -> int:
+    out = ctypes.c_int32()
+    _check(_lib.pa_alloc(handle, ctypes.byref(out)), "pa_alloc")
+    return out.value
+
+
+def pa_alloc_n(handle, n: int) -> np.ndarray:
+    out = np.empty(n, dtype=np.int32)
+    _check(_lib.pa_alloc_n(handle, n, out.ctypes.data_as(_i32p)), "pa_alloc_n")
+    return out
+
+
+def pa_free(handle, block_id: int) -> None:
+    _check(_lib.pa_free(handle, int(block_id)), "pa_free")
+
+
+def pa_free_n(handle, ids) -> None:
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    _check(_lib.pa_free_n(handle, ids.size, ids.ctypes.data_as(_i32p)), "pa_free_n")
+
+
+def pa_add_ref(handle, block_id: int) -> None:
+    _check(_lib.pa_add_ref(handle, int(block_id)), "pa_add_ref")
+
+
+def pa_fork(handle, src) -> np.ndarray:
+    src = np.ascontiguousarray(src, dtype=np.int32)
+    dst = np.empty_like(src)
+    _check(_lib.pa_fork(handle, src.ctypes.data_as(_i32p), src.size, dst.ctypes.data_as(_i32p)), "pa_fork")
+    return dst
+
+
+def pa_refcount(handle, block_id: int) -> int:
+    return _lib.pa_refcount(handle, int(block_id))
+
+
+def pa_num_free(handle) -> int:
+    return _lib.pa_num_free(handle)
+
+
+def pa_num_blocks(handle) -> int:
+    return _lib.pa_num_blocks(handle)
+
+
+def pa_usage(handle) -> float:
+    return _lib.pa_usage(handle)
+
+
+def pa_append_slots(handle, block_tables: np.ndarray, context_lens: np.ndarray, block_size: int) -> np.ndarray:
+    """In place on block_tables (int32 [S, MB]) and context_lens (int32 [S]); returns slot_mapping int64 [S]."""
+    tables = _np_i32(block_tables, "block_tables")
+    lens = _np_i32(context_lens, "context_lens")
+    s, mb = tables.shape
+    slots = np.empty(s, dtype=np.int64)
+    _check(_lib.pa_append_slots(handle, tables.ctypes.data_as(_i32p), mb, lens.ctypes.data_as(_i32p), s,
+                                block_size, slots.ctypes.data_as(_i64p)), "pa_append_slots")
+    return slots
+
+
+class BlockAllocator:
+    """Owning wrapper over a pa_allocator handle."""
+
+    def __init__(self, num_blocks: int, initial_order=None):
+        self.handle = pa_allocator_create(num_blocks, initial_order)
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h:
+            pa_allocator_destroy(h)
+            self.handle = None
+
+    def alloc(self) -> int:
+        return pa_alloc(self.handle)
+
+    def alloc_n(self, n: int) -> np.ndarray:
+        return pa_alloc_n(self.handle, n)
+
+    def free(self, block_id: int) -> None:
+        pa_free(self.handle, block_id)
+
+    def free_n(self, ids) -> None:
+        pa_free_n(self.handle, ids)
+
+    def add_ref(self, block_id: int) -> None:
+        pa_add_ref(self.handle, block_id)
+
+    def fork(self, src) -> np.ndarray:
+        return pa_fork(self.handle, src)
+
+    def refcount(self, block_id: int) -> int:
+        return pa_refcount(self.handle, block_id)
+
+    def num_free(self) -> int:
+        return pa_num_free(self.handle)
+
+    def num_blocks(self) -> int:
+        return pa_num_blocks(self.handle)
+
+    def usage(self) -> float:
+        return pa_usage(self.handle)
+
+    def append_slots(self, block_tables: np.ndarray, context_lens: np.ndarray, block_size: int) -> np.ndarray:
+        return pa_append_slots(self.handle, block_tables, context_lens, block_size)

@@ -1,0 +1,205 @@
+// Host block allocator behind the pa_allocator_* / pa_append_slots calls.
+//
+// The block pool of P3 ("LLM 推理中的 PageAttention 实现原理", §三: BlockPool,
+// BlockTable, PageAttentionManager) as a flat C++ structure: one int32 reference
+// count per physical block and a ring buffer holding the FIFO free queue.  The
+// ring has exactly num_blocks slots, enough because a block sits in the queue only
+// while its count is zero.  Every operation validates first and mutates second, so
+// a failing call leaves the allocator as it was.
+#include <cstdint>
+#include <cstdlib>
+#include <new>
+#include <vector>
+
+#include "../../include/pa.h"
+
+struct pa_allocator {
+    int32_t n = 0;
+    std::vector<int32_t> ref;    // reference count per block
+    std::vector<int32_t> ring;   // free queue storage
+    int32_t head = 0;            // index of the queue's front in `ring`
+    int32_t count = 0;           // blocks in the queue
+
+    int32_t pop_front() {
+        int32_t id = ring[head];
+        head = head + 1 == n ? 0 : head + 1;
+        --count;
+        return id;
+    }
+    void push_back(int32_t id) {
+        int32_t tail = head + count;
+        if (tail >= n) tail -= n;
+        ring[tail] = id;
+        ++count;
+    }
+    bool valid(int32_t id) const { return id >= 0 && id < n; }
+};
+
+extern "C" {
+
+pa_allocator* pa_allocator_create(int num_blocks, const int32_t* initial_order) {
+    if (num_blocks < 0) return nullptr;
+    pa_allocator* a = new (std::nothrow) pa_allocator();
+    if (!a) return nullptr;
+    try {
+        a->n = num_blocks;
+        a->ref.assign(num_blocks, 0);
+        a->ring.resize(num_blocks);
+    } catch (...) {
+        delete a;
+        return nullptr;
+    }
+    std::vector<char> seen(num_blocks, 0);
+    for (int i = 0; i < num_blocks; ++i) {
+        int32_t id = initial_order ? initial_order[i] : i;
+        if (id < 0 || id >= num_blocks || seen[id]) {  // not a permutation
+            delete a;
+            return nullptr;
+        }
+        seen[id] = 1;
+        a->ring[i] = id;
+    }
+    a->head = 0;
+    a->count = num_blocks;
+    return a;
+}
+
+void pa_allocator_destroy(pa_allocator* a) { delete a; }
+
+int pa_num_required_blocks(int num_tokens, int block_size) {
+    if (num_tokens < 0 || block_size <= 0) return -1;
+    return (int)(((int64_t)num_tokens + block_size - 1) / block_size);
+}
+
+int pa_alloc(pa_allocator* a, int32_t* out_id) {
+    if (!a || !out_id) return PA_ERR_INVALID_ARG;
+    if (a->count == 0) return PA_ERR_OUT_OF_BLOCKS;
+    int32_t id = a->pop_front();
+    a->ref[id] = 1;
+    *out_id = id;
+    return PA_OK;
+}
+
+int pa_alloc_n(pa_allocator* a, int n, int32_t* out_ids) {
+    if (!a || n < 0 || (n > 0 && !out_ids)) return PA_ERR_INVALID_ARG;
+    if (a->count < n) return PA_ERR_OUT_OF_BLOCKS;  // checked before anything is taken
+    for (int i = 0; i < n; ++i) {
+        int32_t id = a->pop_front();
+        a->ref[id] = 1;
+        out_ids[i] = id;
+    }
+    return PA_OK;
+}
+
+int pa_free(pa_allocator* a, int32_t id) {
+    if (!a || !a->valid(id)) return PA_ERR_INVALID_ARG;
+    if (a->ref[id] == 0) return PA_ERR_REFCOUNT;
+    if (--a->ref[id] == 0) a->push_back(id);
+    return PA_OK;
+}
+
+int pa_free_n(pa_allocator* a, int n, const int32_t* ids) {
+    if (!a || n < 0 || (n > 0 && !ids)) return PA_ERR_INVALID_ARG;
+    // Validate against the counts the sequence of frees would see (an id may repeat).
+    std::vector<int32_t> drops;
+    try {
+        drops.assign(n, 0);
+    } catch (...) {
+        return PA_ERR_INVALID_ARG;
+    }
+    for (int i = 0; i < n; ++i) {
+        if (!a->valid(ids[i])) return PA_ERR_INVALID_ARG;
+        int seen = 0;
+        for (int j = 0; j < i; ++j) seen += ids[j] == ids[i];
+        if (a->ref[ids[i]] - seen <= 0) return PA_ERR_REFCOUNT;
+    }
+    for (int i = 0; i < n; ++i) {
+        int32_t id = ids[i];
+        if (--a->ref[id] == 0) a->push_back(id);
+    }
+    return PA_OK;
+}
+
+int pa_add_ref(pa_allocator* a, int32_t id) {
+    if (!a || !a->valid(id)) return PA_ERR_INVALID_ARG;
+    if (a->ref[id] == 0) return PA_ERR_REFCOUNT;
+    ++a->ref[id];
+    return PA_OK;
+}
+
+int pa_fork(pa_allocator* a, const int32_t* src, int n, int32_t* dst) {
+    if (!a || n < 0 || (n > 0 && (!src || !dst))) return PA_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        if (!a->valid(src[i])) return PA_ERR_INVALID_ARG;
+        if (a->ref[src[i]] == 0) return PA_ERR_REFCOUNT;
+    }
+    for (int i = 0; i < n; ++i) {
+        int32_t id = src[i];
+        ++a->ref[id];
+        dst[i] = id;
+    }
+    return PA_OK;
+}
+
+int pa_refcount(const pa_allocator* a, int32_t id) {
+    if (!a || !a->valid(id)) return -1;
+    return a->ref[id];
+}
+
+int pa_num_free(const pa_allocator* a) { return a ? a->count : -1; }
+
+int pa_num_blocks(const pa_allocator* a) { return a ? a->n : -1; }
+
+double pa_usage(const pa_allocator* a) {
+    if (!a || a->n == 0) return 0.0;
+    return (double)(a->n - a->count) / (double)a->n;
+}
+
+int pa_append_slots(pa_allocator* a, int32_t* block_tables, int max_blocks_per_seq, int32_t* context_lens,
+                    int num_seqs, int block_size, int64_t* slot_mapping) {
+    if (!a || num_seqs < 0 || max_blocks_per_seq < 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
+    if (num_seqs > 0 && (!block_tables || !context_lens || !slot_mapping)) return PA_ERR_INVALID_ARG;
+    // Pass 1: validate and count the sequences that sit on a block boundary.
+    int need = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        int64_t n = context_lens[s];
+        if (n < 0 || n == INT32_MAX) return PA_ERR_INVALID_ARG;
+        int64_t j = n / block_size;
+        if (j >= max_blocks_per_seq) return PA_ERR_INVALID_ARG;  // the table row is full
+        if (n % block_size == 0) {
+            ++need;
+        } else {
+            int32_t id = block_tables[(int64_t)s * max_blocks_per_seq + j];
+            if (!a->valid(id) || a->ref[id] == 0) return PA_ERR_INVALID_ARG;
+        }
+    }
+    if (a->count < need) return PA_ERR_OUT_OF_BLOCKS;  // "Preemption required"
+    // Pass 2: allocate in sequence order and resolve each new token's slot.
+    for (int s = 0; s < num_seqs; ++s) {
+        int64_t n = context_lens[s];
+        int64_t j = n / block_size;
+        int32_t* row = block_tables + (int64_t)s * max_blocks_per_seq;
+        if (n % block_size == 0) {
+            int32_t id = a->pop_front();
+            a->ref[id] = 1;
+            row[j] = id;
+        }
+        slot_mapping[s] = (int64_t)row[j] * block_size + n % block_size;
+        context_lens[s] = (int32_t)(n + 1);
+    }
+    return PA_OK;
+}
+
+const char* pa_status_string(int status) {
+    switch (status) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+        case PA_ERR_OUT_OF_BLOCKS: return "PA_ERR_OUT_OF_BLOCKS";
+        case PA_ERR_REFCOUNT: return "PA_ERR_REFCOUNT";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA";
+        default: return "PA_ERR_UNKNOWN";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,176 @@
+"""The C++ host allocator against the Python model of the pages' block pool, id for id."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle.block_pool import BlockPoolModel, ManagerModel, OutOfBlocks, RefcountError
+from pins import GOLDEN
+
+
+@pytest.fixture(scope="module")
+def pa():
+    from paged_kv_cache_374_b200 import binding
+    return binding
+
+
+def _expect_error(pa, fn, status):
+    with pytest.raises(pa.PAError) as e:
+        fn()
+    assert e.value.status == status
+
+
+def test_random_operation_sequences_match_the_model(pa):
+    rng = np.random.default_rng(5)
+    for trial in range(20):
+        n = int(rng.integers(1, 40))
+        order = rng.permutation(n).astype(np.int32) if trial % 2 else None
+        a = pa.BlockAllocator(n, order)
+        m = BlockPoolModel(n, order)
+        held = []  # one entry per reference held
+        for _ in range(400):
+            op = rng.integers(0, 6)
+            if op == 0:
+                k = int(rng.integers(0, 5))
+                try:
+                    want = m.allocate_n(k)
+                except OutOfBlocks:
+                    _expect_error(pa, lambda: a.alloc_n(k), pa.PA_ERR_OUT_OF_BLOCKS)
+                    continue
+                assert list(a.alloc_n(k)) == want
+                held += want
+            elif op == 1 and held:
+                b = held.pop(int(rng.integers(0, len(held))))
+                m.free(b)
+                a.free(b)
+            elif op == 2 and held:
+                b = held[int(rng.integers(0, len(held)))]
+                m.add_ref(b)
+                a.add_ref(b)
+                held.append(b)
+            elif op == 3 and held:
+                src = [held[int(i)] for i in rng.integers(0, len(held), size=int(rng.integers(1, 4)))]
+                assert list(a.fork(np.array(src, dtype=np.int32))) == m.fork(src)
+                held += src
+            elif op == 4:
+                b = int(rng.integers(0, n))
+                if m.ref[b] == 0:
+                    with pytest.raises(RefcountError):
+                        m.free(b)
+                    _expect_error(pa, lambda: a.free(b), pa.PA_ERR_REFCOUNT)
+                    _expect_error(pa, lambda: a.add_ref(b), pa.PA_ERR_REFCOUNT)
+            elif op == 5:
+                try:
+                    want = m.allocate()
+                except OutOfBlocks:
+                    _expect_error(pa, a.alloc, pa.PA_ERR_OUT_OF_BLOCKS)
+                    continue
+                assert a.alloc() == want
+                held.append(want)
+            assert a.num_free() == m.num_free()
+            assert a.usage() == pytest.approx(m.usage_ratio(), abs=0)
+            for b in range(n):
+                assert a.refcount(b) == m.ref[b]
+        # drain: the free queue order must match too
+        for b in held:
+            a.free(b)
+            m.free(b)
+        assert list(a.alloc_n(n)) == list(m.allocate_n(n))
+
+
+def test_free_n_and_fork_are_all_or_nothing(pa):
+    a = pa.BlockAllocator(6)
+    ids = a.alloc_n(4)
+    _expect_error(pa, lambda: a.free_n([ids[0], ids[1], 5]), pa.PA_ERR_REFCOUNT)   # 5 is free
+    assert [a.refcount(int(b)) for b in ids] == [1, 1, 1, 1]
+    _expect_error(pa, lambda: a.free_n([ids[0], ids[0]]), pa.PA_ERR_REFCOUNT)      # second drop would underflow
+    assert a.refcount(int(ids[0])) == 1
+    _expect_error(pa, lambda: a.fork(np.array([ids[0], 4], dtype=np.int32)), pa.PA_ERR_REFCOUNT)
+    assert a.refcount(int(ids[0])) == 1
+    _expect_error(pa, lambda: a.alloc_n(3), pa.PA_ERR_OUT_OF_BLOCKS)
+    assert a.num_free() == 2
+    _expect_error(pa, lambda: a.free(99), pa.PA_ERR_INVALID_ARG)
+    assert a.refcount(99) == -1
+
+
+def test_create_rejects_non_permutations(pa):
+    with pytest.raises(pa.PAError):
+        pa.BlockAllocator(3, np.array([0, 0, 1], dtype=np.int32))
+    with pytest.raises(pa.PAError):
+        pa.BlockAllocator(3, np.array([0, 1, 3], dtype=np.int32))
+
+
+def test_demo_program_through_the_library(pa):
+    """P3 §三 main(), with per-request tables kept by the caller."""
+    with open(os.path.join(GOLDEN, "allocator_demo.json")) as f:
+        demo = json.load(f)
+    bs = demo["block_size"]
+    a = pa.BlockAllocator(demo["num_blocks"])
+    tables = {}
+    for st in demo["steps"]:
+        if st["op"] == "allocate_for_request":
+            n = pa.pa_num_required_blocks(st["prompt_len"], bs)
+            assert n == st["returns"]
+            tables[st["rid"]] = list(a.alloc_n(n))
+        elif st["op"] == "append_slot":
+            # append_slot allocates only on a block boundary
+            if st["current_len"] % bs == 0:
+                tables[st["rid"]].append(a.alloc())
+        elif st["op"] == "share_prefix_blocks":
+            n = pa.pa_num_required_blocks(st["shared_len"], bs)
+            tables[st["dst"]] = list(a.fork(np.array(tables[st["src"]][:n], dtype=np.int32)))
+        elif st["op"] == "free_request":
+            a.free_n(np.array(tables.pop(st["rid"]), dtype=np.int32))
+        if "table" in st:
+            rid = st.get("rid", st.get("dst"))
+            assert tables[rid] == st["table"]
+        for b, r in st.get("refcounts", {}).items():
+            assert a.refcount(int(b)) == r
+    assert a.num_free() == demo["final_num_free"] and a.usage() == demo["final_usage"]
+    # the freed blocks were requeued at the back in the order the demo frees them
+    assert list(a.alloc_n(1024))[-4:] == [2, 3, 0, 1]
+
+
+def test_append_slots_matches_model_and_oracle(pa, oracle):
+    rng = np.random.default_rng(9)
+    bs, s, mb = 16, 12, 12
+    nb = 200
+    order = rng.permutation(nb).astype(np.int32)
+    a = pa.BlockAllocator(nb, order)
+    mgr = ManagerModel(nb, bs, order)
+    lens = rng.integers(0, 100, size=s).astype(np.int32)
+    tables = np.full((s, mb), -1, dtype=np.int32)
+    for i in range(s):
+        n = pa.pa_num_required_blocks(int(lens[i]), bs)
+        mgr.allocate_for_request(i, int(lens[i]))
+        tables[i, :n] = a.alloc_n(n)
+        assert list(tables[i, :n]) == mgr.tables[i]
+    for step in range(40):
+        before = lens.copy()
+        slots = a.append_slots(tables, lens, bs)
+        for i in range(s):
+            mgr.append_slot(i, int(before[i]))
+            assert list(tables[i, :len(mgr.tables[i])]) == mgr.tables[i]
+        assert np.array_equal(lens, before + 1)
+        assert np.array_equal(slots, oracle.slot_mapping(tables, lens, bs))
+        assert a.num_free() == mgr.pool.num_free()
+
+
+def test_append_slots_is_all_or_nothing(pa):
+    bs = 16
+    a = pa.BlockAllocator(3)
+    tables = np.full((3, 4), -1, dtype=np.int32)
+    lens = np.array([16, 32, 5], dtype=np.int32)
+    tables[0, 0] = a.alloc()
+    tables[1, :2] = a.alloc_n(2)
+    tables[2, 0] = -1   # token 5 would land in a block the table does not hold
+    t0, l0 = tables.copy(), lens.copy()
+    _expect_error(pa, lambda: a.append_slots(tables, lens, bs), pa.PA_ERR_INVALID_ARG)
+    assert np.array_equal(tables, t0) and np.array_equal(lens, l0) and a.num_free() == 0
+    lens[2] = 0        # now two sequences need a block and none is free: "preemption required"
+    l0 = lens.copy()
+    _expect_error(pa, lambda: a.append_slots(tables, lens, bs), pa.PA_ERR_OUT_OF_BLOCKS)
+    assert np.array_equal(tables, t0) and np.array_equal(lens, l0)
+    full = np.full((1, 1), 0, dtype=np.int32)
+    _expect_error(pa, lambda: a.append_slots(full, np.array([16], dtype=np.int32), bs), pa.PA_ERR_INVALID_ARG)

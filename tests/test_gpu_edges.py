@@ -1,0 +1,141 @@
+"""GPU parity on small paged problems that sweep the supported shapes, plus the
+degenerate and error cases: empty contexts, single tokens, lengths on block and
+partition boundaries, the longest context a table can hold, bad table entries,
+bad lengths and bad slots (reported through the error word, never a fault)."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_cases import assert_close
+from pins import BF16, F16, PagedCase
+import oracle as oracle_pkg
+from paged_kv_cache_374_b200 import binding as pa
+
+pytestmark = pytest.mark.gpu
+
+TDT = {F16: torch.float16, BF16: torch.bfloat16}
+WK = {F16: "f16", BF16: "bf16"}
+
+
+def dev(bits_arr, dtype):
+    return torch.from_numpy(np.ascontiguousarray(bits_arr).view(np.int16)).view(TDT[dtype]).cuda()
+
+
+def run_case(c, partition_tokens=0, err=None, tables=None, lens=None):
+    q = dev(c.q, c.dtype)
+    kc, vc = dev(c.k_cache, c.dtype), dev(c.v_cache, c.dtype)
+    tb = torch.from_numpy(c.tables if tables is None else tables).cuda()
+    ln = torch.from_numpy(c.lens if lens is None else lens).cuda()
+    out = torch.empty_like(q)
+    pa.pa_decode(q, kc, vc, tb, ln, c.scale, c.Hk, out, partition_tokens=partition_tokens, err_word=err)
+    torch.cuda.synchronize()
+    return out
+
+
+SHAPES = list(itertools.product([64, 128], [16, 32, 64], [1, 2, 4, 8], [F16, BF16]))
+
+
+@pytest.mark.parametrize("d,bs,g,dtype", SHAPES)
+def test_shape_sweep(d, bs, g, dtype):
+    rng = np.random.default_rng(d * 1000 + bs * 10 + g + dtype)
+    hk = 2
+    lens = [0, 1, bs - 1, bs, bs + 1, 64, 511, 512, 513, 1000 + bs // 2]
+    c = PagedCase(rng, lens, hk * g, hk, d, bs, dtype, 1 / math.sqrt(d), extra_blocks=4)
+    ref = c.run(oracle_pkg.get(), nthreads=8)
+    for pt in (0, 64, 192):
+        out = run_case(c, partition_tokens=pt)
+        assert_close(out, ref, WK[dtype], f"d{d} bs{bs} g{g} pt{pt}")
+        assert torch.count_nonzero(out[0]) == 0            # empty context: zeros
+
+
+def test_split_invariance_and_relabelling():
+    rng = np.random.default_rng(31)
+    c = PagedCase(rng, [3000, 1500, 64, 4096], 8, 8, 128, 16, F16, 0.088, extra_blocks=10)
+    outs = [run_case(c, partition_tokens=pt).double() for pt in (64, 512, 4096)]
+    assert (outs[0] - outs[2]).abs().max().item() <= 2e-3
+    assert (outs[1] - outs[2]).abs().max().item() <= 2e-3
+    a = run_case(c)
+    c.relabel(rng.permutation(c.NB).astype(np.int32))
+    b = run_case(c)
+    assert torch.equal(a, b), "relabelling physical blocks changed the output"
+
+
+def test_longest_context_and_large_scores():
+    rng = np.random.default_rng(32)
+    c = PagedCase(rng, [64 * 40, 7], 4, 4, 128, 64, BF16, 0.5, extra_blocks=1)   # table exactly full for seq 0
+    ref = c.run(oracle_pkg.get(), nthreads=8)
+    assert_close(run_case(c), ref, "bf16", "full table, large scores")
+
+
+def test_bad_table_entry_gives_nan_row_and_error_bit():
+    rng = np.random.default_rng(33)
+    c = PagedCase(rng, [40, 40, 900], 4, 4, 64, 16, F16, 0.125)
+    ref = c.run(oracle_pkg.get())
+    for bad in (c.NB + 3, -2):
+        tables = c.tables.copy()
+        tables[1, 1] = bad
+        tables[2, 40] = bad          # inside a later partition of sequence 2
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out = run_case(c, err=err, tables=tables)
+        assert err.item() & pa.PA_DEVERR_TABLE_RANGE
+        assert torch.isnan(out[1]).all() and torch.isnan(out[2]).all()
+        assert_close(out[0], ref[0], "f16", "unaffected row")
+
+
+def test_bad_context_len_gives_nan_row_and_error_bit():
+    rng = np.random.default_rng(34)
+    c = PagedCase(rng, [20, 20], 2, 2, 64, 16, F16, 0.125)
+    lens = c.lens.copy()
+    lens[0] = c.MB * 16 + 1
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = run_case(c, err=err, lens=lens)
+    assert err.item() & pa.PA_DEVERR_LEN_RANGE
+    assert torch.isnan(out[0]).all() and not torch.isnan(out[1]).any()
+
+
+def test_reshape_and_cache_slots():
+    """Negative slots are skipped in silence; slots past the pool set an error bit
+    and are skipped; the rest is a bit-exact copy (compared with the oracle)."""
+    rng = np.random.default_rng(35)
+    nb, bs, hk, d, n = 8, 16, 4, 128, 12
+    for dtype in (torch.float16, torch.bfloat16):
+        kc = torch.randn(nb, bs, hk, d, device="cuda").to(dtype)
+        vc = torch.randn(nb, bs, hk, d, device="cuda").to(dtype)
+        k = torch.randn(n, hk, d, device="cuda").to(dtype)
+        v = torch.randn(n, hk, d, device="cuda").to(dtype)
+        slots = rng.choice(nb * bs, size=n, replace=False).astype(np.int64)
+        slots[2] = -1
+        slots[5] = nb * bs
+        kh, vh = kc.view(torch.int16).cpu().numpy().view(np.uint16), vc.view(torch.int16).cpu().numpy().view(np.uint16)
+        skipped = oracle_pkg.get().reshape_and_cache(k.view(torch.int16).cpu().numpy().view(np.uint16),
+                                                     v.view(torch.int16).cpu().numpy().view(np.uint16),
+                                                     slots, kh, vh)
+        assert skipped == 2
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        pa.pa_reshape_and_cache(k, v, torch.from_numpy(slots).cuda(), kc, vc, err_word=err)
+        torch.cuda.synchronize()
+        assert err.item() == pa.PA_DEVERR_SLOT_RANGE
+        assert np.array_equal(kc.view(torch.int16).cpu().numpy().view(np.uint16), kh)
+        assert np.array_equal(vc.view(torch.int16).cpu().numpy().view(np.uint16), vh)
+
+
+def test_empty_batch_and_binding_checks():
+    q = torch.empty(0, 4, 64, dtype=torch.float16, device="cuda")
+    kc = torch.zeros(4, 16, 4, 64, dtype=torch.float16, device="cuda")
+    tb = torch.zeros(0, 2, dtype=torch.int32, device="cuda")
+    ln = torch.zeros(0, dtype=torch.int32, device="cuda")
+    pa.pa_decode(q, kc, kc, tb, ln, 0.125, 4, torch.empty_like(q))
+    q1 = torch.zeros(1, 4, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(TypeError):
+        pa.pa_decode(q1, kc, kc, tb[:1], ln[:1], 0.125, 4, torch.empty_like(q1))
+    with pytest.raises(pa.PAError) as e:
+        pa.pa_decode(torch.zeros(1, 4, 96, dtype=torch.float16, device="cuda"),
+                     torch.zeros(4, 16, 4, 96, dtype=torch.float16, device="cuda"),
+                     torch.zeros(4, 16, 4, 96, dtype=torch.float16, device="cuda"),
+                     torch.zeros(1, 2, dtype=torch.int32, device="cuda"),
+                     torch.ones(1, dtype=torch.int32, device="cuda"), 0.1, 4,
+                     torch.zeros(1, 4, 96, dtype=torch.float16, device="cuda"))
+    assert e.value.status == pa.PA_ERR_UNSUPPORTED
