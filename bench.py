@@ -43,11 +43,12 @@ DECODE_SOURCE = os.path.join(ROOT, "paged_kv_cache_374_b200", "csrc", "paged_dec
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--steps", type=int, default=5000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--workload", default="llama7b")
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--partition-tokens", type=int, default=0)
+    p.add_argument("--num-seqs", type=int, default=None, help="truncate the batch (smaller profiling case)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
     return p.parse_args()
@@ -162,14 +163,14 @@ def gpu_uuid(torch, device):
 
 # --------------------------------------------------------------- workload
 
-def build_step(name, device, partition_tokens):
+def build_step(name, device, partition_tokens, num_seqs=None):
     """Tables from the library's allocator, one step's slots via a1, tensors on
     the device.  Returns a dict of everything the timed loop needs."""
     import torch
     from paged_kv_cache_374_b200 import binding as pa
     from paged_kv_cache_374_b200 import workloads as wk
 
-    wl = wk.make_workload(name)
+    wl = wk.make_workload(name, num_seqs=num_seqs)
     spec = wl.spec
     bs = spec.block_size
     alloc = pa.BlockAllocator(wl.num_blocks, wl.pool_order)
@@ -197,7 +198,7 @@ def build_step(name, device, partition_tokens):
         wl=wl, spec=spec, alloc=alloc, tables_h=tables, lens_h=lens, slots_h=slots, a1_us=a1_us,
         tables=torch.from_numpy(tables).to(device), lens=torch.from_numpy(lens).to(device),
         slots=torch.from_numpy(slots).to(device), out=torch.empty_like(t["q"]),
-        workspace=torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device), ws_bytes=ws_bytes,
+        workspace=torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=device), ws_bytes=ws_bytes,
         partition_tokens=partition_tokens, **t)
     return d
 
@@ -256,7 +257,7 @@ def run_native(args):
                                 timeout=__import__("datetime").timedelta(seconds=120))
     device = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(device)
-    st = build_step(args.workload, device, args.partition_tokens)
+    st = build_step(args.workload, device, args.partition_tokens, args.num_seqs)
     spec = st["spec"]
     stream = torch.cuda.current_stream(device)
 
@@ -431,23 +432,22 @@ def time_oracle_pairs(smp, pairs, nthreads):
 
 
 def cpu_baseline(name, budget_s=12.0):
-    """The oracle as it stands on this host's cores, on a bounded sample: as many
-    (sequence, head) pairs of the workload's first sequences as fit about
-    `budget_s` of wall time; tokens/s counts num_heads pairs as one token."""
+    """The oracle as it stands on this host's cores, on a bounded sample: every
+    (sequence, head) pair of the workload's first sequences, K1 + fp64 decode,
+    repeated until about `budget_s` of wall time has passed."""
     smp = oracle_sample(name)
     spec = smp["spec"]
     nthreads = os.cpu_count() or 1
-    all_pairs = np.array([(s, h) for s in range(len(smp["lens"])) for h in range(spec.num_heads)], dtype=np.int32)
-    probe = all_pairs[:nthreads]
-    t = time_oracle_pairs(smp, probe, nthreads)
-    per_pair = t / len(probe) * nthreads
-    n = int(min(len(all_pairs), max(nthreads, budget_s * nthreads / max(per_pair, 1e-6))))
-    pairs = all_pairs[:n]
-    t = time_oracle_pairs(smp, pairs, nthreads)
-    tokens = n / spec.num_heads
-    return {"value": round(tokens / t, 3), "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
-            "sample": f"{n} (sequence, head) pairs of the first {len(smp['lens'])} sequences of {name} "
-                      f"(mean context {float(np.mean(smp['lens'])):.0f}), K1 + fp64 decode, {t:.1f} s"}
+    pairs = np.array([(s, h) for s in range(len(smp["lens"])) for h in range(spec.num_heads)], dtype=np.int32)
+    reps, total = 0, 0.0
+    while total < budget_s:
+        total += time_oracle_pairs(smp, pairs, nthreads)
+        reps += 1
+    tokens = reps * len(smp["lens"])
+    return {"value": round(tokens / total, 3), "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+            "sample": f"all {spec.num_heads} heads of the first {len(smp['lens'])} sequences of {name} "
+                      f"(mean context {float(np.mean(smp['lens'])):.0f}), K1 + fp64 decode, repeated {reps} "
+                      f"times in {total:.1f} s"}
 
 
 def run_reference(args):

@@ -102,9 +102,11 @@ int pa_decode_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, in
                                int max_blocks_per_seq);
 
 /*
- * Bytes of device workspace pa_decode needs for these sizes (0 when no sequence
- * can span more than one partition).  partition_tokens: 0 = the default above,
- * otherwise a positive multiple of 64.  Returns 0 for invalid sizes as well.
+ * Bytes of device workspace pa_decode needs for these sizes: 256 bytes of
+ * scheduling counters, plus the partial results of split sequences when a
+ * sequence can span more than one partition.  partition_tokens: 0 = the default
+ * above, otherwise a positive multiple of 64, at most 65536.  Returns 0 for
+ * invalid sizes.
  */
 size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                                 int max_blocks_per_seq, int partition_tokens);
@@ -131,8 +133,13 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, i
  *                 L == 0 gives a row of zeros
  *   out           [num_seqs][num_heads][head_dim], dtype, device
  *   partition_tokens  0 = default; else a positive multiple of 64
- *   workspace     device scratch of pa_decode_workspace_size(...) bytes (may be
- *                 NULL when that is 0); its contents on entry do not matter
+ *   workspace     device scratch of at least pa_decode_workspace_size(...)
+ *                 bytes.  Its first 256 bytes are the kernels' work-claim
+ *                 counters: zero them once before the first call (cudaMemset);
+ *                 every call leaves them zero again, so a workspace can be reused
+ *                 call after call on one stream.  Calls that may run at the same
+ *                 time need separate workspaces.  After a PA_DEVERR_TIMEOUT,
+ *                 zero the counters again.
  *
  * Supported: head_dim in {64, 128}; block_size in {16, 32, 64}; num_heads a
  * multiple of num_kv_heads; any num_seqs >= 0.  Otherwise PA_ERR_UNSUPPORTED or

@@ -155,8 +155,8 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_hea
         if t.dtype != q.dtype:
             raise TypeError("q, the caches and out must share one dtype")
     need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
     ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = _lib.pa_decode(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),

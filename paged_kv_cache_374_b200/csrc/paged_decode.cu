@@ -6,31 +6,35 @@
 // in logical order, token t living in physical block block_tables[s][t / B] at
 // offset t % B -- one softmax over all L tokens.
 //
-// Work decomposition (CUDA cores; fp32 arithmetic throughout):
-//   grid = (num_heads * P, num_seqs): one CTA per (query head, context partition,
-//   sequence).  A partition is `partition_tokens` consecutive tokens; sequences
-//   longer than one partition are split across CTAs whose partial results
-//   (running max m, running sum l, unnormalised o) go to the workspace and are
-//   merged by K3.  Query heads of one sequence are the fastest grid dimension, so
-//   CTAs that run together read the same physical blocks (all heads of a token
-//   row sit next to each other) and the CTAs of a GQA group share tiles in L2.
+// Units of work.  A sequence is cut into partitions of P tokens; a unit is one
+// (sequence, partition, query head).  A sequence of one partition gets its output
+// row directly; a longer one leaves a partial result per partition (running max m,
+// running sum l, unnormalised o) in the workspace, merged by K3.
 //
-// Inside a CTA (4 consumer warps + 1 producer warp):
-//   - the producer warp loads the partition's block-table entries with one
-//     coalesced warp load per 32 entries (each entry is read once, by one warp),
-//     then its lane 0 streams K and V tiles of TOK tokens x head_dim into an
-//     NS-deep shared-memory ring with TMA tensor copies (cp.async.bulk.tensor),
-//     completion tracked by mbarriers (full / empty per stage);
-//   - consumer warp w takes stages w, w+4, ...; per stage it computes the TOK
-//     scores with 16-byte shared loads (a token row is split over CH lanes, one
-//     16-byte chunk each), reduces them with a reduce-scatter over warp shuffles,
-//     updates its online softmax (running max / sum, base-2 exponentials with
-//     log2(e) folded into the pre-scaled q) and accumulates p * V;
-//   - the four warp states are merged through shared memory at the end.
-// Rows past the sequence end inside the last block are never used: their scores
-// become -inf and their V rows are skipped (not multiplied by 0, as they may
-// hold NaN).  Table entries outside [0, num_blocks) are never dereferenced: the
-// stage is dropped, the output row becomes NaN and PA_DEVERR_TABLE_RANGE is set.
+// K2 is persistent: one CTA per SM, NW warps per CTA, and every warp is a
+// self-contained streaming engine -- it claims units from a global counter, loads
+// the unit's block-table entries with one coalesced warp load per 32 entries
+// (each entry is read once, by one warp), and keeps its own ring of R
+// shared-memory slots filled with TMA tensor copies (cp.async.bulk.tensor; one
+// slot = K and V of TOK tokens of one kv head), completion tracked by one
+// mbarrier per slot.  Issue runs R stages ahead of compute and crosses into the
+// next claimed unit before the current one ends, so the warp's copies never drain
+// at unit boundaries.  No warp ever waits for another.
+//
+// Claim order: every full partition first (sequence-major, query heads fastest, so
+// warps running together read the same physical blocks), then each sequence's
+// last partition, longest first, so that the units left at the end are the
+// shortest.  Every CTA derives the same order from context_lens in its prologue.
+//
+// Per stage (fp32 arithmetic): a token row is split over CH lanes (one 16-byte
+// chunk each); partial dot products are reduced by a reduce-scatter over warp
+// shuffles, then the online softmax update (running max / sum, base-2 exponentials
+// with log2(e) folded into the pre-scaled q) and p * V accumulate with packed
+// fp32x2 FMAs.  Rows past the sequence end inside the last block are never used:
+// their scores become -inf and their V rows are skipped (not multiplied by 0, as
+// they may hold NaN).  Table entries outside [0, num_blocks) are never
+// dereferenced: the stage is dropped, the output row becomes NaN and
+// PA_DEVERR_TABLE_RANGE is set.
 #include <cmath>
 
 #include "pa_device.cuh"
@@ -38,41 +42,49 @@
 
 namespace pa {
 
-constexpr int kConsumerWarps = 4;
-constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr int kMaxSeqsPerLaunch = 1024;   // sequences scheduled by one K2 launch
+constexpr int kMaxPartitionTokens = 65536;
 
 struct DecodeArgs {
     const uint16_t* q;
     uint16_t* out;
     const int32_t* block_tables;
     const int32_t* context_lens;
-    float* ws_m;   // [S*H][P]
-    float* ws_l;   // [S*H][P]
-    float* ws_o;   // [S*H][P][D]
+    float* ws_m;      // [S*H][Pmax], base-2 units
+    float* ws_l;      // [S*H][Pmax]
+    float* ws_o;      // [S*H][Pmax][D]
+    int32_t* sched;   // [0] claim counter, [1] finished-warp counter; zero between launches
     int32_t* err_word;
-    float scale_log2;  // scale * log2(e)
+    float scale_log2; // scale * log2(e)
+    int num_seqs;     // sequences in this launch (<= kMaxSeqsPerLaunch)
     int num_heads;
-    int group;         // num_heads / num_kv_heads
+    int group;        // num_heads / num_kv_heads
     int block_size;
+    int box_rows;     // token rows per TMA box (min(TOK, block_size))
     int num_blocks;
     int max_blocks_per_seq;
     int partition_tokens;
-    int num_partitions;  // P: partitions allotted per (s, h) in the workspace
+    int num_partitions;  // Pmax: partitions allotted per (s, h) in the workspace
 };
 
-template <int D, int TOK, int NS>
-struct MhaLayout {
+enum UnitKind { kUnitNone = 0, kUnitNormal = 1, kUnitZero = 2, kUnitNaN = 3 };
+
+struct Unit {
+    int kind;
+    int s, h, p, np;
+    int t_begin, t_end, nst, kv_head, blk0, nblk;
+};
+
+template <int D, int TOK, int NW, int R>
+struct Layout {
     static constexpr int kTileBytes = TOK * D * 2;
-    static constexpr int kOffK = 0;
-    static constexpr int kOffV = NS * kTileBytes;
-    static constexpr int kOffFull = 2 * NS * kTileBytes;
-    static constexpr int kOffEmpty = kOffFull + NS * 8;
-    static constexpr int kOffBad = kOffEmpty + NS * 8;
-    static constexpr int kOffAbort = kOffBad + NS * 4;
-    static constexpr int kOffMergeM = (kOffAbort + 4 + 15) / 16 * 16;
-    static constexpr int kOffMergeL = kOffMergeM + kConsumerWarps * 4;
-    static constexpr int kOffMergeO = kOffMergeL + kConsumerWarps * 4;
-    static constexpr int kBytes = kOffMergeO + kConsumerWarps * D * 4;
+    static constexpr int kSlotBytes = 2 * kTileBytes;          // K tile then V tile
+    static constexpr int kOffSlots = 0;
+    static constexpr int kOffBars = NW * R * kSlotBytes;
+    static constexpr int kOffCum = kOffBars + NW * R * 8;         // int[S + 1]
+    static constexpr int kOffKey = kOffCum + (kMaxSeqsPerLaunch + 1) * 4 + 12;  // uint32[S_pow2]
+    static constexpr int kOffLen = kOffKey + kMaxSeqsPerLaunch * 4;            // int[S]
+    static constexpr int kBytes = kOffLen + kMaxSeqsPerLaunch * 4;
     static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1 KiB
 };
 
@@ -89,264 +101,427 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 template <class Tag>
-__device__ __forceinline__ void widen8(const uint4& w, float (&f)[8]) {
-    float2 a = Tag::widen2(w.x), b = Tag::widen2(w.y), c = Tag::widen2(w.z), d = Tag::widen2(w.w);
-    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
-    f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+__device__ __forceinline__ void widen8(const uint4& w, float2 (&f)[4]) {
+    f[0] = Tag::widen2(w.x);
+    f[1] = Tag::widen2(w.y);
+    f[2] = Tag::widen2(w.z);
+    f[3] = Tag::widen2(w.w);
 }
 
-template <class Tag, int D>
-__device__ __forceinline__ void write_row_const(uint16_t* row, float value) {
-    for (int i = threadIdx.x; i < D; i += blockDim.x) row[i] = Tag::round1(value);
+template <class Tag>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    return (uint32_t)Tag::round1(a) | ((uint32_t)Tag::round1(b) << 16);
 }
 
-template <class Tag, int D, int TOK, int NS>
-__global__ void __launch_bounds__(kDecodeThreads) paged_decode_mha_kernel(const DecodeArgs a,
-                                                                          const __grid_constant__ CUtensorMap kmap,
-                                                                          const __grid_constant__ CUtensorMap vmap) {
-    using Lay = MhaLayout<D, TOK, NS>;
+// Decode claim index u into a unit (warp-uniform; reads the schedule in smem).
+__device__ __forceinline__ Unit decode_unit(int u, const DecodeArgs& a, const int* s_cum, const uint32_t* s_key,
+                                            const int* s_len, int TOK) {
+    Unit U;
+    const int S = a.num_seqs, H = a.num_heads;
+    const int A = s_cum[S];
+    if (u < 0 || u >= H * (A + S)) {
+        U.kind = kUnitNone;
+        U.s = U.h = U.p = U.np = U.t_begin = U.t_end = U.nst = U.kv_head = U.blk0 = U.nblk = 0;
+        return U;
+    }
+    int s, p, h;
+    if (u < H * A) {
+        const int idx = u / H;
+        h = u - idx * H;
+        int lo = 0, hi = S - 1;  // largest s with s_cum[s] <= idx
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_cum[mid] <= idx) lo = mid; else hi = mid - 1;
+        }
+        s = lo;
+        p = idx - s_cum[s];
+    } else {
+        const int v = u - H * A;
+        const int idx = v / H;
+        h = v - idx * H;
+        s = (int)(s_key[idx] & 0xfffu);
+        p = s_cum[s + 1] - s_cum[s];
+    }
+    U.s = s;
+    U.h = h;
+    U.p = p;
+    U.np = s_cum[s + 1] - s_cum[s] + 1;
+    const int L = s_len[s];
+    const int maxlen = a.max_blocks_per_seq * a.block_size;
+    U.kind = (L < 0 || L > maxlen) ? kUnitNaN : (L == 0 ? kUnitZero : kUnitNormal);
+    const int P = a.partition_tokens;
+    U.t_begin = p * P;
+    U.t_end = U.kind == kUnitNormal ? min(L, U.t_begin + P) : U.t_begin;
+    U.nst = (U.t_end - U.t_begin + TOK - 1) / TOK;
+    U.kv_head = h / a.group;
+    U.blk0 = U.t_begin / a.block_size;
+    U.nblk = U.kind == kUnitNormal ? (U.t_end + a.block_size - 1) / a.block_size - U.blk0 : 0;
+    return U;
+}
+
+template <class Tag, int D, int TOK, int NW, int R>
+__global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeArgs a,
+                                                                  const __grid_constant__ CUtensorMap kmap,
+                                                                  const __grid_constant__ CUtensorMap vmap) {
+    using Lay = Layout<D, TOK, NW, R>;
     constexpr int CH = D / 8;       // 16-byte chunks per token row
     constexpr int RPI = 32 / CH;    // token rows covered by one warp-wide 16-byte load
     constexpr int NV = TOK / RPI;   // row groups per stage (values each lane reduces)
     static_assert(NV >= 1 && NV <= CH && CH % NV == 0, "stage shape");
     constexpr int DUP = CH / NV;    // lanes that end up holding the same token's score
     constexpr int SH = DUP == 1 ? 0 : DUP == 2 ? 1 : DUP == 4 ? 2 : DUP == 8 ? 3 : 4;
+    constexpr int MAXSUB = TOK / 16;  // TMA boxes per tile (box_rows >= 16)
+    constexpr unsigned FULL = 0xffffffffu;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::kOffFull);
-    uint64_t* empty = reinterpret_cast<uint64_t*>(smem + Lay::kOffEmpty);
-    volatile int* bad = reinterpret_cast<volatile int*>(smem + Lay::kOffBad);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kOffAbort);
-    float* merge_m = reinterpret_cast<float*>(smem + Lay::kOffMergeM);
-    float* merge_l = reinterpret_cast<float*>(smem + Lay::kOffMergeL);
-    float* merge_o = reinterpret_cast<float*>(smem + Lay::kOffMergeO);
+    int* s_cum = reinterpret_cast<int*>(smem + Lay::kOffCum);
+    uint32_t* s_key = reinterpret_cast<uint32_t*>(smem + Lay::kOffKey);
+    int* s_len = reinterpret_cast<int*>(smem + Lay::kOffLen);
 
-    const int h = blockIdx.x % a.num_heads;
-    const int part = blockIdx.x / a.num_heads;
-    const int s = blockIdx.y;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bs = a.block_size;
-    const int64_t sh = (int64_t)s * a.num_heads + h;
-    uint16_t* out_row = a.out + sh * D;
-
-    const int L = a.context_lens[s];
-    if (L < 0 || L > a.max_blocks_per_seq * bs) {
-        if (part == 0) {
-            write_row_const<Tag, D>(out_row, __int_as_float(0x7fc00000));
-            if (threadIdx.x == 0) report(a.err_word, PA_DEVERR_LEN_RANGE);
-        }
-        return;
-    }
-    if (L == 0) {
-        if (part == 0) write_row_const<Tag, D>(out_row, 0.f);
-        return;
-    }
+    const int S = a.num_seqs;
+    const int H = a.num_heads;
     const int P = a.partition_tokens;
-    const int nparts = (L + P - 1) / P;
-    if (part >= nparts) return;
-    const int t_begin = part * P;
-    const int t_end = min(L, t_begin + P);
-    const int nst = (t_end - t_begin + TOK - 1) / TOK;
-    const int kv_head = h / a.group;
+    const int bs = a.block_size;
+    const int maxlen = a.max_blocks_per_seq * bs;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBars) + warp * R;
+    uint8_t* slots = smem + Lay::kOffSlots + warp * R * Lay::kSlotBytes;
 
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < NS; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
-            bad[i] = 0;
+    // ------------------------------------------------------------- prologue
+    int spow = 1;
+    while (spow < S) spow <<= 1;
+    for (int s = threadIdx.x; s < spow; s += blockDim.x) {
+        if (s < S) {
+            const int L = a.context_lens[s];
+            s_len[s] = L;
+            const bool normal = L > 0 && L <= maxlen;
+            const int np = normal ? (L + P - 1) / P : 1;
+            const int last = normal ? L - (np - 1) * P : 0;
+            s_cum[s] = np - 1;  // full partitions, scanned below
+            s_key[s] = ((uint32_t)(P - last) << 12) | (uint32_t)s;
+        } else {
+            s_key[s] = 0xffffffffu;
         }
-        *abort_flag = 0;
+    }
+    if (lane == 0) {
+        for (int i = 0; i < R; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
     }
     __syncthreads();
-
-    if (warp == kConsumerWarps) {
-        // ------------------------------------------------------------ producer
-        constexpr int BR = TOK;  // rows per box: a stage never spans two blocks (TOK <= block_size)
-        const int32_t* trow = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
-        const int blk0 = t_begin / bs;
-        const int nblk = (t_end + bs - 1) / bs - blk0;  // table entries this partition reads
-        if (lane == 0) {
-            prefetch_tensormap(&kmap);
-            prefetch_tensormap(&vmap);
+    if (warp == 0) {  // exclusive scan of the full-partition counts; s_cum[S] = total
+        const int per = (S + 31) / 32;
+        const int b = min(S, lane * per), e = min(S, b + per);
+        int local = 0;
+        for (int i = b; i < e; ++i) local += s_cum[i];
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(FULL, incl, o);
+            if (lane >= o) incl += y;
         }
-        int tab = -1, tab_chunk = -1;
-        int issued = 0;
-        for (int st = 0; st < nst; ++st) {
-            const int slot = st % NS;
-            const int t0 = t_begin + st * TOK;
-            const int e = t0 / bs - blk0;  // warp-uniform
-            if ((e >> 5) != tab_chunk) {
-                tab_chunk = e >> 5;
-                const int idx = (tab_chunk << 5) + lane;
-                tab = idx < nblk ? __ldg(trow + blk0 + idx) : -1;
-            }
-            const int phys = __shfl_sync(0xffffffffu, tab, e & 31);
-            bool ok = true;
-            if (lane == 0 && st >= NS) ok = mbar_wait(&empty[slot], ((st / NS) - 1) & 1);
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok || *abort_flag) {
-                if (lane == 0) {
-                    if (!ok) report(a.err_word, PA_DEVERR_TIMEOUT);
-                    *abort_flag = 1;
-                }
-                break;
-            }
-            if (lane == 0) {
-                if (phys < 0 || phys >= a.num_blocks) {
-                    report(a.err_word, PA_DEVERR_TABLE_RANGE);
-                    bad[slot] = 1;
-                    mbar_arrive(&full[slot]);
-                } else {
-                    bad[slot] = 0;
-                    const int row = phys * bs + (t0 % bs);
-                    mbar_arrive_expect_tx(&full[slot], 2u * BR * D * 2);
-                    tma_load_3d(smem + Lay::kOffK + slot * Lay::kTileBytes, &kmap, 0, kv_head, row, &full[slot]);
-                    tma_load_3d(smem + Lay::kOffV + slot * Lay::kTileBytes, &vmap, 0, kv_head, row, &full[slot]);
-                }
-            }
-            issued = st + 1;
+        int run = incl - local;
+        for (int i = b; i < e; ++i) {
+            const int v = s_cum[i];
+            s_cum[i] = run;
+            run += v;
         }
-        // Do not leave while copies into this CTA's shared memory are in flight.
-        if (lane == 0) {
-            for (int st = issued > NS ? issued - NS : 0; st < issued; ++st)
-                if (!mbar_wait(&full[st % NS], (st / NS) & 1)) report(a.err_word, PA_DEVERR_TIMEOUT);
-        }
-        return;
+        if (lane == 31) s_cum[S] = incl;
     }
+    // bitonic sort of the last-partition keys: (P - size) ascending, then s
+    for (int k = 2; k <= spow; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < spow; i += blockDim.x) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const uint32_t x = s_key[i], y = s_key[ixj];
+                    if ((x > y) == ((i & k) == 0)) {
+                        s_key[i] = y;
+                        s_key[ixj] = x;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    __syncthreads();
 
-    // ---------------------------------------------------------------- consumers
+    // ------------------------------------------------------------ warp engine
     const int c = lane % CH;  // 16-byte chunk of the row this lane reads
     const int r = lane / CH;  // row within a warp-wide load
-    float qv[8];
-    {
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(a.q + sh * D) + c);
+    int32_t* claim_ctr = a.sched;
+
+    auto claim = [&]() -> int { return lane == 0 ? atomicAdd(claim_ctr, 1) : 0; };
+    auto load_q = [&](const Unit& U, float2 (&qv)[4]) {
+        if (U.kind != kUnitNormal) return;
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(a.q + ((int64_t)U.s * H + U.h) * D) + c);
         widen8<Tag>(w, qv);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) qv[k] *= a.scale_log2;
-    }
+        for (int k = 0; k < 4; ++k) {
+            qv[k].x *= a.scale_log2;
+            qv[k].y *= a.scale_log2;
+        }
+    };
+    auto load_tab = [&](const Unit& U, int chunk) -> int {
+        const int idx = chunk * 32 + lane;
+        return (U.kind == kUnitNormal && idx < U.nblk)
+                   ? __ldg(a.block_tables + (int64_t)U.s * a.max_blocks_per_seq + U.blk0 + idx)
+                   : -1;
+    };
+
+    // current unit C (being consumed), next unit N, and a pending raw claim
+    Unit C = decode_unit(__shfl_sync(FULL, claim(), 0), a, s_cum, s_key, s_len, TOK);
+    Unit N = decode_unit(__shfl_sync(FULL, claim(), 0), a, s_cum, s_key, s_len, TOK);
+    int pend = claim();
+    float2 qc[4], qn[4];
+    load_q(C, qc);
+    load_q(N, qn);
+    int ntab0 = load_tab(N, 0), ntab1 = load_tab(N, 1);
+    // issue cursor: in C (in_next = false) or N; its rolling table chunk pair
+    bool in_next = false;
+    int ist = 0;
+    int ichunk = 0, itab_cur = load_tab(C, 0), itab_nxt = load_tab(C, 1);
+    uint32_t issued = 0, consumed = 0;
+    uint32_t badmask = 0;  // slots whose stage was dropped for a bad table entry
+    bool aborted = false;
+
+    // softmax state of C
     float m = -INFINITY, lsum = 0.f;
-    float o[8];
+    float2 o[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) o[k] = 0.f;
+    for (int k = 0; k < 4; ++k) o[k] = make_float2(0.f, 0.f);
     bool poisoned = false;
+    int cst = 0;
 
-    for (int st = warp; st < nst; st += kConsumerWarps) {
-        const int slot = st % NS;
-        if (*abort_flag) break;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[slot], (st / NS) & 1));
-        if (!ok) {
+    auto issue_stage = [&](const Unit& I, int st) {
+        const int slot = issued % R;
+        const int t0 = I.t_begin + st * TOK;
+        const int br = a.box_rows;
+        const int first_e = t0 / bs - I.blk0;
+        while ((first_e >> 5) > ichunk) {  // roll the table window forward
+            ++ichunk;
+            itab_cur = itab_nxt;
+            itab_nxt = load_tab(I, ichunk + 1);
+        }
+        int phys[MAXSUB];
+        bool bad = false;
+        uint32_t tx = 0;
+#pragma unroll
+        for (int j = 0; j < MAXSUB; ++j) {
+            const int tj = t0 + j * br;
+            const bool use = j * br < TOK && tj < I.t_end;
+            const int e = tj / bs - I.blk0;
+            const int v = (e >> 5) == ichunk ? itab_cur : itab_nxt;
+            phys[j] = __shfl_sync(FULL, v, e & 31);
+            if (use) {
+                bad |= phys[j] < 0 || phys[j] >= a.num_blocks;
+                tx += 2u * br * D * 2;
+            }
+        }
+        uint8_t* dst = slots + slot * Lay::kSlotBytes;
+        if (bad) badmask |= 1u << slot;
+        if (lane == 0) {
+            if (bad) {
+                report(a.err_word, PA_DEVERR_TABLE_RANGE);
+                mbar_arrive(&bars[slot]);
+            } else {
+                fence_proxy_async_shared();  // our earlier reads of this slot come first
+                mbar_arrive_expect_tx(&bars[slot], tx);
+#pragma unroll
+                for (int j = 0; j < MAXSUB; ++j) {
+                    const int tj = t0 + j * br;
+                    if (j * br < TOK && tj < I.t_end) {
+                        const int row = phys[j] * bs + (tj % bs);
+                        tma_load_3d(dst + j * br * D * 2, &kmap, 0, I.kv_head, row, &bars[slot]);
+                        tma_load_3d(dst + Lay::kTileBytes + j * br * D * 2, &vmap, 0, I.kv_head, row, &bars[slot]);
+                    }
+                }
+            }
+        }
+        ++issued;
+    };
+
+    auto finish_unit = [&](const Unit& U) {
+        const int64_t sh = (int64_t)U.s * H + U.h;
+        if (U.kind == kUnitZero || U.kind == kUnitNaN) {
+            if (r == 0) {
+                const uint32_t w = U.kind == kUnitZero ? 0u : pack2<Tag>(__int_as_float(0x7fc00000),
+                                                                          __int_as_float(0x7fc00000));
+                reinterpret_cast<uint4*>(a.out + sh * D)[c] = make_uint4(w, w, w, w);
+            }
+            if (U.kind == kUnitNaN && lane == 0) report(a.err_word, PA_DEVERR_LEN_RANGE);
+            return;
+        }
+        // fold the RPI row groups; each token's p sits on DUP lanes
+#pragma unroll
+        for (int off = CH; off < 32; off <<= 1) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                o[k].x += __shfl_xor_sync(FULL, o[k].x, off);
+                o[k].y += __shfl_xor_sync(FULL, o[k].y, off);
+            }
+        }
+        float l = warp_sum(lsum) * (1.f / DUP);
+        if (__any_sync(FULL, poisoned)) l = __int_as_float(0x7fc00000);
+        if (U.np == 1) {
+            if (r == 0) {
+                const float inv = 1.f / l;
+                uint4 w;
+                w.x = pack2<Tag>(o[0].x * inv, o[0].y * inv);
+                w.y = pack2<Tag>(o[1].x * inv, o[1].y * inv);
+                w.z = pack2<Tag>(o[2].x * inv, o[2].y * inv);
+                w.w = pack2<Tag>(o[3].x * inv, o[3].y * inv);
+                reinterpret_cast<uint4*>(a.out + sh * D)[c] = w;
+            }
+        } else {
+            const int64_t pi = sh * a.num_partitions + U.p;
+            if (r == 0) {
+                float4* dst = reinterpret_cast<float4*>(a.ws_o + pi * D + c * 8);
+                dst[0] = make_float4(o[0].x, o[0].y, o[1].x, o[1].y);
+                dst[1] = make_float4(o[2].x, o[2].y, o[3].x, o[3].y);
+            }
             if (lane == 0) {
-                report(a.err_word, PA_DEVERR_TIMEOUT);
-                *abort_flag = 1;
-            }
-            break;
-        }
-        if (bad[slot]) {
-            poisoned = true;
-        } else {
-            const int ntok = min(TOK, t_end - (t_begin + st * TOK));
-            const uint8_t* kt = smem + Lay::kOffK + slot * Lay::kTileBytes;
-            const uint8_t* vt = smem + Lay::kOffV + slot * Lay::kTileBytes;
-            // scores: lane (c, r) forms the partial dot of row i*RPI + r over its chunk
-            float acc[NV];
-#pragma unroll
-            for (int i = 0; i < NV; ++i) {
-                const int row = i * RPI + r;
-                const uint4 w = *reinterpret_cast<const uint4*>(kt + (row * D + c * 8) * 2);
-                float kf[8];
-                widen8<Tag>(w, kf);
-                float d0 = 0.f;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) d0 = fmaf(qv[k], kf[k], d0);
-                acc[i] = d0;
-            }
-            // reduce-scatter over the CH lanes of a row: after it, lane c holds the
-            // full score of row group (c >> SH)
-#pragma unroll
-            for (int width = NV; width > 1; width >>= 1) {
-                const int half = width >> 1;
-                const int mask = half << SH;
-                const bool upper = (c & mask) != 0;
-#pragma unroll
-                for (int j = 0; j < half; ++j) {
-                    const float keep = upper ? acc[j + half] : acc[j];
-                    const float send = upper ? acc[j] : acc[j + half];
-                    acc[j] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
-                }
-            }
-            float x = acc[0];
-#pragma unroll
-            for (int mask = 1; mask < DUP; mask <<= 1) x += __shfl_xor_sync(0xffffffffu, x, mask);
-            const int tok = (c >> SH) * RPI + r;
-            if (tok >= ntok) x = -INFINITY;
-            const float m_new = fmaxf(m, warp_max(x));
-            const float alpha = exp2f(m - m_new);
-            const float p = exp2f(x - m_new);
-            lsum = lsum * alpha + p;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) o[k] *= alpha;
-            m = m_new;
-            // o += p_row * V_row for the rows this lane covers
-#pragma unroll
-            for (int i = 0; i < NV; ++i) {
-                const int row = i * RPI + r;
-                const float pr = __shfl_sync(0xffffffffu, p, r * CH + (i << SH));
-                if (row < ntok) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(vt + (row * D + c * 8) * 2);
-                    float vf[8];
-                    widen8<Tag>(w, vf);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) o[k] = fmaf(pr, vf[k], o[k]);
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[slot]);
-    }
-
-    // warp state: fold the RPI row groups, then the DUP copies of each p in lsum
-#pragma unroll
-    for (int off = CH; off < 32; off <<= 1) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) o[k] += __shfl_xor_sync(0xffffffffu, o[k], off);
-    }
-    lsum = warp_sum(lsum) * (1.f / DUP);
-    poisoned = __any_sync(0xffffffffu, poisoned);
-    if (r == 0) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) merge_o[warp * D + c * 8 + k] = o[k];
-    }
-    if (lane == 0) {
-        merge_m[warp] = m;
-        merge_l[warp] = poisoned ? __int_as_float(0x7fc00000) : lsum;
-    }
-    named_barrier(1, kConsumerWarps * 32);
-
-    const int tid = threadIdx.x;
-    if (tid < D) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge_m[w]);
-        float l = 0.f, acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-            const float mw = merge_m[w];
-            const float sc = mw == -INFINITY ? 0.f : exp2f(mw - M);
-            l = fmaf(merge_l[w], sc, l);
-            acc = fmaf(merge_o[w * D + tid], sc, acc);
-        }
-        if (nparts == 1) {
-            out_row[tid] = Tag::round1(acc / l);
-        } else {
-            const int64_t pi = sh * a.num_partitions + part;
-            a.ws_o[pi * D + tid] = acc;
-            if (tid == 0) {
-                a.ws_m[pi] = M;
+                a.ws_m[pi] = m;
                 a.ws_l[pi] = l;
             }
+        }
+    };
+
+    while (C.kind != kUnitNone && !aborted) {
+        if (C.kind != kUnitNormal || C.nst == 0) {
+            finish_unit(C);
+        } else {
+            // keep R stages in flight: C's remaining stages, then N's
+            while (issued - consumed < (uint32_t)R) {
+                if (!in_next) {
+                    if (ist < C.nst) {
+                        issue_stage(C, ist++);
+                        continue;
+                    }
+                    if (N.kind != kUnitNormal) break;
+                    in_next = true;
+                    ist = 0;
+                    ichunk = 0;
+                    itab_cur = ntab0;
+                    itab_nxt = ntab1;
+                }
+                if (ist < N.nst) issue_stage(N, ist++);
+                else break;
+            }
+            // consume one stage of C
+            const int slot = consumed % R;
+            const bool ok = __all_sync(FULL, mbar_wait(&bars[slot], (consumed / R) & 1));
+            if (!ok) {
+                if (lane == 0) report(a.err_word, PA_DEVERR_TIMEOUT);
+                aborted = true;
+                break;
+            }
+            if ((badmask >> slot) & 1u) {
+                poisoned = true;
+                badmask &= ~(1u << slot);
+            } else {
+                const int ntok = min(TOK, C.t_end - (C.t_begin + cst * TOK));
+                const uint8_t* kt = slots + slot * Lay::kSlotBytes;
+                const uint8_t* vt = kt + Lay::kTileBytes;
+                float acc[NV];
+#pragma unroll
+                for (int i = 0; i < NV; ++i) {
+                    const int row = i * RPI + r;
+                    const uint4 w = *reinterpret_cast<const uint4*>(kt + (row * D + c * 8) * 2);
+                    float2 kf[4];
+                    widen8<Tag>(w, kf);
+                    float2 d2 = __fmul2_rn(qc[0], kf[0]);
+                    d2 = __ffma2_rn(qc[1], kf[1], d2);
+                    d2 = __ffma2_rn(qc[2], kf[2], d2);
+                    d2 = __ffma2_rn(qc[3], kf[3], d2);
+                    acc[i] = d2.x + d2.y;
+                }
+                // reduce-scatter over the CH lanes of a row: lane c ends up with
+                // the full score of row group (c >> SH)
+#pragma unroll
+                for (int width = NV; width > 1; width >>= 1) {
+                    const int half = width >> 1;
+                    const int mask = half << SH;
+                    const bool upper = (c & mask) != 0;
+#pragma unroll
+                    for (int j = 0; j < half; ++j) {
+                        const float keep = upper ? acc[j + half] : acc[j];
+                        const float send = upper ? acc[j] : acc[j + half];
+                        acc[j] = keep + __shfl_xor_sync(FULL, send, mask);
+                    }
+                }
+                float x = acc[0];
+#pragma unroll
+                for (int mask = 1; mask < DUP; mask <<= 1) x += __shfl_xor_sync(FULL, x, mask);
+                const int tok = (c >> SH) * RPI + r;
+                if (tok >= ntok) x = -INFINITY;
+                const float m_new = fmaxf(m, warp_max(x));
+                const float alpha = exp2f(m - m_new);
+                const float p = exp2f(x - m_new);
+                lsum = lsum * alpha + p;
+                const float2 al2 = make_float2(alpha, alpha);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) o[k] = __fmul2_rn(o[k], al2);
+                m = m_new;
+#pragma unroll
+                for (int i = 0; i < NV; ++i) {
+                    const int row = i * RPI + r;
+                    const float pr = __shfl_sync(FULL, p, r * CH + (i << SH));
+                    if (row < ntok) {
+                        const uint4 w = *reinterpret_cast<const uint4*>(vt + (row * D + c * 8) * 2);
+                        float2 vf[4];
+                        widen8<Tag>(w, vf);
+                        const float2 p2 = make_float2(pr, pr);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) o[k] = __ffma2_rn(p2, vf[k], o[k]);
+                    }
+                }
+            }
+            __syncwarp();
+            ++consumed;
+            if (++cst < C.nst) continue;
+            finish_unit(C);
+        }
+        // rotate: N becomes current; decode the pending claim as the new N
+        const bool issue_was_in_next = in_next;
+        C = N;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) qc[k] = qn[k];
+        N = decode_unit(__shfl_sync(FULL, pend, 0), a, s_cum, s_key, s_len, TOK);
+        load_q(N, qn);
+        ntab0 = load_tab(N, 0);
+        ntab1 = load_tab(N, 1);
+        if (N.kind != kUnitNone) pend = claim();
+        if (issue_was_in_next) {
+            in_next = false;  // the issue cursor already runs inside the new C
+        } else {
+            in_next = false;
+            ist = 0;
+            ichunk = 0;
+            itab_cur = load_tab(C, 0);
+            itab_nxt = load_tab(C, 1);
+        }
+        m = -INFINITY;
+        lsum = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) o[k] = make_float2(0.f, 0.f);
+        poisoned = false;
+        cst = 0;
+    }
+
+    // never leave with copies into shared memory in flight
+    for (uint32_t k = consumed; k < issued; ++k)
+        if (!__all_sync(FULL, mbar_wait(&bars[k % R], (k / R) & 1)) && lane == 0)
+            report(a.err_word, PA_DEVERR_TIMEOUT);
+    // the last warp of the launch to finish puts the claim counters back to zero
+    if (lane == 0) {
+        __threadfence();
+        const int total = (int)(gridDim.x * NW);
+        if (atomicAdd(a.sched + 1, 1) == total - 1) {
+            atomicExch(a.sched, 0);
+            atomicExch(a.sched + 1, 0);
+            __threadfence();
         }
     }
 }
@@ -369,7 +544,7 @@ __global__ void __launch_bounds__(D) paged_decode_merge_kernel(const DecodeArgs 
     float den = 0.f, acc = 0.f;
     const int i = threadIdx.x;
     for (int p = 0; p < nparts; ++p) {
-        const float w = exp2f(pm[p] - M);
+        const float w = pm[p] == -INFINITY ? 0.f : exp2f(pm[p] - M);
         den = fmaf(pl[p], w, den);
         acc = fmaf(po[(int64_t)p * D + i], w, acc);
     }
@@ -381,40 +556,65 @@ __global__ void __launch_bounds__(D) paged_decode_merge_kernel(const DecodeArgs 
 namespace {
 
 constexpr int kDefaultPartition = 512;
+constexpr size_t kSchedBytes = 256;
 
 int64_t num_partitions(int max_blocks_per_seq, int block_size, int ptok) {
     const int64_t max_len = (int64_t)max_blocks_per_seq * block_size;
     return max_len <= 0 ? 1 : (max_len + ptok - 1) / ptok;
 }
 
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
 size_t workspace_bytes_for(int64_t sh, int64_t P, int D) {
-    if (P <= 1) return 0;
-    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-    return up(sh * P * 4) * 2 + up(sh * P * D * 4);
+    if (P <= 1) return kSchedBytes;
+    return kSchedBytes + up256(sh * P * 4) * 2 + up256(sh * P * D * 4);
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
 }
 
 template <class Tag, int D>
-int launch_mha(DecodeArgs args, int num_seqs, const void* k_cache, const void* v_cache, int num_kv_heads,
-               cudaStream_t stream) {
-    constexpr int TOK = 16;
-    constexpr int NS = 8;
-    using Lay = MhaLayout<D, TOK, NS>;
+int launch_decode(DecodeArgs args, const void* k_cache, const void* v_cache, int num_kv_heads,
+                  cudaStream_t stream) {
+    constexpr int TOK = D == 128 ? 16 : 32;
+    constexpr int NW = 12;
+    constexpr int R = 2;
+    using Lay = Layout<D, TOK, NW, R>;
     static std::atomic<uint64_t> smem_done{0};
-    auto kernel = paged_decode_mha_kernel<Tag, D, TOK, NS>;
+    auto kernel = paged_decode_kernel<Tag, D, TOK, NW, R>;
     if (ensure_smem_limit(kernel, Lay::kAlloc, smem_done) != cudaSuccess) return PA_ERR_CUDA;
-    if (TOK > args.block_size) return PA_ERR_UNSUPPORTED;
+    args.box_rows = TOK < args.block_size ? TOK : args.block_size;
     const int64_t total_tokens = (int64_t)args.num_blocks * args.block_size;
     CUtensorMap kmap, vmap;
-    if (!encode_cache_map(&kmap, k_cache, D, num_kv_heads, total_tokens, TOK) ||
-        !encode_cache_map(&vmap, v_cache, D, num_kv_heads, total_tokens, TOK))
+    if (!encode_cache_map(&kmap, k_cache, D, num_kv_heads, total_tokens, args.box_rows) ||
+        !encode_cache_map(&vmap, v_cache, D, num_kv_heads, total_tokens, args.box_rows))
         return PA_ERR_CUDA;
-    const int64_t gx = (int64_t)args.num_heads * args.num_partitions;
-    dim3 grid((unsigned)gx, (unsigned)num_seqs);
-    kernel<<<grid, kDecodeThreads, Lay::kAlloc, stream>>>(args, kmap, vmap);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-    if (args.num_partitions > 1) {
-        paged_decode_merge_kernel<Tag, D><<<(unsigned)((int64_t)num_seqs * args.num_heads), D, 0, stream>>>(args);
+    const int sms = sm_count();
+    if (sms <= 0) return PA_ERR_CUDA;
+    const int total_seqs = args.num_seqs;
+    for (int s0 = 0; s0 < total_seqs; s0 += kMaxSeqsPerLaunch) {
+        DecodeArgs c = args;
+        c.num_seqs = total_seqs - s0 < kMaxSeqsPerLaunch ? total_seqs - s0 : kMaxSeqsPerLaunch;
+        const int64_t shoff = (int64_t)s0 * args.num_heads;
+        c.q += shoff * D;
+        c.out += shoff * D;
+        c.block_tables += (int64_t)s0 * args.max_blocks_per_seq;
+        c.context_lens += s0;
+        if (args.num_partitions > 1) {
+            c.ws_m += shoff * args.num_partitions;
+            c.ws_l += shoff * args.num_partitions;
+            c.ws_o += shoff * args.num_partitions * D;
+        }
+        kernel<<<sms, NW * 32, Lay::kAlloc, stream>>>(c, kmap, vmap);
         if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+        if (args.num_partitions > 1) {
+            paged_decode_merge_kernel<Tag, D><<<(unsigned)((int64_t)c.num_seqs * args.num_heads), D, 0, stream>>>(c);
+            if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+        }
     }
     return PA_OK;
 }
@@ -432,7 +632,8 @@ extern "C" int pa_decode_partition_tokens(int num_seqs, int num_heads, int num_k
 extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                            int block_size, int max_blocks_per_seq, int partition_tokens) {
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
-        max_blocks_per_seq < 0 || partition_tokens < 0 || partition_tokens % 64 != 0)
+        max_blocks_per_seq < 0 || partition_tokens < 0 || partition_tokens % 64 != 0 ||
+        partition_tokens > pa::kMaxPartitionTokens)
         return 0;
     const int ptok = partition_tokens > 0
                          ? partition_tokens
@@ -449,43 +650,48 @@ extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache
                          int32_t* err_word, void* stream) {
     using namespace pa;
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
-        num_blocks <= 0 || max_blocks_per_seq <= 0 || partition_tokens < 0 || partition_tokens % 64 != 0)
+        num_blocks <= 0 || max_blocks_per_seq <= 0 || partition_tokens < 0 || partition_tokens % 64 != 0 ||
+        partition_tokens > kMaxPartitionTokens)
         return PA_ERR_INVALID_ARG;
     if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
     if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
     if (block_size != 16 && block_size != 32 && block_size != 64) return PA_ERR_UNSUPPORTED;
-    if ((int64_t)num_blocks * block_size > INT32_MAX ||
-        (int64_t)max_blocks_per_seq * block_size > INT32_MAX || num_seqs > 65535)
+    if ((int64_t)num_blocks * block_size > INT32_MAX || (int64_t)max_blocks_per_seq * block_size > INT32_MAX)
         return PA_ERR_UNSUPPORTED;
     if (num_seqs == 0) return PA_OK;
-    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PA_ERR_INVALID_ARG;
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out || !workspace)
+        return PA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
-        !aligned4(block_tables) || !aligned4(context_lens) || (err_word && !aligned4(err_word)))
+        !aligned16(workspace) || !aligned4(block_tables) || !aligned4(context_lens) ||
+        (err_word && !aligned4(err_word)))
         return PA_ERR_INVALID_ARG;
     const int ptok = partition_tokens > 0
                          ? partition_tokens
                          : pa_decode_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                                       max_blocks_per_seq);
     const int64_t P = num_partitions(max_blocks_per_seq, block_size, ptok);
-    if ((int64_t)num_heads * P > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    // claim indices of one launch must fit in int32
+    const int64_t chunk = num_seqs < kMaxSeqsPerLaunch ? num_seqs : kMaxSeqsPerLaunch;
+    if ((int64_t)num_heads * chunk * (P + 1) > INT32_MAX) return PA_ERR_UNSUPPORTED;
     const int64_t SH = (int64_t)num_seqs * num_heads;
     const size_t need = workspace_bytes_for(SH, P, head_dim);
-    if (need > 0 && (!workspace || !aligned16(workspace) || workspace_bytes < need)) return PA_ERR_INVALID_ARG;
+    if (workspace_bytes < need) return PA_ERR_INVALID_ARG;
 
     DecodeArgs args{};
     args.q = static_cast<const uint16_t*>(q);
     args.out = static_cast<uint16_t*>(out);
     args.block_tables = block_tables;
     args.context_lens = context_lens;
-    if (need > 0) {
-        auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-        uint8_t* w = static_cast<uint8_t*>(workspace);
-        args.ws_m = reinterpret_cast<float*>(w);
-        args.ws_l = reinterpret_cast<float*>(w + up(SH * P * 4));
-        args.ws_o = reinterpret_cast<float*>(w + 2 * up(SH * P * 4));
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    args.sched = reinterpret_cast<int32_t*>(w);
+    if (P > 1) {
+        args.ws_m = reinterpret_cast<float*>(w + kSchedBytes);
+        args.ws_l = reinterpret_cast<float*>(w + kSchedBytes + up256(SH * P * 4));
+        args.ws_o = reinterpret_cast<float*>(w + kSchedBytes + 2 * up256(SH * P * 4));
     }
     args.err_word = err_word;
     args.scale_log2 = scale * 1.4426950408889634f;
+    args.num_seqs = num_seqs;
     args.num_heads = num_heads;
     args.group = num_heads / num_kv_heads;
     args.block_size = block_size;
@@ -495,8 +701,8 @@ extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache
     args.num_partitions = (int)P;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (head_dim == 128)
-        return dtype == PA_F16 ? launch_mha<F16Tag, 128>(args, num_seqs, k_cache, v_cache, num_kv_heads, st)
-                               : launch_mha<BF16Tag, 128>(args, num_seqs, k_cache, v_cache, num_kv_heads, st);
-    return dtype == PA_F16 ? launch_mha<F16Tag, 64>(args, num_seqs, k_cache, v_cache, num_kv_heads, st)
-                           : launch_mha<BF16Tag, 64>(args, num_seqs, k_cache, v_cache, num_kv_heads, st);
+        return dtype == PA_F16 ? launch_decode<F16Tag, 128>(args, k_cache, v_cache, num_kv_heads, st)
+                               : launch_decode<BF16Tag, 128>(args, k_cache, v_cache, num_kv_heads, st);
+    return dtype == PA_F16 ? launch_decode<F16Tag, 64>(args, k_cache, v_cache, num_kv_heads, st)
+                           : launch_decode<BF16Tag, 64>(args, k_cache, v_cache, num_kv_heads, st);
 }

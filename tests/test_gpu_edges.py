@@ -129,8 +129,10 @@ def test_empty_batch_and_binding_checks():
     ln = torch.zeros(0, dtype=torch.int32, device="cuda")
     pa.pa_decode(q, kc, kc, tb, ln, 0.125, 4, torch.empty_like(q))
     q1 = torch.zeros(1, 4, 64, dtype=torch.bfloat16, device="cuda")
-    with pytest.raises(TypeError):
-        pa.pa_decode(q1, kc, kc, tb[:1], ln[:1], 0.125, 4, torch.empty_like(q1))
+    tb1 = torch.zeros(1, 2, dtype=torch.int32, device="cuda")
+    ln1 = torch.ones(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(TypeError):                       # q bf16, caches fp16
+        pa.pa_decode(q1, kc, kc, tb1, ln1, 0.125, 4, torch.empty_like(q1))
     with pytest.raises(pa.PAError) as e:
         pa.pa_decode(torch.zeros(1, 4, 96, dtype=torch.float16, device="cuda"),
                      torch.zeros(4, 16, 4, 96, dtype=torch.float16, device="cuda"),
