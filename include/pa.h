@@ -151,6 +151,35 @@ int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int
               int dtype, int partition_tokens, void* workspace, size_t workspace_bytes, int32_t* err_word,
               void* stream);
 
+/*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device memory.
+ *
+ * No counterpart on the pages: this is an interface convenience of the library,
+ * not a step of the method.  Some callers cannot call cudaMalloc (or any routine
+ * that allocates) where they run attention: code running inside a device memory
+ * allocator or pool, which would re-enter itself; plug-in hosts that pass in only
+ * the tensors they own; launch sequences that must keep the device memory
+ * footprint fixed.  This call takes pa_decode's workspace from a fixed array in the
+ * library's own device memory instead, so it allocates nothing.
+ *
+ * Arguments, results and errors as pa_decode, without workspace/workspace_bytes.
+ *   - The array holds PA_DECODE_NOALLOC_SCRATCH_BYTES on every GPU that loads the
+ *     library, until the process exits.  Sizes whose pa_decode_workspace_size(...)
+ *     exceeds it are refused with PA_ERR_UNSUPPORTED (use pa_decode with a
+ *     workspace of your own for those).
+ *   - The first call on a device looks up the array's device address on that
+ *     device (a one-time set-up); make that first call before any stream capture.
+ *   - Every call on a device uses the same array, which keeps the previous call's
+ *     contents; the call clears the part that must start at zero.  Calls whose
+ *     work may overlap on the GPU (several streams or host threads) race on the
+ *     array and give wrong results: serialise them, e.g. on one stream.
+ */
+#define PA_DECODE_NOALLOC_SCRATCH_BYTES (64u << 20)
+int pa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      const int32_t* context_lens, float scale, int num_kv_heads, void* out, int num_seqs,
+                      int num_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                      int dtype, int partition_tokens, int32_t* err_word, void* stream);
+
 /* ---------------------------------------------------------- host allocator */
 
 /*

@@ -44,6 +44,8 @@ _sig("pa_decode_partition_tokens", _i32, _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_decode_workspace_size", ctypes.c_size_t, _i32, _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_decode", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
      _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
+_sig("pa_decode_noalloc", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32, _i32, _i32, _i32, _i32,
+     _i32, _i32, _i32, _vp, _vp)
 _sig("pa_allocator_create", _vp, _i32, _i32p)
 _sig("pa_allocator_destroy", None, _vp)
 _sig("pa_num_required_blocks", _i32, _i32, _i32)
@@ -165,6 +167,30 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_hea
                         s, h, d, bs, nb, mb, dt, int(partition_tokens), ws_ptr, ws_bytes,
                         _dev(err_word, "err_word", torch.int32), _stream(stream, q))
     _check(st, "pa_decode")
+    return out
+
+
+def pa_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out,
+                      partition_tokens=0, err_word=None, stream=None):
+    """pa_decode with its workspace taken from the library's fixed device array
+    (for callers that cannot allocate device memory).  Returns ``out``."""
+    import torch
+    s, h, d = q.shape
+    nb, bs, hk, d2 = k_cache.shape
+    if hk != num_kv_heads or d2 != d or v_cache.shape != k_cache.shape or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [S, MB] and context_lens [S]")
+    dt = _dtype_code(q)
+    for t in (k_cache, v_cache, out):
+        if t.dtype != q.dtype:
+            raise TypeError("q, the caches and out must share one dtype")
+    st = _lib.pa_decode_noalloc(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                _dev(block_tables, "block_tables", torch.int32),
+                                _dev(context_lens, "context_lens", torch.int32), float(scale), hk,
+                                _dev(out, "out"), s, h, d, bs, nb, block_tables.shape[1], dt,
+                                int(partition_tokens), _dev(err_word, "err_word", torch.int32), _stream(stream, q))
+    _check(st, "pa_decode_noalloc")
     return out
 
 
