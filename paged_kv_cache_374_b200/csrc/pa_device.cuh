@@ -38,6 +38,14 @@ struct BF16Tag {
     }
 };
 
+// 2^x by the hardware's approximate base-2 exponential (MUFU), subnormal
+// results flushed to zero; exp2(-inf) = 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ------------------------------------------------------------------- error word
 
 __device__ __forceinline__ void report(int32_t* err_word, int bits) {

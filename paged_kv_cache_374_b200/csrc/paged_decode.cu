@@ -40,6 +40,23 @@
 #include "pa_device.cuh"
 #include "pa_host.h"
 
+// Tile configuration (compile-time; the defaults are the tuned ones).
+#ifndef PA_DECODE_WARPS
+#define PA_DECODE_WARPS 12       // warps (streaming engines) per CTA, one CTA per SM
+#endif
+#ifndef PA_DECODE_SLOTS
+#define PA_DECODE_SLOTS 2        // shared-memory slots per warp
+#endif
+#ifndef PA_DECODE_TOK128
+#define PA_DECODE_TOK128 16      // tokens per slot at head_dim 128
+#endif
+#ifndef PA_DECODE_TOK64
+#define PA_DECODE_TOK64 32       // tokens per slot at head_dim 64
+#endif
+#ifndef PA_DECODE_PARTITION
+#define PA_DECODE_PARTITION 256  // default context partition, tokens
+#endif
+
 namespace pa {
 
 constexpr int kMaxSeqsPerLaunch = 1024;   // sequences scheduled by one K2 launch
@@ -164,13 +181,17 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
                                                                   const __grid_constant__ CUtensorMap kmap,
                                                                   const __grid_constant__ CUtensorMap vmap) {
     using Lay = Layout<D, TOK, NW, R>;
-    constexpr int CH = D / 8;       // 16-byte chunks per token row
-    constexpr int RPI = 32 / CH;    // token rows covered by one warp-wide 16-byte load
-    constexpr int NV = TOK / RPI;   // row groups per stage (values each lane reduces)
-    static_assert(NV >= 1 && NV <= CH && CH % NV == 0, "stage shape");
-    constexpr int DUP = CH / NV;    // lanes that end up holding the same token's score
-    constexpr int SH = DUP == 1 ? 0 : DUP == 2 ? 1 : DUP == 4 ? 2 : DUP == 8 ? 3 : 4;
-    constexpr int MAXSUB = TOK / 16;  // TMA boxes per tile (box_rows >= 16)
+    // Lane layout for a stage of TOK tokens held as swizzled 128-byte half rows:
+    // lane = c * 8 + r.  Lane (c, r) owns dims [c*DL, (c+1)*DL) and token rows
+    // r, r + 8, ... of the stage, so a row's dot product is split over the 4 lanes
+    // with the same r (lanes r, r+8, r+16, r+24).
+    constexpr int DL = D / 4;          // dims per lane
+    constexpr int NCH = DL / 8;        // 16-byte chunks per lane per row
+    constexpr int NROW = TOK / 8;      // rows per lane per stage
+    static_assert(NROW == 1 || NROW == 2 || NROW == 4, "stage shape");
+    constexpr int DUP = 4 / NROW;      // lanes that end up holding one token's score
+    constexpr int HALF_BYTES = TOK * 128;   // one 64-dim half tile
+    constexpr int MAXSUB = TOK / 8 > 2 ? 2 : 1;  // TMA boxes per half tile (box_rows >= TOK/2)
     constexpr unsigned FULL = 0xffffffffu;
 
     extern __shared__ uint8_t smem_raw[];
@@ -248,19 +269,32 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
     __syncthreads();
 
     // ------------------------------------------------------------ warp engine
-    const int c = lane % CH;  // 16-byte chunk of the row this lane reads
-    const int r = lane / CH;  // row within a warp-wide load
+    const int r = lane & 7;
+    const int c = lane >> 3;
+    // shared-memory offset of this lane's chunk j of row (i*8 + r) in a K or V tile:
+    // half tile of the lane's dims, the row, and the swizzled 16-byte chunk
+    const int lane_half = (D == 128) ? (c >> 1) : 0;
+    const int chunk0 = (D == 128) ? (c & 1) * 4 : c * 2;
+    int swz[NCH];
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) swz[j] = lane_half * HALF_BYTES + r * 128 + (((chunk0 + j) ^ r) << 4);
     int32_t* claim_ctr = a.sched;
 
     auto claim = [&]() -> int { return lane == 0 ? atomicAdd(claim_ctr, 1) : 0; };
-    auto load_q = [&](const Unit& U, float2 (&qv)[4]) {
+    // q of a unit: fetched as raw 16-bit values, widened and pre-scaled on use
+    auto fetch_q = [&](const Unit& U, uint4 (&raw)[NCH]) {
         if (U.kind != kUnitNormal) return;
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(a.q + ((int64_t)U.s * H + U.h) * D) + c);
-        widen8<Tag>(w, qv);
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)U.s * H + U.h) * D + c * DL);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            qv[k].x *= a.scale_log2;
-            qv[k].y *= a.scale_log2;
+        for (int j = 0; j < NCH; ++j) raw[j] = __ldg(src + j);
+    };
+    auto widen_q = [&](const uint4 (&raw)[NCH], float2 (&qv)[DL / 2]) {
+#pragma unroll
+        for (int j = 0; j < NCH; ++j) {
+            float2 f[4];
+            widen8<Tag>(raw[j], f);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) qv[j * 4 + k] = make_float2(f[k].x * a.scale_log2, f[k].y * a.scale_log2);
         }
     };
     auto load_tab = [&](const Unit& U, int chunk) -> int {
@@ -274,9 +308,14 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
     Unit C = decode_unit(__shfl_sync(FULL, claim(), 0), a, s_cum, s_key, s_len, TOK);
     Unit N = decode_unit(__shfl_sync(FULL, claim(), 0), a, s_cum, s_key, s_len, TOK);
     int pend = claim();
-    float2 qc[4], qn[4];
-    load_q(C, qc);
-    load_q(N, qn);
+    float2 qc[DL / 2];
+    uint4 qn[NCH];
+    {
+        uint4 q0[NCH];
+        fetch_q(C, q0);
+        widen_q(q0, qc);
+    }
+    fetch_q(N, qn);
     int ntab0 = load_tab(N, 0), ntab1 = load_tab(N, 1);
     // issue cursor: in C (in_next = false) or N; its rolling table chunk pair
     bool in_next = false;
@@ -286,11 +325,11 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
     uint32_t badmask = 0;  // slots whose stage was dropped for a bad table entry
     bool aborted = false;
 
-    // softmax state of C
+    // softmax state of C (m is warp-uniform, base-2 units)
     float m = -INFINITY, lsum = 0.f;
-    float2 o[4];
+    float2 o[DL / 2];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) o[k] = make_float2(0.f, 0.f);
+    for (int k = 0; k < DL / 2; ++k) o[k] = make_float2(0.f, 0.f);
     bool poisoned = false;
     int cst = 0;
 
@@ -333,8 +372,12 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
                     const int tj = t0 + j * br;
                     if (j * br < TOK && tj < I.t_end) {
                         const int row = phys[j] * bs + (tj % bs);
-                        tma_load_3d(dst + j * br * D * 2, &kmap, 0, I.kv_head, row, &bars[slot]);
-                        tma_load_3d(dst + Lay::kTileBytes + j * br * D * 2, &vmap, 0, I.kv_head, row, &bars[slot]);
+#pragma unroll
+                        for (int hh = 0; hh < D / 64; ++hh) {
+                            uint8_t* kd = dst + hh * HALF_BYTES + j * br * 128;
+                            tma_load_3d(kd, &kmap, hh * 64, I.kv_head, row, &bars[slot]);
+                            tma_load_3d(kd + Lay::kTileBytes, &vmap, hh * 64, I.kv_head, row, &bars[slot]);
+                        }
                     }
                 }
             }
@@ -345,19 +388,19 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
     auto finish_unit = [&](const Unit& U) {
         const int64_t sh = (int64_t)U.s * H + U.h;
         if (U.kind == kUnitZero || U.kind == kUnitNaN) {
-            if (r == 0) {
+            if (lane < D / 8) {
                 const uint32_t w = U.kind == kUnitZero ? 0u : pack2<Tag>(__int_as_float(0x7fc00000),
                                                                           __int_as_float(0x7fc00000));
-                reinterpret_cast<uint4*>(a.out + sh * D)[c] = make_uint4(w, w, w, w);
+                reinterpret_cast<uint4*>(a.out + sh * D)[lane] = make_uint4(w, w, w, w);
             }
             if (U.kind == kUnitNaN && lane == 0) report(a.err_word, PA_DEVERR_LEN_RANGE);
             return;
         }
-        // fold the RPI row groups; each token's p sits on DUP lanes
+        // fold the 8 row classes r; each token's p sits on DUP lanes
 #pragma unroll
-        for (int off = CH; off < 32; off <<= 1) {
+        for (int off = 1; off < 8; off <<= 1) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < DL / 2; ++k) {
                 o[k].x += __shfl_xor_sync(FULL, o[k].x, off);
                 o[k].y += __shfl_xor_sync(FULL, o[k].y, off);
             }
@@ -367,19 +410,24 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
         if (U.np == 1) {
             if (r == 0) {
                 const float inv = 1.f / l;
-                uint4 w;
-                w.x = pack2<Tag>(o[0].x * inv, o[0].y * inv);
-                w.y = pack2<Tag>(o[1].x * inv, o[1].y * inv);
-                w.z = pack2<Tag>(o[2].x * inv, o[2].y * inv);
-                w.w = pack2<Tag>(o[3].x * inv, o[3].y * inv);
-                reinterpret_cast<uint4*>(a.out + sh * D)[c] = w;
+                uint4* dst = reinterpret_cast<uint4*>(a.out + sh * D + c * DL);
+#pragma unroll
+                for (int j = 0; j < NCH; ++j) {
+                    uint4 w;
+                    w.x = pack2<Tag>(o[j * 4 + 0].x * inv, o[j * 4 + 0].y * inv);
+                    w.y = pack2<Tag>(o[j * 4 + 1].x * inv, o[j * 4 + 1].y * inv);
+                    w.z = pack2<Tag>(o[j * 4 + 2].x * inv, o[j * 4 + 2].y * inv);
+                    w.w = pack2<Tag>(o[j * 4 + 3].x * inv, o[j * 4 + 3].y * inv);
+                    dst[j] = w;
+                }
             }
         } else {
             const int64_t pi = sh * a.num_partitions + U.p;
             if (r == 0) {
-                float4* dst = reinterpret_cast<float4*>(a.ws_o + pi * D + c * 8);
-                dst[0] = make_float4(o[0].x, o[0].y, o[1].x, o[1].y);
-                dst[1] = make_float4(o[2].x, o[2].y, o[3].x, o[3].y);
+                float4* dst = reinterpret_cast<float4*>(a.ws_o + pi * D + c * DL);
+#pragma unroll
+                for (int k = 0; k < DL / 4; ++k)
+                    dst[k] = make_float4(o[2 * k].x, o[2 * k].y, o[2 * k + 1].x, o[2 * k + 1].y);
             }
             if (lane == 0) {
                 a.ws_m[pi] = m;
@@ -424,26 +472,27 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
                 const int ntok = min(TOK, C.t_end - (C.t_begin + cst * TOK));
                 const uint8_t* kt = slots + slot * Lay::kSlotBytes;
                 const uint8_t* vt = kt + Lay::kTileBytes;
-                float acc[NV];
+                // partial dot products of rows i*8 + r over this lane's dims
+                float acc[NROW];
 #pragma unroll
-                for (int i = 0; i < NV; ++i) {
-                    const int row = i * RPI + r;
-                    const uint4 w = *reinterpret_cast<const uint4*>(kt + (row * D + c * 8) * 2);
-                    float2 kf[4];
-                    widen8<Tag>(w, kf);
-                    float2 d2 = __fmul2_rn(qc[0], kf[0]);
-                    d2 = __ffma2_rn(qc[1], kf[1], d2);
-                    d2 = __ffma2_rn(qc[2], kf[2], d2);
-                    d2 = __ffma2_rn(qc[3], kf[3], d2);
+                for (int i = 0; i < NROW; ++i) {
+                    float2 d2 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int j = 0; j < NCH; ++j) {
+                        const uint4 w = *reinterpret_cast<const uint4*>(kt + i * 1024 + swz[j]);
+                        float2 kf[4];
+                        widen8<Tag>(w, kf);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) d2 = __ffma2_rn(qc[j * 4 + k], kf[k], d2);
+                    }
                     acc[i] = d2.x + d2.y;
                 }
-                // reduce-scatter over the CH lanes of a row: lane c ends up with
-                // the full score of row group (c >> SH)
+                // reduce over the 4 lanes of a row (lane bits 4 and 3), scattering
+                // the NROW rows so that lane c keeps row group g(c)
 #pragma unroll
-                for (int width = NV; width > 1; width >>= 1) {
+                for (int width = NROW, mask = 16; width > 1; width >>= 1, mask >>= 1) {
                     const int half = width >> 1;
-                    const int mask = half << SH;
-                    const bool upper = (c & mask) != 0;
+                    const bool upper = (lane & mask) != 0;
 #pragma unroll
                     for (int j = 0; j < half; ++j) {
                         const float keep = upper ? acc[j + half] : acc[j];
@@ -452,29 +501,41 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
                     }
                 }
                 float x = acc[0];
+                if (NROW == 1) {
+                    x += __shfl_xor_sync(FULL, x, 16);
+                    x += __shfl_xor_sync(FULL, x, 8);
+                } else if (NROW == 2) {
+                    x += __shfl_xor_sync(FULL, x, 8);
+                }
+                const int g = NROW == 4 ? c : (NROW == 2 ? (c >> 1) : 0);
+                if (g * 8 + r >= ntok) x = -INFINITY;
+                // online softmax: the warp-wide max and the rescale of o are needed
+                // only when some score exceeds the running max
+                if (__any_sync(FULL, x > m)) {
+                    const float m_new = fmaxf(m, warp_max(x));
+                    const float alpha = fast_exp2(m - m_new);
+                    lsum *= alpha;
+                    const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll
-                for (int mask = 1; mask < DUP; mask <<= 1) x += __shfl_xor_sync(FULL, x, mask);
-                const int tok = (c >> SH) * RPI + r;
-                if (tok >= ntok) x = -INFINITY;
-                const float m_new = fmaxf(m, warp_max(x));
-                const float alpha = exp2f(m - m_new);
-                const float p = exp2f(x - m_new);
-                lsum = lsum * alpha + p;
-                const float2 al2 = make_float2(alpha, alpha);
+                    for (int k = 0; k < DL / 2; ++k) o[k] = __fmul2_rn(o[k], al2);
+                    m = m_new;
+                }
+                const float p = fast_exp2(x - m);
+                lsum += p;
+                // o += p_row * V_row for the rows this lane covers
 #pragma unroll
-                for (int k = 0; k < 4; ++k) o[k] = __fmul2_rn(o[k], al2);
-                m = m_new;
-#pragma unroll
-                for (int i = 0; i < NV; ++i) {
-                    const int row = i * RPI + r;
-                    const float pr = __shfl_sync(FULL, p, r * CH + (i << SH));
-                    if (row < ntok) {
-                        const uint4 w = *reinterpret_cast<const uint4*>(vt + (row * D + c * 8) * 2);
-                        float2 vf[4];
-                        widen8<Tag>(w, vf);
+                for (int i = 0; i < NROW; ++i) {
+                    const float pr = __shfl_sync(FULL, p, (i * DUP) * 8 + r);
+                    if (i * 8 + r < ntok) {
                         const float2 p2 = make_float2(pr, pr);
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) o[k] = __ffma2_rn(p2, vf[k], o[k]);
+                        for (int j = 0; j < NCH; ++j) {
+                            const uint4 w = *reinterpret_cast<const uint4*>(vt + i * 1024 + swz[j]);
+                            float2 vf[4];
+                            widen8<Tag>(w, vf);
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) o[j * 4 + k] = __ffma2_rn(p2, vf[k], o[j * 4 + k]);
+                        }
                     }
                 }
             }
@@ -486,10 +547,9 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
         // rotate: N becomes current; decode the pending claim as the new N
         const bool issue_was_in_next = in_next;
         C = N;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) qc[k] = qn[k];
+        if (C.kind == kUnitNormal) widen_q(qn, qc);
         N = decode_unit(__shfl_sync(FULL, pend, 0), a, s_cum, s_key, s_len, TOK);
-        load_q(N, qn);
+        fetch_q(N, qn);
         ntab0 = load_tab(N, 0);
         ntab1 = load_tab(N, 1);
         if (N.kind != kUnitNone) pend = claim();
@@ -505,7 +565,7 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
         m = -INFINITY;
         lsum = 0.f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) o[k] = make_float2(0.f, 0.f);
+        for (int k = 0; k < DL / 2; ++k) o[k] = make_float2(0.f, 0.f);
         poisoned = false;
         cst = 0;
     }
@@ -555,7 +615,7 @@ __global__ void __launch_bounds__(D) paged_decode_merge_kernel(const DecodeArgs 
 
 namespace {
 
-constexpr int kDefaultPartition = 512;
+constexpr int kDefaultPartition = PA_DECODE_PARTITION;
 constexpr size_t kSchedBytes = 256;
 
 int64_t num_partitions(int max_blocks_per_seq, int block_size, int ptok) {
@@ -580,9 +640,9 @@ int sm_count() {
 template <class Tag, int D>
 int launch_decode(DecodeArgs args, const void* k_cache, const void* v_cache, int num_kv_heads,
                   cudaStream_t stream) {
-    constexpr int TOK = D == 128 ? 16 : 32;
-    constexpr int NW = 12;
-    constexpr int R = 2;
+    constexpr int TOK = D == 128 ? PA_DECODE_TOK128 : PA_DECODE_TOK64;
+    constexpr int NW = PA_DECODE_WARPS;
+    constexpr int R = PA_DECODE_SLOTS;
     using Lay = Layout<D, TOK, NW, R>;
     static std::atomic<uint64_t> smem_done{0};
     auto kernel = paged_decode_kernel<Tag, D, TOK, NW, R>;
@@ -590,8 +650,8 @@ int launch_decode(DecodeArgs args, const void* k_cache, const void* v_cache, int
     args.box_rows = TOK < args.block_size ? TOK : args.block_size;
     const int64_t total_tokens = (int64_t)args.num_blocks * args.block_size;
     CUtensorMap kmap, vmap;
-    if (!encode_cache_map(&kmap, k_cache, D, num_kv_heads, total_tokens, args.box_rows) ||
-        !encode_cache_map(&vmap, v_cache, D, num_kv_heads, total_tokens, args.box_rows))
+    if (!encode_cache_map_swizzled(&kmap, k_cache, D, num_kv_heads, total_tokens, args.box_rows) ||
+        !encode_cache_map_swizzled(&vmap, v_cache, D, num_kv_heads, total_tokens, args.box_rows))
         return PA_ERR_CUDA;
     const int sms = sm_count();
     if (sms <= 0) return PA_ERR_CUDA;
