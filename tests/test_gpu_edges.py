@@ -35,7 +35,8 @@ def run_case(c, partition_tokens=0, err=None, tables=None, lens=None):
     return out
 
 
-SHAPES = list(itertools.product([64, 128], [16, 32, 64], [1, 2, 4, 8], [F16, BF16]))
+# groups 1 (CUDA-core path), 2..16 (tensor-core path), 32 (CUDA-core path again)
+SHAPES = list(itertools.product([64, 128], [16, 32, 64], [1, 2, 4, 8, 16], [F16, BF16])) + [(128, 16, 32, F16)]
 
 
 @pytest.mark.parametrize("d,bs,g,dtype", SHAPES)
