@@ -392,6 +392,8 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
     for (uint32_t k = consumed; k < issued; ++k)
         if (!__all_sync(kFullMask, mbar_wait(&bars[k % R], (k / R) & 1)) && lane == 0)
             report(a.err_word, PA_DEVERR_TIMEOUT);
+    // this warp writes nothing more: the merge kernel may be scheduled
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // the last warp of the launch to finish puts the claim counters back to zero
     if (lane == 0) {
         __threadfence();

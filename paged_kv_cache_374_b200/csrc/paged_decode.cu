@@ -34,6 +34,9 @@
 #ifndef PA_GQA_WARPS
 #define PA_GQA_WARPS 12          // GQA path: warps per CTA
 #endif
+#ifndef PA_GQA_SLOTS
+#define PA_GQA_SLOTS 2           // GQA path: shared-memory slots per warp
+#endif
 #ifndef PA_GQA_TOK
 #define PA_GQA_TOK 16            // GQA path: tokens per slot (a multiple of 16)
 #endif
@@ -43,10 +46,21 @@
 
 namespace pa {
 
-// K3: merge the partitions of each (s, h): M = max_p m_p,
-// out = sum_p o_p 2^(m_p - M) / sum_p l_p 2^(m_p - M)  (scores are in base-2 units).
+// K3: merge the partitions of each (s, h) (base-2 units):
+//   M = max_p m_p,  out = sum_p o_p 2^(m_p - M) / sum_p l_p 2^(m_p - M).
+// One CTA of 4 warps per (s, h): the max and the denominator are block-wide
+// reductions over the partitions; for the numerator each warp takes every 4th
+// partition and each lane 4 dims (16-byte loads), and the warps' sums meet in
+// shared memory.  Launched as a programmatic dependent of K2: its blocks may start
+// while K2's last CTAs finish and wait (griddepcontrol.wait) until K2's writes are
+// complete and visible.
+constexpr int kMergeThreads = 128;
+
 template <class Tag, int D>
-__global__ void __launch_bounds__(D) paged_decode_merge_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const DecodeArgs a) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ float s_red[kMergeThreads / 32];
+    __shared__ float4 s_acc[kMergeThreads / 32][D / 4];
     const int64_t sh = blockIdx.x;
     const int s = (int)(sh / a.num_heads);
     const int L = a.context_lens[s];
@@ -55,20 +69,57 @@ __global__ void __launch_bounds__(D) paged_decode_merge_kernel(const DecodeArgs 
     if (nparts <= 1) return;
     const float* pm = a.ws_m + sh * a.num_partitions;
     const float* pl = a.ws_l + sh * a.num_partitions;
-    const float* po = a.ws_o + sh * a.num_partitions * D;
-    float M = -INFINITY;
-    for (int p = 0; p < nparts; ++p) M = fmaxf(M, pm[p]);
-    float den = 0.f, acc = 0.f;
-    const int i = threadIdx.x;
-    for (int p = 0; p < nparts; ++p) {
-        const float w = pm[p] == -INFINITY ? 0.f : exp2f(pm[p] - M);
-        den = fmaf(pl[p], w, den);
-        acc = fmaf(po[(int64_t)p * D + i], w, acc);
-    }
-    a.out[sh * D + i] = Tag::round1(acc / den);
-}
+    const float4* po = reinterpret_cast<const float4*>(a.ws_o + sh * a.num_partitions * D);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-// ------------------------------------------------------------------------ host
+    float mx = -INFINITY;
+    for (int p = tid; p < nparts; p += kMergeThreads) mx = fmaxf(mx, pm[p]);
+    mx = warp_max(mx);
+    if (lane == 0) s_red[warp] = mx;
+    __syncthreads();
+    float M = s_red[0];
+#pragma unroll
+    for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, s_red[w]);
+    __syncthreads();
+
+    float den = 0.f;
+    for (int p = tid; p < nparts; p += kMergeThreads) den += pl[p] * (pm[p] == -INFINITY ? 0.f : exp2f(pm[p] - M));
+    den = warp_sum(den);
+    if (lane == 0) s_red[warp] = den;
+
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane < D / 4) {
+#pragma unroll 4
+        for (int p = warp; p < nparts; p += kMergeThreads / 32) {
+            const float w = pm[p] == -INFINITY ? 0.f : exp2f(pm[p] - M);
+            const float4 v = po[(int64_t)p * (D / 4) + lane];
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
+        s_acc[warp][lane] = acc;
+    }
+    __syncthreads();
+    if (tid < D / 4) {
+        float dsum = 0.f;
+        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kMergeThreads / 32; ++w) {
+            dsum += s_red[w];
+            const float4 v = s_acc[w][tid];
+            t.x += v.x;
+            t.y += v.y;
+            t.z += v.z;
+            t.w += v.w;
+        }
+        const float inv = 1.f / dsum;
+        uint2 packed;
+        packed.x = pack2<Tag>(t.x * inv, t.y * inv);
+        packed.y = pack2<Tag>(t.z * inv, t.w * inv);
+        reinterpret_cast<uint2*>(a.out + sh * D)[tid] = packed;
+    }
+}
 
 namespace {
 
@@ -127,8 +178,16 @@ int launch_engine(DecodeArgs args, const void* k_cache, const void* v_cache, int
         kernel<<<sms, NW * 32, Lay::kAlloc, stream>>>(c, kmap, vmap);
         if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
         if (args.num_partitions > 1) {
-            paged_decode_merge_kernel<Tag, D><<<(unsigned)((int64_t)c.num_seqs * args.num_heads), D, 0, stream>>>(c);
-            if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)((int64_t)c.num_seqs * args.num_heads));
+            cfg.blockDim = dim3(kMergeThreads);
+            cfg.stream = stream;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[0].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaLaunchKernelEx(&cfg, paged_decode_merge_kernel<Tag, D>, c) != cudaSuccess) return PA_ERR_CUDA;
         }
     }
     return PA_OK;
@@ -140,14 +199,16 @@ int launch_decode(DecodeArgs args, const void* k_cache, const void* v_cache, int
     constexpr int R = PA_DECODE_SLOTS;
     if (args.group >= 2 && args.group <= PA_GQA_MAX_GROUP) {
         constexpr int TOK = PA_GQA_TOK;
+        constexpr int GR = PA_GQA_SLOTS;
         args.unit_heads = num_kv_heads;
         args.heads_per_unit = args.group;
         if (args.group <= 8)
-            return launch_engine<Tag, D, TOK, PA_GQA_WARPS, R, GqaPolicy<Tag, D, TOK, 1>>(args, k_cache, v_cache,
-                                                                                          num_kv_heads, stream);
-        // two head tiles need more registers per thread: fewer warps per CTA
-        return launch_engine<Tag, D, TOK, 8, R, GqaPolicy<Tag, D, TOK, 2>>(args, k_cache, v_cache, num_kv_heads,
-                                                                           stream);
+            return launch_engine<Tag, D, TOK, PA_GQA_WARPS, GR, GqaPolicy<Tag, D, TOK, 1>>(args, k_cache, v_cache,
+                                                                                           num_kv_heads, stream);
+        // two head tiles need more registers per thread: at most 8 warps per CTA
+        constexpr int NW2 = PA_GQA_WARPS < 8 ? PA_GQA_WARPS : 8;
+        return launch_engine<Tag, D, TOK, NW2, GR, GqaPolicy<Tag, D, TOK, 2>>(args, k_cache, v_cache, num_kv_heads,
+                                                                              stream);
     }
     constexpr int TOK = D == 128 ? PA_DECODE_TOK128 : PA_DECODE_TOK64;
     args.unit_heads = args.num_heads;
