@@ -37,7 +37,8 @@ METRIC = "decode-attention tokens/s and KV-cache HBM GB/s (fraction of ~8 TB/s) 
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "paged_decode_llama7b.md")
-DECODE_SOURCE = os.path.join(ROOT, "paged_kv_cache_374_b200", "csrc", "paged_decode.cu")
+DECODE_SOURCES = [os.path.join(ROOT, "paged_kv_cache_374_b200", "csrc", f) for f in
+                  ("paged_decode.cu", "decode_engine.cuh", "decode_mha.cuh", "decode_gqa.cuh", "pa_device.cuh")]
 
 
 def parse():
@@ -71,9 +72,12 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def source_digest(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_digest(paths):
+    h = hashlib.sha256()
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def profiled_traffic(units_now: int):
@@ -87,7 +91,7 @@ def profiled_traffic(units_now: int):
                 if line.startswith("- ") and ": " in line:
                     k, v = line[2:].split(": ", 1)
                     fields[k.strip()] = v.strip().strip("`")
-        if fields.get("source_sha256_16") != source_digest(DECODE_SOURCE):
+        if fields.get("source_sha256_16") != source_digest(DECODE_SOURCES):
             return None
         per_token = float(fields["dram_bytes_per_launch"]) / float(fields["tokens_per_launch"])
         return per_token * units_now

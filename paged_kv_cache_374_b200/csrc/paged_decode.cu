@@ -48,19 +48,21 @@ namespace pa {
 
 // K3: merge the partitions of each (s, h) (base-2 units):
 //   M = max_p m_p,  out = sum_p o_p 2^(m_p - M) / sum_p l_p 2^(m_p - M).
-// One CTA of 4 warps per (s, h): the max and the denominator are block-wide
-// reductions over the partitions; for the numerator each warp takes every 4th
-// partition and each lane 4 dims (16-byte loads), and the warps' sums meet in
-// shared memory.  Launched as a programmatic dependent of K2: its blocks may start
-// while K2's last CTAs finish and wait (griddepcontrol.wait) until K2's writes are
-// complete and visible.
-constexpr int kMergeThreads = 128;
+// One CTA of 8 warps per (s, h), one pass over the partials: each warp takes
+// every 8th partition (each lane 4 dims, 16-byte loads, 4 partitions in flight)
+// and keeps its own running max, rescaling its sums when the max grows; the 8
+// warp results are combined with the same formula in shared memory.  Launched as
+// a programmatic dependent of K2: its blocks may start while K2's last CTAs
+// finish and wait (griddepcontrol.wait) until K2's writes are complete and visible.
+constexpr int kMergeThreads = 256;
 
 template <class Tag, int D>
 __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const DecodeArgs a) {
+    constexpr int NWM = kMergeThreads / 32;
+    constexpr int BATCH = 4;
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    __shared__ float s_red[kMergeThreads / 32];
-    __shared__ float4 s_acc[kMergeThreads / 32][D / 4];
+    __shared__ float s_m[NWM], s_l[NWM];
+    __shared__ float4 s_acc[NWM][D / 4];
     const int64_t sh = blockIdx.x;
     const int s = (int)(sh / a.num_heads);
     const int L = a.context_lens[s];
@@ -71,49 +73,64 @@ __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const
     const float* pl = a.ws_l + sh * a.num_partitions;
     const float4* po = reinterpret_cast<const float4*>(a.ws_o + sh * a.num_partitions * D);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool active = lane < D / 4;
 
-    float mx = -INFINITY;
-    for (int p = tid; p < nparts; p += kMergeThreads) mx = fmaxf(mx, pm[p]);
-    mx = warp_max(mx);
-    if (lane == 0) s_red[warp] = mx;
-    __syncthreads();
-    float M = s_red[0];
-#pragma unroll
-    for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, s_red[w]);
-    __syncthreads();
-
-    float den = 0.f;
-    for (int p = tid; p < nparts; p += kMergeThreads) den += pl[p] * (pm[p] == -INFINITY ? 0.f : exp2f(pm[p] - M));
-    den = warp_sum(den);
-    if (lane == 0) s_red[warp] = den;
-
+    float m = -INFINITY, l = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (lane < D / 4) {
-#pragma unroll 4
-        for (int p = warp; p < nparts; p += kMergeThreads / 32) {
-            const float w = pm[p] == -INFINITY ? 0.f : exp2f(pm[p] - M);
-            const float4 v = po[(int64_t)p * (D / 4) + lane];
-            acc.x = fmaf(w, v.x, acc.x);
-            acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z);
-            acc.w = fmaf(w, v.w, acc.w);
+    for (int p0 = warp; p0 < nparts; p0 += NWM * BATCH) {
+        float mb[BATCH], lb[BATCH];
+        float4 ob[BATCH];
+#pragma unroll
+        for (int j = 0; j < BATCH; ++j) {  // loads of BATCH partitions first
+            const int p = p0 + j * NWM;
+            const bool in = p < nparts;
+            mb[j] = in ? pm[p] : -INFINITY;
+            lb[j] = in ? pl[p] : 0.f;
+            ob[j] = (in && active) ? po[(int64_t)p * (D / 4) + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        s_acc[warp][lane] = acc;
+#pragma unroll
+        for (int j = 0; j < BATCH; ++j) {
+            if (mb[j] == -INFINITY) continue;  // partition absent (warp-uniform)
+            if (mb[j] > m) {
+                const float alpha = exp2f(m - mb[j]);
+                l *= alpha;
+                acc.x *= alpha;
+                acc.y *= alpha;
+                acc.z *= alpha;
+                acc.w *= alpha;
+                m = mb[j];
+            }
+            const float w = exp2f(mb[j] - m);
+            l = fmaf(w, lb[j], l);
+            acc.x = fmaf(w, ob[j].x, acc.x);
+            acc.y = fmaf(w, ob[j].y, acc.y);
+            acc.z = fmaf(w, ob[j].z, acc.z);
+            acc.w = fmaf(w, ob[j].w, acc.w);
+        }
     }
+    if (lane == 0) {
+        s_m[warp] = m;
+        s_l[warp] = l;
+    }
+    if (active) s_acc[warp][lane] = acc;
     __syncthreads();
     if (tid < D / 4) {
-        float dsum = 0.f;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NWM; ++w) M = fmaxf(M, s_m[w]);
+        float den = 0.f;
         float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int w = 0; w < kMergeThreads / 32; ++w) {
-            dsum += s_red[w];
+        for (int w = 0; w < NWM; ++w) {
+            const float sc = s_m[w] == -INFINITY ? 0.f : exp2f(s_m[w] - M);
+            den = fmaf(sc, s_l[w], den);
             const float4 v = s_acc[w][tid];
-            t.x += v.x;
-            t.y += v.y;
-            t.z += v.z;
-            t.w += v.w;
+            t.x = fmaf(sc, v.x, t.x);
+            t.y = fmaf(sc, v.y, t.y);
+            t.z = fmaf(sc, v.z, t.z);
+            t.w = fmaf(sc, v.w, t.w);
         }
-        const float inv = 1.f / dsum;
+        const float inv = 1.f / den;
         uint2 packed;
         packed.x = pack2<Tag>(t.x * inv, t.y * inv);
         packed.y = pack2<Tag>(t.z * inv, t.w * inv);
