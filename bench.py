@@ -64,6 +64,25 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise max of a list of floats over all ranks (identity on one rank).
+
+    Every rank of a replica run times its own copy of the workload; the job's time
+    is the slowest rank's.
+    """
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return list(values)
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_throughput(world, tokens_per_step, ms_per_step):
+    """Whole-job tokens/s: every rank decodes tokens_per_step tokens per step."""
+    return world * tokens_per_step / (ms_per_step / 1e3)
+
+
 def measured_hbm_peak():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -305,10 +324,7 @@ def run_native(args):
     elapsed_ms = start.elapsed_time(stop)
     k1_ms = statistics.mean(a.elapsed_time(b) for a, b in k1_ev)
     k2_ms = statistics.mean(a.elapsed_time(b) for a, b in k2_ev)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    (elapsed_ms,) = max_over_ranks([elapsed_ms], dist if world > 1 else None, device)
 
     # e2e through the binding: per step, H2D of the step's inputs from pinned
     # host memory, K1, K2(+K3), D2H of the output
@@ -339,15 +355,12 @@ def run_native(args):
     e1.record(stream)
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    (e2e_ms,) = max_over_ranks([e2e_ms], dist if world > 1 else None, device)
 
     ab = algorithmic_bytes(st)
     ms_per_step = elapsed_ms / args.steps
     tokens_per_step = spec.num_seqs
-    value = world * tokens_per_step / (ms_per_step / 1e3)
+    value = job_throughput(world, tokens_per_step, ms_per_step)
     peak, peak_kind = measured_hbm_peak()
     achieved = ab["unique"] / (k2_ms / 1e3) / 1e9
     nparts_max = -(-int(st["wl"].max_blocks_per_seq * spec.block_size) // (
@@ -381,7 +394,7 @@ def run_native(args):
             "unit": "GB/s", "frac": round(achieved / peak, 4),
             "traffic": profiled_traffic(ab["unique_tokens"]),
         },
-        "e2e": {"value": round(world * tokens_per_step / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(job_throughput(world, tokens_per_step, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * launches_per_step,
         "clocks": sampler.summary() if sampler else None,
