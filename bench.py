@@ -52,6 +52,8 @@ def parse():
     p.add_argument("--num-seqs", type=int, default=None, help="truncate the batch (smaller profiling case)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--row", default="decode", choices=["decode", "copy_blocks"],
+                   help="decode: the hot path (default); copy_blocks: copy-on-write block copies alone")
     return p.parse_args()
 
 
@@ -503,8 +505,43 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_copy_blocks(args):
+    """Copy-on-write block copies: 512 (src, dst) pairs of the beam workload's blocks
+    (block size 64, 32 kv heads, head_dim 128, fp16: 512 KiB per block per cache),
+    i.e. 512 MiB read + 512 MiB written per call, timed with CUDA events."""
+    import torch
+    from paged_kv_cache_374_b200 import binding as pa
+    nb, bs, hk, d, n = 1536, 64, 32, 128, 512
+    kc = torch.empty(nb, bs, hk, d, dtype=torch.float16, device="cuda").normal_()
+    vc = torch.empty_like(kc).normal_()
+    g = torch.Generator().manual_seed(5)
+    perm = torch.randperm(nb, generator=g)
+    pairs = torch.stack([perm[:n], perm[n:2 * n]], dim=1).to(torch.int32).cuda()
+    for _ in range(max(3, args.warmup)):
+        pa.pa_copy_blocks(kc, vc, pairs)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = min(args.steps, 200)
+    e0.record()
+    for _ in range(steps):
+        pa.pa_copy_blocks(kc, vc, pairs)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    moved = 2 * 2 * n * bs * hk * d * 2
+    peak, kind = measured_hbm_peak()
+    gbs = moved / (ms / 1e3) / 1e9
+    print(json.dumps({"row": "copy_blocks", "metric": "copy-on-write block copy GB/s (read + write)",
+                      "value": round(gbs, 1), "unit": "GB/s", "ms_per_call": round(ms, 4), "pairs": n,
+                      "bytes_per_call": moved, "frac_of_copy_peak": round(gbs / peak, 4), "peak_kind": kind,
+                      "steps": steps}), flush=True)
+
+
 def main():
     args = parse()
+    if args.row == "copy_blocks":
+        run_copy_blocks(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

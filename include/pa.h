@@ -237,6 +237,45 @@ double pa_usage(const pa_allocator* a);                             /* allocated
 int pa_append_slots(pa_allocator* a, int32_t* block_tables, int max_blocks_per_seq, int32_t* context_lens,
                     int num_seqs, int block_size, int64_t* slot_mapping);
 
+/* ------------------------------------------------------------ copy-on-write */
+
+/*
+ * pa_cow_prepare -- copy-on-write before appending into a shared block (host).
+ *
+ * A beam fork copies block references, each shared block's count going up by one
+ * (P3 §四, beam search; P3 §三, share_prefix_blocks).  When a sequence then appends
+ * into a shared block that is only partly filled, it must first get a private copy
+ * (the pages stop at the fork; this is the plainest completion of it).  For each
+ * sequence s with n = context_lens[s] stored tokens and n % block_size != 0, the
+ * next token goes into block j = n / block_size; if that block's reference count
+ * is above 1, a fresh block is allocated into block_tables[s][j], one reference of
+ * the shared block is dropped, and the pair (shared, fresh) is appended to
+ * copy_pairs.  Sequences are handled in order, so of c sequences appending into
+ * one block held by exactly c references, the last keeps the original.
+ *
+ *   block_tables  host int32 [num_seqs][max_blocks_per_seq], in/out
+ *   context_lens  host int32 [num_seqs] (stored tokens, not changed)
+ *   copy_pairs    host int32 [2 * num_seqs] out: (src, dst) pairs; *num_copies pairs
+ * All or nothing: PA_ERR_OUT_OF_BLOCKS or PA_ERR_INVALID_ARG change nothing.  Run
+ * pa_copy_blocks on the pairs before the step's pa_reshape_and_cache.
+ */
+int pa_cow_prepare(pa_allocator* a, int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                   int num_seqs, int block_size, int32_t* copy_pairs, int* num_copies);
+
+/*
+ * pa_copy_blocks -- copy whole physical blocks of both caches on the device.
+ *
+ * For i < num_pairs: k_cache[dst_i] = k_cache[src_i] and v_cache[dst_i] =
+ * v_cache[src_i], all block_size x num_kv_heads x head_dim elements, bit for bit.
+ *   copy_pairs  device int32 [2 * num_pairs]: (src, dst) per pair
+ *   element_bytes  bytes per cache element (2 for fp16/bf16, 1 for 8-bit caches)
+ * Destinations must be distinct and must not be sources of other pairs.  A pair
+ * with an id outside [0, num_blocks) is skipped and sets PA_DEVERR_TABLE_RANGE.
+ */
+int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* copy_pairs, int num_pairs, int num_kv_heads,
+                   int head_dim, int block_size, int num_blocks, int element_bytes, int32_t* err_word,
+                   void* stream);
+
 #ifdef __cplusplus
 }
 #endif

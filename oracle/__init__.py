@@ -8,6 +8,7 @@ module is argument marshalling over numpy arrays of raw 16-bit patterns.
 Functions and what they follow (page titles are given in full in pa_oracle.c):
   decode               softmax(q K^T * scale) V, one softmax over all tokens (P1 §1)
   reshape_and_cache    new K/V rows copied into their slots, bit for bit (P2 §2.1)
+  copy_blocks          whole-block copies for copy-on-write after a fork (P3 §四)
   slot_mapping         slot of the newest token through the table (P3 §三)
   physical_location    token -> (table[idx // B], idx % B)  (P3 §三)
   num_required_blocks  ceil(n / B)  (P3 §三)
@@ -61,6 +62,8 @@ class Oracle:
         lib.pa_oracle_decode.restype = ctypes.c_int
         lib.pa_oracle_decode.argtypes = ([_c_u16p, _c_u16p, _c_u16p, _c_i32p, _c_i32p, ctypes.c_double]
                                          + [ctypes.c_int] * 8 + [_c_i32p, ctypes.c_int, _c_f64p, ctypes.c_int])
+        lib.pa_oracle_copy_blocks.restype = ctypes.c_int
+        lib.pa_oracle_copy_blocks.argtypes = [_c_u16p, _c_u16p, _c_i32p] + [ctypes.c_int] * 5
         lib.pa_oracle_mutant_id.restype = ctypes.c_int
         lib.pa_oracle_mutant_id.argtypes = []
         self._lib = lib
@@ -112,6 +115,15 @@ class Oracle:
         return self._lib.pa_oracle_reshape_and_cache(_ptr(k, _c_u16p), _ptr(v, _c_u16p), _ptr(slots, _c_i64p),
                                                      _ptr(k_cache, _c_u16p), _ptr(v_cache, _c_u16p),
                                                      num_tokens, hk, d, bs, nb)
+
+    def copy_blocks(self, k_cache: np.ndarray, v_cache: np.ndarray, pairs) -> int:
+        """In place: block dst of both caches := block src, for each (src, dst)."""
+        for a in (k_cache, v_cache):
+            assert a.dtype == np.uint16 and a.flags.c_contiguous
+        nb, bs, hk, d = k_cache.shape
+        pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+        return self._lib.pa_oracle_copy_blocks(_ptr(k_cache, _c_u16p), _ptr(v_cache, _c_u16p), _ptr(pr, _c_i32p),
+                                               pr.shape[0], nb, bs, hk, d)
 
     # -- K2 + K3 -------------------------------------------------------------
     def decode(self, q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, block_tables: np.ndarray,

@@ -14,6 +14,10 @@ by step, in Python, as the oracle the C++ allocator is compared with id for id:
                 (PageAttentionManager::append_slot)
   fork          copy a table's ids, each add_ref'd (P3 §四, beam search: "fork copies
                 the block references, reference count + 1")
+  cow_prepare   before appending into a partly filled block that is still shared,
+                take a private copy: allocate, drop one reference of the shared
+                block, record (shared, fresh) -- the completion of the fork that the
+                pages leave implicit
 
 One deliberate difference from the listing: its ``free`` saturates at zero in
 silence; here freeing (or add_ref-ing) a block whose count is already zero is an
@@ -125,6 +129,34 @@ class ManagerModel:
     def free_request(self, rid: int) -> None:
         for b in self.tables.pop(rid, []):
             self.pool.free(b)
+
+    def cow_prepare(self, stored_lens: dict[int, int]) -> list[tuple[int, int]]:
+        """Copy-on-write for the requests about to append (request id -> stored tokens),
+        handled in ascending request order; returns the (src, dst) copies."""
+        pairs = []
+        pending = []
+        for rid in sorted(stored_lens):
+            n = stored_lens[rid]
+            if n % self.block_size == 0:
+                continue  # the next token opens a fresh block
+            pending.append((rid, n // self.block_size))
+        # all or nothing: simulate the counts first
+        need, ref = 0, list(self.pool.ref)
+        for rid, j in pending:
+            b = self.tables[rid][j]
+            if ref[b] > 1:
+                ref[b] -= 1
+                need += 1
+        if need > self.pool.num_free():
+            raise OutOfBlocks(f"copy-on-write needs {need}, available {self.pool.num_free()}")
+        for rid, j in pending:
+            b = self.tables[rid][j]
+            if self.pool.ref[b] > 1:
+                fresh = self.pool.allocate()
+                self.pool.ref[b] -= 1
+                self.tables[rid][j] = fresh
+                pairs.append((b, fresh))
+        return pairs
 
     def share_prefix_blocks(self, src: int, dst: int, shared_len: int) -> None:
         n = num_required_blocks(shared_len, self.block_size)

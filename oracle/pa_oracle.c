@@ -178,6 +178,27 @@ int pa_oracle_reshape_and_cache(const uint16_t* k, const uint16_t* v, const int6
     return skipped;
 }
 
+/* ------------------------------------------------------ whole-block copies */
+
+/* For each pair (src, dst): the dst block of both caches becomes a copy of the
+ * src block (block_size * num_kv_heads * head_dim elements), bit for bit.  Pairs
+ * with an id outside [0, num_blocks) are skipped; the return value counts them. */
+int pa_oracle_copy_blocks(uint16_t* k_cache, uint16_t* v_cache, const int32_t* pairs, int num_pairs,
+                          int num_blocks, int block_size, int num_kv_heads, int head_dim) {
+    int skipped = 0;
+    const int64_t per_block = (int64_t)block_size * num_kv_heads * head_dim;
+    for (int i = 0; i < num_pairs; ++i) {
+        const int32_t src = pairs[2 * i], dst = pairs[2 * i + 1];
+        if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+            ++skipped;
+            continue;
+        }
+        memmove(k_cache + dst * per_block, k_cache + src * per_block, sizeof(uint16_t) * (size_t)per_block);
+        memmove(v_cache + dst * per_block, v_cache + src * per_block, sizeof(uint16_t) * (size_t)per_block);
+    }
+    return skipped;
+}
+
 /* ------------------------------------------------------------- decode (K2+K3) */
 
 typedef struct {

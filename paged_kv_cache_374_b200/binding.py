@@ -60,6 +60,8 @@ _sig("pa_num_free", _i32, _vp)
 _sig("pa_num_blocks", _i32, _vp)
 _sig("pa_usage", ctypes.c_double, _vp)
 _sig("pa_append_slots", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32, _i64p)
+_sig("pa_cow_prepare", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32, _i32p, ctypes.POINTER(ctypes.c_int))
+_sig("pa_copy_blocks", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp)
 
 
 class PAError(RuntimeError):
@@ -282,6 +284,32 @@ def pa_append_slots(handle, block_tables: np.ndarray, context_lens: np.ndarray, 
     return slots
 
 
+def pa_cow_prepare(handle, block_tables: np.ndarray, context_lens: np.ndarray, block_size: int) -> np.ndarray:
+    """In place on block_tables (int32 [S, MB]); returns the (src, dst) copy pairs, int32 [k, 2]."""
+    tables = _np_i32(block_tables, "block_tables")
+    lens = _np_i32(np.ascontiguousarray(context_lens, dtype=np.int32), "context_lens")
+    s, mb = tables.shape
+    pairs = np.empty(2 * max(s, 1), dtype=np.int32)
+    k = ctypes.c_int(0)
+    _check(_lib.pa_cow_prepare(handle, tables.ctypes.data_as(_i32p), mb, lens.ctypes.data_as(_i32p), s, block_size,
+                               pairs.ctypes.data_as(_i32p), ctypes.byref(k)), "pa_cow_prepare")
+    return pairs[:2 * k.value].reshape(-1, 2).copy()
+
+
+def pa_copy_blocks(k_cache, v_cache, copy_pairs, err_word=None, stream=None) -> None:
+    """Device block copies; copy_pairs: int32 CUDA tensor [n, 2] of (src, dst)."""
+    import torch
+    nb, bs, hk, d = k_cache.shape
+    if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
+        raise ValueError("k_cache and v_cache must match")
+    if copy_pairs.dim() != 2 or copy_pairs.shape[1] != 2:
+        raise ValueError("copy_pairs must be [n, 2]")
+    st = _lib.pa_copy_blocks(_dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                             _dev(copy_pairs, "copy_pairs", torch.int32), copy_pairs.shape[0], hk, d, bs, nb,
+                             k_cache.element_size(), _dev(err_word, "err_word", torch.int32), _stream(stream, k_cache))
+    _check(st, "pa_copy_blocks")
+
+
 class BlockAllocator:
     """Owning wrapper over a pa_allocator handle."""
 
@@ -326,3 +354,6 @@ class BlockAllocator:
 
     def append_slots(self, block_tables: np.ndarray, context_lens: np.ndarray, block_size: int) -> np.ndarray:
         return pa_append_slots(self.handle, block_tables, context_lens, block_size)
+
+    def cow_prepare(self, block_tables: np.ndarray, context_lens: np.ndarray, block_size: int) -> np.ndarray:
+        return pa_cow_prepare(self.handle, block_tables, context_lens, block_size)

@@ -190,6 +190,58 @@ int pa_append_slots(pa_allocator* a, int32_t* block_tables, int max_blocks_per_s
     return PA_OK;
 }
 
+int pa_cow_prepare(pa_allocator* a, int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                   int num_seqs, int block_size, int32_t* copy_pairs, int* num_copies) {
+    if (!a || num_seqs < 0 || max_blocks_per_seq < 0 || block_size <= 0 || !num_copies) return PA_ERR_INVALID_ARG;
+    if (num_seqs > 0 && (!block_tables || !context_lens || !copy_pairs)) return PA_ERR_INVALID_ARG;
+    // Pass 1: validate, and count per shared block how many sequences append into it.
+    std::vector<int32_t> appenders;
+    try {
+        appenders.assign(a->n, 0);
+    } catch (...) {
+        return PA_ERR_INVALID_ARG;
+    }
+    for (int s = 0; s < num_seqs; ++s) {
+        const int64_t n = context_lens[s];
+        if (n < 0) return PA_ERR_INVALID_ARG;
+        if (n % block_size == 0) continue;  // the next token opens a new block: nothing shared to copy
+        const int64_t j = n / block_size;
+        if (j >= max_blocks_per_seq) return PA_ERR_INVALID_ARG;
+        const int32_t id = block_tables[(int64_t)s * max_blocks_per_seq + j];
+        if (!a->valid(id) || a->ref[id] == 0) return PA_ERR_INVALID_ARG;
+        ++appenders[id];
+    }
+    // A block with r references and c appenders in this batch needs c copies when
+    // r > c (someone outside the batch keeps the original), else c - 1 (the last
+    // appender keeps it).
+    int64_t need = 0;
+    for (int32_t id = 0; id < a->n; ++id) {
+        const int32_t c = appenders[id];
+        if (c == 0) continue;
+        if (a->ref[id] < c) return PA_ERR_INVALID_ARG;  // a table lists a block it does not hold
+        need += a->ref[id] > c ? c : c - 1;
+    }
+    if (a->count < need) return PA_ERR_OUT_OF_BLOCKS;
+    // Pass 2: in sequence order, move each appender off a still-shared block.
+    int k = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        const int64_t n = context_lens[s];
+        if (n % block_size == 0) continue;
+        int32_t* slot = block_tables + (int64_t)s * max_blocks_per_seq + n / block_size;
+        const int32_t src = *slot;
+        if (a->ref[src] <= 1) continue;
+        const int32_t dst = a->pop_front();
+        a->ref[dst] = 1;
+        --a->ref[src];
+        *slot = dst;
+        copy_pairs[2 * k] = src;
+        copy_pairs[2 * k + 1] = dst;
+        ++k;
+    }
+    *num_copies = k;
+    return PA_OK;
+}
+
 const char* pa_status_string(int status) {
     switch (status) {
         case PA_OK: return "PA_OK";

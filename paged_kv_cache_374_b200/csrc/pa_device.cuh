@@ -78,26 +78,33 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// One poll of an mbarrier phase.  The thread may be suspended by the hardware for
+// up to `hint_ns` while the phase is still open (it resumes as soon as the phase
+// completes), so a waiting warp sleeps instead of spinning on issue slots.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
         : "memory");
     return ok != 0;
 }
 
-// Every wait in the library is bounded: after this many polls (each poll may
-// suspend the thread for a short, hardware-chosen time) the caller gives up,
-// reports PA_DEVERR_TIMEOUT and unwinds.
-constexpr uint32_t kWaitPolls = 1u << 22;
+// Every wait in the library is bounded: after kWaitPolls polls of at most
+// kWaitHintNs each (about 2 s in all) the caller gives up, reports
+// PA_DEVERR_TIMEOUT and unwinds.
+#ifndef PA_WAIT_HINT_NS
+#define PA_WAIT_HINT_NS 20000
+#endif
+constexpr uint32_t kWaitHintNs = PA_WAIT_HINT_NS;
+constexpr uint32_t kWaitPolls = 2000000000u / kWaitHintNs;
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     for (uint32_t i = 0; i < kWaitPolls; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait(bar, parity, kWaitHintNs)) return true;
     return false;
 }
 

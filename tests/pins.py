@@ -201,6 +201,21 @@ def pin_reshape_and_cache(o):
     assert np.array_equal(kc, ek) and np.array_equal(vc, ev), "cache write differs from the slot rule"
 
 
+def pin_copy_blocks(o):
+    """Whole-block copies against numpy assignment on the 4-D view; bad ids skipped."""
+    rng = np.random.default_rng(23)
+    nb, bs, hk, d = 9, 16, 2, 64
+    kc = rng.integers(0, 65535, size=(nb, bs, hk, d), dtype=np.uint16)
+    vc = rng.integers(0, 65535, size=(nb, bs, hk, d), dtype=np.uint16)
+    pairs = np.array([[3, 7], [0, 5], [8, 1], [2, 99]], dtype=np.int32)
+    ek, ev = kc.copy(), vc.copy()
+    for src, dst in pairs[:3]:
+        ek[dst] = kc[src]
+        ev[dst] = vc[src]
+    assert o.copy_blocks(kc, vc, pairs) == 1
+    assert np.array_equal(kc, ek) and np.array_equal(vc, ev)
+
+
 # -------------------------------------------------------------------- decode
 
 def pin_decode_one_token(o):

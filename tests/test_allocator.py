@@ -174,3 +174,41 @@ def test_append_slots_is_all_or_nothing(pa):
     assert np.array_equal(tables, t0) and np.array_equal(lens, l0)
     full = np.full((1, 1), 0, dtype=np.int32)
     _expect_error(pa, lambda: a.append_slots(full, np.array([16], dtype=np.int32), bs), pa.PA_ERR_INVALID_ARG)
+
+
+def test_cow_prepare_matches_model(pa):
+    """Random forks and appends: the library's copy-on-write step equals the model's,
+    id for id, including the tables and every reference count."""
+    rng = np.random.default_rng(10)
+    for trial in range(30):
+        bs = int(rng.choice([4, 16]))
+        nb = 64
+        order = rng.permutation(nb).astype(np.int32)
+        a = pa.BlockAllocator(nb, order)
+        mgr = ManagerModel(nb, bs, order)
+        nreq, mb = 6, 12
+        tables = np.full((nreq, mb), -1, dtype=np.int32)
+        prompt = int(rng.integers(1, 3 * bs))
+        mgr.allocate_for_request(0, prompt)
+        n0 = pa.pa_num_required_blocks(prompt, bs)
+        tables[0, :n0] = a.alloc_n(n0)
+        stored = {0: prompt}
+        for rid in range(1, nreq):           # forks of request 0's prompt, some of them partial
+            shared = int(rng.integers(1, prompt + 1))
+            mgr.share_prefix_blocks(0, rid, shared)
+            k = pa.pa_num_required_blocks(shared, bs)
+            tables[rid, :k] = a.fork(tables[0, :k])
+            stored[rid] = shared
+        lens = np.array([stored[r] for r in range(nreq)], dtype=np.int32)
+        try:
+            want = mgr.cow_prepare(dict(stored))
+        except OutOfBlocks:
+            with pytest.raises(pa.PAError):
+                a.cow_prepare(tables, lens, bs)
+            continue
+        got = a.cow_prepare(tables, lens, bs)
+        assert [tuple(x) for x in got.tolist()] == want
+        for r in range(nreq):
+            assert list(tables[r, :len(mgr.tables[r])]) == mgr.tables[r]
+        for b in range(nb):
+            assert a.refcount(b) == mgr.pool.ref[b]

@@ -50,3 +50,35 @@ def test_all_or_nothing_and_errors():
     assert p.ref[2] == 1 and 2 not in p.free_queue   # back to the queue only at zero
     p.free(2)
     assert list(p.free_queue) == [1, 0, 2]
+
+
+def test_copy_on_write_after_a_beam_fork():
+    """Four beams share a 40-token prompt (block size 16: two full blocks and one
+    holding 8 tokens).  Before appending, each beam still sharing the partly filled
+    block takes a private copy, in request order; the last holder keeps the original.
+    The full blocks stay shared."""
+    m = ManagerModel(20, 16)
+    m.allocate_for_request(0, 40)
+    a, b, c = m.tables[0]
+    for rid in (1, 2, 3):
+        m.share_prefix_blocks(0, rid, 40)
+    assert [m.pool.ref[x] for x in (a, b, c)] == [4, 4, 4]
+    pairs = m.cow_prepare({0: 40, 1: 40, 2: 40, 3: 40})
+    fresh = [3, 4, 5]                      # FIFO: the next free ids
+    assert pairs == [(c, f) for f in fresh]
+    assert [m.tables[r][2] for r in range(4)] == fresh + [c]
+    assert m.pool.ref[c] == 1 and all(m.pool.ref[f] == 1 for f in fresh)
+    assert m.pool.ref[a] == m.pool.ref[b] == 4
+    # nothing left to copy; a request on a block boundary never copies
+    assert m.cow_prepare({0: 40, 3: 40}) == []
+    assert m.cow_prepare({1: 48}) == []
+
+
+def test_copy_on_write_is_all_or_nothing():
+    m = ManagerModel(4, 16)
+    m.allocate_for_request(0, 20)          # 2 blocks, 2 free
+    for rid in (1, 2, 3):
+        m.share_prefix_blocks(0, rid, 20)  # refs 4
+    with pytest.raises(OutOfBlocks):
+        m.cow_prepare({0: 20, 1: 20, 2: 20, 3: 20})   # needs 3 copies, 2 free
+    assert m.pool.num_free() == 2 and m.pool.ref[m.tables[0][1]] == 4
