@@ -52,8 +52,9 @@ def parse():
     p.add_argument("--num-seqs", type=int, default=None, help="truncate the batch (smaller profiling case)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
-    p.add_argument("--row", default="decode", choices=["decode", "copy_blocks"],
-                   help="decode: the hot path (default); copy_blocks: copy-on-write block copies alone")
+    p.add_argument("--row", default="decode", choices=["decode", "copy_blocks", "swap"],
+                   help="decode: the hot path (default); copy_blocks: copy-on-write block copies alone; "
+                        "swap: swap-out / swap-in of blocks to pinned host memory")
     return p.parse_args()
 
 
@@ -537,10 +538,48 @@ def run_copy_blocks(args):
                       "steps": steps}), flush=True)
 
 
+def run_swap(args):
+    """Swap-out (device -> pinned host) and swap-in (host -> device) of 256 blocks of
+    the 7B layer geometry (block size 16, 32 kv heads, head_dim 128, fp16: 128 KiB
+    per block per cache, 64 MiB per call), timed with CUDA events."""
+    import torch
+    from paged_kv_cache_374_b200 import binding as pa
+    nd, nh, bs, hk, d, n = 1024, 512, 16, 32, 128, 256
+    kc = torch.empty(nd, bs, hk, d, dtype=torch.float16, device="cuda").normal_()
+    vc = torch.empty_like(kc).normal_()
+    kh = torch.zeros(nh, bs, hk, d, dtype=torch.float16).pin_memory()
+    vh = torch.zeros_like(kh).pin_memory()
+    g = torch.Generator().manual_seed(6)
+    pairs = torch.stack([torch.randperm(nd, generator=g)[:n], torch.randperm(nh, generator=g)[:n]], 1)
+    out_pairs = pairs.to(torch.int32).cuda()
+    in_pairs = pairs.flip(1).contiguous().to(torch.int32).cuda()
+    moved = 2 * n * bs * hk * d * 2
+    res = {}
+    for name, fn in (("swap_out", lambda: pa.pa_swap_blocks(kc, vc, kh, vh, out_pairs)),
+                     ("swap_in", lambda: pa.pa_swap_blocks(kh, vh, kc, vc, in_pairs))):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        steps = min(args.steps, 50)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        res[name] = {"GB/s": round(moved / (ms / 1e3) / 1e9, 2), "ms_per_call": round(ms, 4)}
+    print(json.dumps({"row": "swap", "metric": "swap-out / swap-in GB/s over the host link",
+                      "bytes_per_call": moved, "blocks_per_call": n, **res}), flush=True)
+
+
 def main():
     args = parse()
     if args.row == "copy_blocks":
         run_copy_blocks(args)
+        return
+    if args.row == "swap":
+        run_swap(args)
         return
     if args.impl == "reference":
         run_reference(args)

@@ -276,6 +276,38 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* copy_pairs, int 
                    int head_dim, int block_size, int num_blocks, int element_bytes, int32_t* err_word,
                    void* stream);
 
+/* ---------------------------------------------------------------- swapping */
+
+/*
+ * pa_swap_plan -- move one sequence's blocks from one pool to another (host).
+ *
+ * When no block is free for an append, a sequence is preempted: its KV blocks go to
+ * host memory and come back when the device has room (P3 §三, append_slot's
+ * "Preemption required"; P3 §五, swap to CPU memory and back).  With one allocator
+ * per pool (device pool, pinned host pool), this allocates num_blocks blocks in
+ * `to`, drops one reference of each listed block in `from` (a block shared with
+ * other sequences stays allocated for them), writes the (old, new) id pairs to
+ * `pairs` (int32 [2 * num_blocks]) and rewrites table_row with the new ids.
+ * All or nothing.  Copy the data with pa_swap_blocks before the freed blocks can
+ * be written again (stream order does this when both run on one stream).
+ */
+int pa_swap_plan(pa_allocator* from, pa_allocator* to, int32_t* table_row, int num_blocks, int32_t* pairs);
+
+/*
+ * pa_swap_blocks -- copy blocks between two block pools of the same geometry.
+ *
+ * For i < num_pairs: dst pool block pairs[2i+1] := src pool block pairs[2i], K and
+ * V, bit for bit.  Either pool may be pinned host memory that the device can
+ * address (cudaHostAlloc / cudaMallocHost memory under unified addressing), so
+ * one kernel moves a preempted sequence's blocks out to host memory or back in,
+ * without a staging buffer.  Pools are [num_blocks][block_size][num_kv_heads]
+ * [head_dim] of element_bytes each; pairs is int32 [2 * num_pairs] in device-
+ * readable memory.  Ids outside their pool are skipped and set PA_DEVERR_TABLE_RANGE.
+ */
+int pa_swap_blocks(const void* src_k, const void* src_v, int src_num_blocks, void* dst_k, void* dst_v,
+                   int dst_num_blocks, const int32_t* pairs, int num_pairs, int num_kv_heads, int head_dim,
+                   int block_size, int element_bytes, int32_t* err_word, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -14,6 +14,9 @@ by step, in Python, as the oracle the C++ allocator is compared with id for id:
                 (PageAttentionManager::append_slot)
   fork          copy a table's ids, each add_ref'd (P3 §四, beam search: "fork copies
                 the block references, reference count + 1")
+  swap_plan     move a preempted request's blocks to another pool (device <-> host):
+                allocate there, drop one reference here (P3 §三 "Preemption
+                required", P3 §五 swap to CPU memory and back)
   cow_prepare   before appending into a partly filled block that is still shared,
                 take a private copy: allocate, drop one reference of the shared
                 block, record (shared, fresh) -- the completion of the fork that the
@@ -98,6 +101,26 @@ class BlockPoolModel:
     def _check(self, b: int) -> None:
         if not 0 <= b < self.total:
             raise ValueError(f"block id {b} out of range")
+
+
+def swap_plan(src: BlockPoolModel, dst: BlockPoolModel, table: list[int]) -> list[tuple[int, int]]:
+    """Move the blocks of ``table`` (in place) from pool ``src`` to pool ``dst``:
+    all or nothing; returns the (old, new) pairs in table order."""
+    held = {}
+    for b in table:
+        src._check(b)
+        held[b] = held.get(b, 0) + 1
+        if src.ref[b] < held[b]:
+            raise RefcountError(f"block {b} is not held often enough")
+    if dst.num_free() < len(table):
+        raise OutOfBlocks(f"need {len(table)}, available {dst.num_free()}")
+    pairs = []
+    for i, b in enumerate(table):
+        fresh = dst.allocate()
+        src.free(b)
+        pairs.append((b, fresh))
+        table[i] = fresh
+    return pairs
 
 
 def num_required_blocks(num_tokens: int, block_size: int) -> int:

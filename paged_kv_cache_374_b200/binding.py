@@ -62,6 +62,8 @@ _sig("pa_usage", ctypes.c_double, _vp)
 _sig("pa_append_slots", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32, _i64p)
 _sig("pa_cow_prepare", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32, _i32p, ctypes.POINTER(ctypes.c_int))
 _sig("pa_copy_blocks", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp)
+_sig("pa_swap_plan", _i32, _vp, _vp, _i32p, _i32, _i32p)
+_sig("pa_swap_blocks", _i32, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp)
 
 
 class PAError(RuntimeError):
@@ -308,6 +310,40 @@ def pa_copy_blocks(k_cache, v_cache, copy_pairs, err_word=None, stream=None) -> 
                              _dev(copy_pairs, "copy_pairs", torch.int32), copy_pairs.shape[0], hk, d, bs, nb,
                              k_cache.element_size(), _dev(err_word, "err_word", torch.int32), _stream(stream, k_cache))
     _check(st, "pa_copy_blocks")
+
+
+def pa_swap_plan(from_handle, to_handle, table_row: np.ndarray, num_blocks: int) -> np.ndarray:
+    """Move num_blocks ids of table_row (int32, in place) from one pool to another;
+    returns the (old, new) pairs, int32 [num_blocks, 2]."""
+    row = _np_i32(table_row, "table_row")
+    pairs = np.empty(2 * max(num_blocks, 1), dtype=np.int32)
+    _check(_lib.pa_swap_plan(from_handle, to_handle, row.ctypes.data_as(_i32p), num_blocks,
+                             pairs.ctypes.data_as(_i32p)), "pa_swap_plan")
+    return pairs[:2 * num_blocks].reshape(-1, 2).copy()
+
+
+def pa_swap_blocks(src_k, src_v, dst_k, dst_v, pairs, err_word=None, stream=None) -> None:
+    """Copy blocks between two pools (torch tensors [NB, B, Hk, d]; either may be pinned
+    host memory); pairs: int32 tensor [n, 2] of (src, dst) in device-readable memory."""
+    import torch
+    snb, bs, hk, d = src_k.shape
+    dnb = dst_k.shape[0]
+    if dst_k.shape[1:] != src_k.shape[1:] or src_v.shape != src_k.shape or dst_v.shape != dst_k.shape:
+        raise ValueError("pools must share block geometry")
+    if src_k.dtype != dst_k.dtype:
+        raise TypeError("pools must share one dtype")
+    for name, t in (("src_k", src_k), ("src_v", src_v), ("dst_k", dst_k), ("dst_v", dst_v), ("pairs", pairs)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if not t.is_cuda and not t.is_pinned():
+            raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    if pairs.dtype != torch.int32 or pairs.dim() != 2 or pairs.shape[1] != 2:
+        raise ValueError("pairs must be int32 [n, 2]")
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    st = _lib.pa_swap_blocks(ptr(src_k), ptr(src_v), snb, ptr(dst_k), ptr(dst_v), dnb, ptr(pairs), pairs.shape[0],
+                             hk, d, bs, src_k.element_size(), _dev(err_word, "err_word", torch.int32),
+                             _stream(stream, src_k if src_k.is_cuda else dst_k))
+    _check(st, "pa_swap_blocks")
 
 
 class BlockAllocator:

@@ -242,6 +242,29 @@ int pa_cow_prepare(pa_allocator* a, int32_t* block_tables, int max_blocks_per_se
     return PA_OK;
 }
 
+int pa_swap_plan(pa_allocator* from, pa_allocator* to, int32_t* table_row, int num_blocks, int32_t* pairs) {
+    if (!from || !to || from == to || num_blocks < 0 || (num_blocks > 0 && (!table_row || !pairs)))
+        return PA_ERR_INVALID_ARG;
+    for (int i = 0; i < num_blocks; ++i) {
+        const int32_t id = table_row[i];
+        if (!from->valid(id) || from->ref[id] == 0) return PA_ERR_INVALID_ARG;
+        int seen = 0;  // a row listing one block twice would drop two references
+        for (int j = 0; j < i; ++j) seen += table_row[j] == id;
+        if (from->ref[id] - seen <= 0) return PA_ERR_REFCOUNT;
+    }
+    if (to->count < num_blocks) return PA_ERR_OUT_OF_BLOCKS;
+    for (int i = 0; i < num_blocks; ++i) {
+        const int32_t old = table_row[i];
+        const int32_t fresh = to->pop_front();
+        to->ref[fresh] = 1;
+        if (--from->ref[old] == 0) from->push_back(old);
+        pairs[2 * i] = old;
+        pairs[2 * i + 1] = fresh;
+        table_row[i] = fresh;
+    }
+    return PA_OK;
+}
+
 const char* pa_status_string(int status) {
     switch (status) {
         case PA_OK: return "PA_OK";

@@ -1,5 +1,5 @@
 // pa_copy_blocks: whole-block copies inside the paged caches (copy-on-write after
-// a beam fork).  One physical block of one cache is block_size * num_kv_heads *
+// a beam fork); pa_swap_blocks: the same between two pools (swap-out / swap-in).  One physical block of one cache is block_size * num_kv_heads *
 // head_dim elements, contiguous in the [num_blocks][block_size][num_kv_heads]
 // [head_dim] layout, so a pair is one contiguous run per cache; threads copy
 // 16-byte vectors, grid-stride over (pair, vector), K and V alike.
@@ -27,7 +27,55 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_
     }
 }
 
+// Cross-pool variant (swap-out / swap-in): source and destination are different
+// pools, either of which may be device-addressable pinned host memory.
+__global__ void __launch_bounds__(256) swap_blocks_kernel(const uint4* __restrict__ src_k,
+                                                           const uint4* __restrict__ src_v, int src_blocks,
+                                                           uint4* __restrict__ dst_k, uint4* __restrict__ dst_v,
+                                                           int dst_blocks, const int32_t* __restrict__ pairs,
+                                                           int num_pairs, int64_t block_vecs, int32_t* err_word) {
+    const int64_t total = (int64_t)num_pairs * block_vecs;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+        const int64_t pi = i / block_vecs;
+        const int64_t c = i - pi * block_vecs;
+        const int32_t src = __ldg(pairs + 2 * pi), dst = __ldg(pairs + 2 * pi + 1);
+        if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+            if (c == 0) report(err_word, PA_DEVERR_TABLE_RANGE);
+            continue;
+        }
+        dst_k[(int64_t)dst * block_vecs + c] = src_k[(int64_t)src * block_vecs + c];
+        dst_v[(int64_t)dst * block_vecs + c] = src_v[(int64_t)src * block_vecs + c];
+    }
+}
+
 }  // namespace pa
+
+extern "C" int pa_swap_blocks(const void* src_k, const void* src_v, int src_num_blocks, void* dst_k, void* dst_v,
+                              int dst_num_blocks, const int32_t* pairs, int num_pairs, int num_kv_heads,
+                              int head_dim, int block_size, int element_bytes, int32_t* err_word, void* stream) {
+    using namespace pa;
+    if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || src_num_blocks < 0 ||
+        dst_num_blocks < 0 || (element_bytes != 1 && element_bytes != 2))
+        return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PA_OK;
+    if (!src_k || !src_v || !dst_k || !dst_v || !pairs) return PA_ERR_INVALID_ARG;
+    const int64_t block_bytes = (int64_t)block_size * num_kv_heads * head_dim * element_bytes;
+    if (block_bytes % 16 != 0) return PA_ERR_UNSUPPORTED;
+    if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v) || !aligned4(pairs) ||
+        (err_word && !aligned4(err_word)))
+        return PA_ERR_INVALID_ARG;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t total = (int64_t)num_pairs * (block_bytes / 16);
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+    swap_blocks_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(src_k), static_cast<const uint4*>(src_v), src_num_blocks,
+        static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v), dst_num_blocks, pairs, num_pairs, block_bytes / 16,
+        err_word);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
 
 extern "C" int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* copy_pairs, int num_pairs,
                               int num_kv_heads, int head_dim, int block_size, int num_blocks, int element_bytes,

@@ -5,7 +5,7 @@ import os
 import numpy as np
 import pytest
 
-from oracle.block_pool import BlockPoolModel, ManagerModel, OutOfBlocks, RefcountError
+from oracle.block_pool import BlockPoolModel, ManagerModel, OutOfBlocks, RefcountError, swap_plan
 from pins import GOLDEN
 
 
@@ -212,3 +212,40 @@ def test_cow_prepare_matches_model(pa):
             assert list(tables[r, :len(mgr.tables[r])]) == mgr.tables[r]
         for b in range(nb):
             assert a.refcount(b) == mgr.pool.ref[b]
+
+
+def test_swap_plan_matches_model(pa):
+    """Preempting a sequence moves its blocks to the other pool; a block it shares
+    with another sequence stays allocated in the source pool for that sequence."""
+    rng = np.random.default_rng(12)
+    for trial in range(30):
+        nd, nh = 24, 10
+        od, oh = rng.permutation(nd).astype(np.int32), rng.permutation(nh).astype(np.int32)
+        dev, host = pa.BlockAllocator(nd, od), pa.BlockAllocator(nh, oh)
+        mdev, mhost = BlockPoolModel(nd, od), BlockPoolModel(nh, oh)
+        k = int(rng.integers(1, 8))
+        row = dev.alloc_n(k)
+        assert list(row) == mdev.allocate_n(k)
+        shared = [int(b) for b in row[: int(rng.integers(0, k + 1))]]   # another sequence holds a prefix
+        dev.fork(np.array(shared, dtype=np.int32))
+        mdev.fork(shared)
+        other = host.alloc_n(int(rng.integers(0, 5)))
+        mhost.allocate_n(len(other))
+        mrow = [int(b) for b in row]
+        try:
+            want = swap_plan(mdev, mhost, mrow)
+        except OutOfBlocks:
+            with pytest.raises(pa.PAError) as e:
+                pa.pa_swap_plan(dev.handle, host.handle, row, k)
+            assert e.value.status == pa.PA_ERR_OUT_OF_BLOCKS
+            continue
+        got = pa.pa_swap_plan(dev.handle, host.handle, row, k)
+        assert [tuple(x) for x in got.tolist()] == want and list(row) == mrow
+        assert dev.num_free() == mdev.num_free() and host.num_free() == mhost.num_free()
+        for b in range(nd):
+            assert dev.refcount(b) == mdev.ref[b]
+        # and back again
+        back = swap_plan(mhost, mdev, mrow)
+        got = pa.pa_swap_plan(host.handle, dev.handle, row, k)
+        assert [tuple(x) for x in got.tolist()] == back and list(row) == mrow
+        assert host.num_free() == mhost.num_free()
