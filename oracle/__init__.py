@@ -9,6 +9,7 @@ Functions and what they follow (page titles are given in full in pa_oracle.c):
   decode               softmax(q K^T * scale) V, one softmax over all tokens (P1 §1)
   reshape_and_cache    new K/V rows copied into their slots, bit for bit (P2 §2.1)
   copy_blocks          whole-block copies for copy-on-write after a fork (P3 §四)
+  reshape_and_cache_fp8 / decode_fp8 / e4m3_*   the fp8 (E4M3) cache variant
   slot_mapping         slot of the newest token through the table (P3 §三)
   physical_location    token -> (table[idx // B], idx % B)  (P3 §三)
   num_required_blocks  ceil(n / B)  (P3 §三)
@@ -31,6 +32,7 @@ BF16 = 1
 _c_i32p = ctypes.POINTER(ctypes.c_int32)
 _c_i64p = ctypes.POINTER(ctypes.c_int64)
 _c_u16p = ctypes.POINTER(ctypes.c_uint16)
+_c_u8p = ctypes.POINTER(ctypes.c_uint8)
 _c_f64p = ctypes.POINTER(ctypes.c_double)
 
 
@@ -64,6 +66,16 @@ class Oracle:
                                          + [ctypes.c_int] * 8 + [_c_i32p, ctypes.c_int, _c_f64p, ctypes.c_int])
         lib.pa_oracle_copy_blocks.restype = ctypes.c_int
         lib.pa_oracle_copy_blocks.argtypes = [_c_u16p, _c_u16p, _c_i32p] + [ctypes.c_int] * 5
+        lib.pa_oracle_e4m3_to_double.restype = ctypes.c_double
+        lib.pa_oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.pa_oracle_e4m3_from_float.restype = ctypes.c_uint8
+        lib.pa_oracle_e4m3_from_float.argtypes = [ctypes.c_float]
+        lib.pa_oracle_reshape_and_cache_fp8.restype = ctypes.c_int
+        lib.pa_oracle_reshape_and_cache_fp8.argtypes = ([_c_u16p, _c_u16p, _c_i64p, _c_u8p, _c_u8p]
+                                                        + [ctypes.c_int] * 6 + [ctypes.c_float] * 2)
+        lib.pa_oracle_decode_fp8.restype = ctypes.c_int
+        lib.pa_oracle_decode_fp8.argtypes = ([_c_u16p, _c_u8p, _c_u8p, _c_i32p, _c_i32p] + [ctypes.c_double] * 3
+                                             + [ctypes.c_int] * 8 + [_c_i32p, ctypes.c_int, _c_f64p, ctypes.c_int])
         lib.pa_oracle_mutant_id.restype = ctypes.c_int
         lib.pa_oracle_mutant_id.argtypes = []
         self._lib = lib
@@ -75,6 +87,12 @@ class Oracle:
 
     def bf16_to_double(self, bits: int) -> float:
         return self._lib.pa_oracle_bf16_to_double(int(bits))
+
+    def e4m3_to_double(self, code: int) -> float:
+        return self._lib.pa_oracle_e4m3_to_double(int(code))
+
+    def e4m3_from_float(self, x: float) -> int:
+        return self._lib.pa_oracle_e4m3_from_float(float(x))
 
     # -- slot arithmetic -----------------------------------------------------
     def num_required_blocks(self, num_tokens: int, block_size: int) -> int:
@@ -124,6 +142,49 @@ class Oracle:
         pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
         return self._lib.pa_oracle_copy_blocks(_ptr(k_cache, _c_u16p), _ptr(v_cache, _c_u16p), _ptr(pr, _c_i32p),
                                                pr.shape[0], nb, bs, hk, d)
+
+    def reshape_and_cache_fp8(self, k: np.ndarray, v: np.ndarray, slot_mapping: np.ndarray, k_cache: np.ndarray,
+                              v_cache: np.ndarray, dtype: int, k_scale: float, v_scale: float) -> int:
+        """Quantising cache write into uint8 E4M3 caches [NB, B, Hk, d]; returns skipped count."""
+        for a in (k, v):
+            assert a.dtype == np.uint16 and a.flags.c_contiguous
+        for a in (k_cache, v_cache):
+            assert a.dtype == np.uint8 and a.flags.c_contiguous
+        num_tokens, hk, d = k.shape
+        nb, bs = k_cache.shape[:2]
+        slots = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+        return self._lib.pa_oracle_reshape_and_cache_fp8(_ptr(k, _c_u16p), _ptr(v, _c_u16p), _ptr(slots, _c_i64p),
+                                                         _ptr(k_cache, _c_u8p), _ptr(v_cache, _c_u8p), num_tokens,
+                                                         hk, d, bs, nb, dtype, float(k_scale), float(v_scale))
+
+    def decode_fp8(self, q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, block_tables: np.ndarray,
+                   context_lens: np.ndarray, scale: float, k_scale: float, v_scale: float, dtype: int, pairs=None,
+                   nthreads: int = 1) -> np.ndarray:
+        """fp64 decode over uint8 E4M3 caches (K = code * k_scale, V = code * v_scale)."""
+        assert q.dtype == np.uint16 and q.flags.c_contiguous
+        for a in (k_cache, v_cache):
+            assert a.dtype == np.uint8 and a.flags.c_contiguous
+        num_seqs, num_heads, d = q.shape
+        nb, bs, hk, d2 = k_cache.shape
+        assert d2 == d and v_cache.shape == k_cache.shape
+        tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+        lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+        mb = tables.shape[1] if tables.ndim == 2 else 0
+        if pairs is None:
+            out = np.zeros((num_seqs, num_heads, d), dtype=np.float64)
+            pp, npairs = None, 0
+        else:
+            pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+            npairs = pr.shape[0]
+            out = np.zeros((npairs, d), dtype=np.float64)
+            pp = _ptr(pr, _c_i32p)
+        rc = self._lib.pa_oracle_decode_fp8(_ptr(q, _c_u16p), _ptr(k_cache, _c_u8p), _ptr(v_cache, _c_u8p),
+                                            _ptr(tables, _c_i32p), _ptr(lens, _c_i32p), float(scale), float(k_scale),
+                                            float(v_scale), num_seqs, num_heads, hk, d, bs, nb, mb, dtype, pp,
+                                            npairs, _ptr(out, _c_f64p), int(nthreads))
+        if rc != 0:
+            raise ValueError(f"oracle decode_fp8 rejected its input (code {rc})")
+        return out
 
     # -- K2 + K3 -------------------------------------------------------------
     def decode(self, q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, block_tables: np.ndarray,

@@ -94,6 +94,52 @@ static double widen(uint16_t bits, int dtype) {
     return dtype == ORACLE_BF16 ? pa_oracle_bf16_to_double(bits) : pa_oracle_half_to_double(bits);
 }
 
+/* OCP FP8 E4M3 ("e4m3fn"): 1 sign, 4 exponent bits (bias 7), 3 fraction bits, no
+ * infinities, S.1111.111 is NaN; largest finite magnitude 448. */
+double pa_oracle_e4m3_to_double(uint8_t b) {
+    int sign = (b >> 7) & 1;
+    int e = (b >> 3) & 0xf;
+    int m = b & 7;
+    double v;
+    if (e == 15 && m == 7)
+        v = NAN;
+    else if (e == 0)
+        v = ldexp((double)m, -9); /* subnormal: m/8 * 2^(1-7) */
+    else
+        v = ldexp((double)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */
+    return sign ? -v : v;
+}
+
+/* Nearest E4M3 code to x, ties to even; finite magnitudes at or beyond 448 and
+ * infinities saturate to +-448; NaN gives the NaN code. */
+uint8_t pa_oracle_e4m3_from_float(float x) {
+    if (isnan(x)) return 0x7f;
+    const int sign = signbit(x) ? 0x80 : 0;
+    const double a = fabs((double)x);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7e);
+    int e2;
+    frexp(a, &e2); /* a = f * 2^e2, f in [0.5, 1): floor(log2 a) = e2 - 1 */
+    const int subnormal = a < ldexp(1.0, -6);
+    const double quantum = subnormal ? ldexp(1.0, -9) : ldexp(1.0, e2 - 1 - 3);
+#if PA_ORACLE_MUTANT == 11
+    double n = trunc(a / quantum); /* planted: rounds toward zero */
+#else
+    double n = rint(a / quantum); /* the division is exact; rint rounds half to even */
+#endif
+    int code;
+    if (subnormal) {
+        code = (int)n; /* n == 8 is the smallest normal, whose code is 0x08 as well */
+    } else {
+        int E = e2 - 1 + 7;
+        if (n >= 16.0) { /* rounded up into the next binade */
+            ++E;
+            n = 8.0;
+        }
+        code = (E << 3) | ((int)n - 8);
+    }
+    return (uint8_t)(sign | code);
+}
+
 /* ---------------------------------------------------------- slot arithmetic */
 
 /* P3 §三, BlockTable::num_required_blocks: ceil(n / B). */
@@ -178,6 +224,36 @@ int pa_oracle_reshape_and_cache(const uint16_t* k, const uint16_t* v, const int6
     return skipped;
 }
 
+/* The cache write into an fp8 cache: each element of k (v) is widened to fp32,
+ * divided by k_scale (v_scale) in fp32 (IEEE, round to nearest) and stored as the
+ * nearest E4M3 code (saturating).  Slots outside [0, num_blocks*block_size) are
+ * skipped; the return value counts them. */
+int pa_oracle_reshape_and_cache_fp8(const uint16_t* k, const uint16_t* v, const int64_t* slot_mapping,
+                                    uint8_t* k_cache, uint8_t* v_cache, int num_tokens, int num_kv_heads,
+                                    int head_dim, int block_size, int num_blocks, int dtype, float k_scale,
+                                    float v_scale) {
+    int skipped = 0;
+    int64_t num_slots = (int64_t)num_blocks * block_size;
+    for (int i = 0; i < num_tokens; ++i) {
+        int64_t slot = slot_mapping[i];
+        if (slot < 0 || slot >= num_slots) {
+            ++skipped;
+            continue;
+        }
+        for (int h = 0; h < num_kv_heads; ++h) {
+            int64_t src = ((int64_t)i * num_kv_heads + h) * head_dim;
+            int64_t dst = (slot * num_kv_heads + h) * head_dim;
+            for (int j = 0; j < head_dim; ++j) {
+                const float kx = (float)widen(k[src + j], dtype) / k_scale;
+                const float vx = (float)widen(v[src + j], dtype) / v_scale;
+                k_cache[dst + j] = pa_oracle_e4m3_from_float(kx);
+                v_cache[dst + j] = pa_oracle_e4m3_from_float(vx);
+            }
+        }
+    }
+    return skipped;
+}
+
 /* ------------------------------------------------------ whole-block copies */
 
 /* For each pair (src, dst): the dst block of both caches becomes a copy of the
@@ -203,6 +279,8 @@ int pa_oracle_copy_blocks(uint16_t* k_cache, uint16_t* v_cache, const int32_t* p
 
 typedef struct {
     const uint16_t *q, *k_cache, *v_cache;
+    const uint8_t *k8, *v8; /* fp8 caches (k_cache / v_cache unused then) */
+    double k_scale, v_scale;
     const int32_t *tables, *context_lens;
     double scale;
     int num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype;
@@ -217,6 +295,14 @@ typedef struct {
     decode_job* job;
     int tid;
 } worker_arg;
+
+/* Value of cache element `idx`: a 16-bit element widened, or an fp8 code times its scale. */
+static double kval(const decode_job* j, int64_t idx) {
+    return j->k8 ? pa_oracle_e4m3_to_double(j->k8[idx]) * j->k_scale : widen(j->k_cache[idx], j->dtype);
+}
+static double vval(const decode_job* j, int64_t idx) {
+    return j->v8 ? pa_oracle_e4m3_to_double(j->v8[idx]) * j->v_scale : widen(j->v_cache[idx], j->dtype);
+}
 
 /* Element offset of (token slot, kv head, 0) in the cache layout above. */
 static int64_t cache_row(const decode_job* j, int64_t phys, int64_t off, int kv_head) {
@@ -257,9 +343,9 @@ static int decode_one(const decode_job* j, int s, int h, double* out, double* qd
         off = (t + 1) % bs; /* planted: off-by-one offset inside the block */
 #endif
         if (phys < 0 || phys >= j->num_blocks) return 1;
-        const uint16_t* krow = j->k_cache + cache_row(j, phys, off, kv_head);
+        const int64_t krow = cache_row(j, phys, off, kv_head);
         double dot = 0.0;
-        for (int i = 0; i < d; ++i) dot += qd[i] * widen(krow[i], j->dtype);
+        for (int i = 0; i < d; ++i) dot += qd[i] * kval(j, krow + i);
 #if PA_ORACLE_MUTANT == 1
         x[t] = dot; /* planted: scale dropped */
 #else
@@ -277,9 +363,9 @@ static int decode_one(const decode_job* j, int s, int h, double* out, double* qd
         for (int64_t t = b0; t < b1; ++t) {
             int64_t phys, off;
             pa_oracle_physical_location(table, j->max_blocks_per_seq, t, bs, &phys, &off);
-            const uint16_t* vrow = j->v_cache + cache_row(j, phys, off, kv_head);
+            const int64_t vrow = cache_row(j, phys, off, kv_head);
             double w = exp(x[t] - m) / den;
-            for (int i = 0; i < d; ++i) out[i] += w * widen(vrow[i], j->dtype);
+            for (int i = 0; i < d; ++i) out[i] += w * vval(j, vrow + i);
         }
     }
     return 0;
@@ -293,10 +379,10 @@ static int decode_one(const decode_job* j, int s, int h, double* out, double* qd
 #if PA_ORACLE_MUTANT == 2
         off = (t + 1) % bs;
 #endif
-        const uint16_t* vrow = j->v_cache + cache_row(j, phys, off, kv_head);
+        const int64_t vrow = cache_row(j, phys, off, kv_head);
         double w = exp(x[t] - m);
         den += w;
-        for (int i = 0; i < d; ++i) out[i] += w * widen(vrow[i], j->dtype);
+        for (int i = 0; i < d; ++i) out[i] += w * vval(j, vrow + i);
     }
 #if PA_ORACLE_MUTANT == 6
     (void)den; /* planted: the softmax denominator is left out */
@@ -339,22 +425,8 @@ static void* decode_worker(void* p) {
     return NULL;
 }
 
-/* Decode attention for every (s, h) (pairs == NULL, out is [S][H][d]) or for the
- * listed (s, h) pairs (out is [npairs][d]).  Returns 0, 1 on a bad argument or an
- * out-of-range table entry / length, 2 on allocation failure. */
-int pa_oracle_decode(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
-                     const int32_t* block_tables, const int32_t* context_lens, double scale, int num_seqs,
-                     int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
-                     int max_blocks_per_seq, int dtype, const int32_t* pairs, int npairs, double* out,
-                     int nthreads) {
-    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
-        head_dim <= 0 || block_size <= 0 || num_blocks < 0 || max_blocks_per_seq < 0 ||
-        (dtype != ORACLE_F16 && dtype != ORACLE_BF16))
-        return 1;
-    if (nthreads < 1) nthreads = 1;
-    decode_job job = {q, k_cache, v_cache, block_tables, context_lens, scale, num_seqs, num_heads,
-                      num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype,
-                      pairs, npairs, out, nthreads, 0};
+static int run_decode(decode_job* job) {
+    int nthreads = job->nthreads;
     pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
     worker_arg* args = (worker_arg*)malloc(sizeof(worker_arg) * (size_t)nthreads);
     if (!th || !args) {
@@ -363,7 +435,7 @@ int pa_oracle_decode(const uint16_t* q, const uint16_t* k_cache, const uint16_t*
         return 2;
     }
     for (int t = 0; t < nthreads; ++t) {
-        args[t].job = &job;
+        args[t].job = job;
         args[t].tid = t;
         if (t > 0) pthread_create(&th[t], NULL, decode_worker, &args[t]);
     }
@@ -371,7 +443,44 @@ int pa_oracle_decode(const uint16_t* q, const uint16_t* k_cache, const uint16_t*
     for (int t = 1; t < nthreads; ++t) pthread_join(th[t], NULL);
     free(th);
     free(args);
-    return job.error;
+    return job->error;
+}
+
+static int bad_sizes(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                     int max_blocks_per_seq, int dtype) {
+    return num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
+           head_dim <= 0 || block_size <= 0 || num_blocks < 0 || max_blocks_per_seq < 0 ||
+           (dtype != ORACLE_F16 && dtype != ORACLE_BF16);
+}
+
+/* Decode attention for every (s, h) (pairs == NULL, out is [S][H][d]) or for the
+ * listed (s, h) pairs (out is [npairs][d]).  Returns 0, 1 on a bad argument or an
+ * out-of-range table entry / length, 2 on allocation failure. */
+int pa_oracle_decode(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                     const int32_t* block_tables, const int32_t* context_lens, double scale, int num_seqs,
+                     int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                     int max_blocks_per_seq, int dtype, const int32_t* pairs, int npairs, double* out,
+                     int nthreads) {
+    if (bad_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype))
+        return 1;
+    decode_job job = {q, k_cache, v_cache, NULL, NULL, 1.0, 1.0, block_tables, context_lens, scale, num_seqs,
+                      num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype,
+                      pairs, npairs, out, nthreads < 1 ? 1 : nthreads, 0};
+    return run_decode(&job);
+}
+
+/* The same over fp8 caches: K = code * k_scale, V = code * v_scale, exactly. */
+int pa_oracle_decode_fp8(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                         const int32_t* block_tables, const int32_t* context_lens, double scale, double k_scale,
+                         double v_scale, int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, int max_blocks_per_seq, int dtype, const int32_t* pairs, int npairs,
+                         double* out, int nthreads) {
+    if (bad_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype))
+        return 1;
+    decode_job job = {q, NULL, NULL, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale,
+                      num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                      dtype, pairs, npairs, out, nthreads < 1 ? 1 : nthreads, 0};
+    return run_decode(&job);
 }
 
 /* Build-time identification for the tests: which mistake (0 = none) is planted. */

@@ -216,6 +216,77 @@ def pin_copy_blocks(o):
     assert np.array_equal(kc, ek) and np.array_equal(vc, ev)
 
 
+# ------------------------------------------------------------ fp8 (E4M3) cache
+
+def pin_e4m3_decoding(o):
+    """All 256 codes against torch's float8_e4m3fn widening."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([o.e4m3_to_double(int(c)) for c in range(256)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    m = ~np.isnan(ref)
+    assert np.array_equal(got[m], ref[m])
+
+
+def pin_e4m3_rounding(o):
+    """Round to nearest even against torch inside the finite range (ties included);
+    saturation to +-448 beyond it (closed form: the largest finite code)."""
+    rng = np.random.default_rng(24)
+    vals = np.concatenate([
+        rng.uniform(-464, 464, 4000), rng.normal(0, 1, 4000), rng.normal(0, 1e-2, 2000),
+        np.ldexp(rng.integers(-60, 60, 2000).astype(np.float64), -12),       # ties and exact values
+        np.array([0.0, -0.0, 448.0, -448.0, 464.0, 2.0 ** -10, 3 * 2.0 ** -11, 2.0 ** -6, 15.0 * 2.0 ** -10]),
+    ]).astype(np.float32)
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([o.e4m3_from_float(float(x)) for x in vals], dtype=np.uint8)
+    assert np.array_equal(got, ref), vals[got != ref][:5]
+    for x, code in ((465.0, 0x7e), (1e30, 0x7e), (float("inf"), 0x7e), (-1e9, 0xfe), (-float("inf"), 0xfe)):
+        assert o.e4m3_from_float(x) == code, x
+    assert o.e4m3_from_float(float("nan")) & 0x7f == 0x7f
+
+
+def pin_reshape_and_cache_fp8(o):
+    """Codes land in their slots: the fp32 quotient rounded by torch, compared per slot."""
+    rng = np.random.default_rng(25)
+    nb, bs, hk, d, n = 5, 16, 2, 64, 7
+    k = to_bits(rng.normal(0, 2, (n, hk, d)), BF16)
+    v = to_bits(rng.normal(0, 2, (n, hk, d)), BF16)
+    kc = np.zeros((nb, bs, hk, d), dtype=np.uint8)
+    vc = np.zeros_like(kc)
+    slots = rng.choice(nb * bs, size=n, replace=False).astype(np.int64)
+    slots[1] = -1
+    ks, vs = np.float32(0.5), np.float32(0.125)
+    assert o.reshape_and_cache_fp8(k, v, slots, kc, vc, BF16, ks, vs) == 1
+    q = lambda x, sc: torch.from_numpy((from_bits(x, BF16).astype(np.float32) / sc).astype(np.float32)) \
+        .to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    for i in range(n):
+        if slots[i] < 0:
+            continue
+        blk, off = divmod(int(slots[i]), bs)
+        assert np.array_equal(kc[blk, off], q(k[i], ks)) and np.array_equal(vc[blk, off], q(v[i], vs))
+    assert np.count_nonzero(kc) <= (n - 1) * hk * d
+
+
+def pin_decode_fp8_matches_16bit_decode(o):
+    """With power-of-two scales every dequantised value is exact in fp16, so decode
+    over the codes equals decode over the dequantised fp16 cache, bit for bit."""
+    rng = np.random.default_rng(26)
+    c = PagedCase(rng, [7, 40, 100], 4, 2, 64, 16, F16, 0.125)
+    k8 = rng.integers(0, 256, size=c.k_cache.shape, dtype=np.uint8)
+    v8 = rng.integers(0, 256, size=c.v_cache.shape, dtype=np.uint8)
+    for arr in (k8, v8):            # keep clear of the NaN codes and of fp16 subnormals after scaling
+        arr[(arr & 0x7f) == 0x7f] = 0x38
+        arr[(arr & 0x78) == 0] = 0x38
+    ks, vs = 0.25, 2.0
+    deq = lambda a, sc: torch.from_numpy(a).view(torch.float8_e4m3fn).to(torch.float64).numpy() * sc
+    kc16 = to_bits(deq(k8, ks), F16)
+    vc16 = to_bits(deq(v8, vs), F16)
+    assert np.array_equal(from_bits(kc16, F16), deq(k8, ks)) and np.array_equal(from_bits(vc16, F16), deq(v8, vs))
+    got = o.decode_fp8(c.q, k8, v8, c.tables, c.lens, c.scale, ks, vs, F16)
+    ref = o.decode(c.q, kc16, vc16, c.tables, c.lens, c.scale, F16)
+    assert np.array_equal(got, ref)
+
+
 # -------------------------------------------------------------------- decode
 
 def pin_decode_one_token(o):
