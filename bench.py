@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--partition-tokens", type=int, default=0)
     p.add_argument("--num-seqs", type=int, default=None, help="truncate the batch (smaller profiling case)")
+    p.add_argument("--kv-dtype", default="native", choices=["native", "fp8"],
+                   help="fp8: the cache is stored as E4M3 codes (pa_reshape_and_cache_fp8 / pa_decode_fp8)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
     p.add_argument("--row", default="decode", choices=["decode", "copy_blocks", "swap"],
@@ -189,7 +191,10 @@ def gpu_uuid(torch, device):
 
 # --------------------------------------------------------------- workload
 
-def build_step(name, device, partition_tokens, num_seqs=None):
+FP8_INV_SCALE = 32.0  # fp8 caches: stored value = code / 32 (N(0,1) values use codes up to ~150)
+
+
+def build_step(name, device, partition_tokens, num_seqs=None, kv_dtype="native"):
     """Tables from the library's allocator, one step's slots via a1, tensors on
     the device.  Returns a dict of everything the timed loop needs."""
     import torch
@@ -218,6 +223,10 @@ def build_step(name, device, partition_tokens, num_seqs=None):
     slots = alloc.append_slots(tables, lens, bs)
     a1_us = (time.perf_counter() - t0) * 1e6
     t = wk.make_tensors(wl, device=device)
+    if kv_dtype == "fp8":
+        import torch
+        for key in ("k_cache", "v_cache"):
+            t[key] = (t[key].float() * FP8_INV_SCALE).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
     ws_bytes = pa.pa_decode_workspace_size(s, spec.num_heads, spec.num_kv_heads, spec.head_dim, bs,
                                            wl.max_blocks_per_seq, partition_tokens)
     d = dict(
@@ -235,9 +244,10 @@ def algorithmic_bytes(st):
     and the partials written by K2 and read by K3."""
     spec, wl = st["spec"], st["wl"]
     lens = st["lens_h"].astype(np.int64)
-    e = 2
+    e = 2                                  # q and out elements
+    ec = st["k_cache"].element_size()      # cache elements (1 for fp8 codes)
     hk, d, h, s, bs = spec.num_kv_heads, spec.head_dim, spec.num_heads, spec.num_seqs, spec.block_size
-    row = 2 * hk * d * e  # K and V of one token, all kv heads
+    row = 2 * hk * d * ec  # K and V of one token, all kv heads
     if spec.prefix_tokens:
         unique_tokens = spec.prefix_tokens + int(np.sum(lens - spec.prefix_tokens))
     else:
@@ -251,7 +261,7 @@ def algorithmic_bytes(st):
     qo = 2 * s * h * d * e
     return {"unique": unique_tokens * row + qo + meta + partials,
             "logical": logical_tokens * row + qo + meta + partials,
-            "unique_tokens": unique_tokens, "k1": 2 * s * hk * d * e * 2 + 8 * s}
+            "unique_tokens": unique_tokens, "k1": 2 * s * hk * d * (e + ec) + 8 * s}
 
 
 def static_config(wl, args, world):
@@ -283,15 +293,30 @@ def run_native(args):
                                 timeout=__import__("datetime").timedelta(seconds=120))
     device = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(device)
-    st = build_step(args.workload, device, args.partition_tokens, args.num_seqs)
+    st = build_step(args.workload, device, args.partition_tokens, args.num_seqs, args.kv_dtype)
+    fp8 = args.kv_dtype == "fp8"
+    ks = vs = 1.0 / FP8_INV_SCALE
     spec = st["spec"]
     stream = torch.cuda.current_stream(device)
 
+    def k1(k, v, slots):
+        if fp8:
+            pa.pa_reshape_and_cache_fp8(k, v, slots, st["k_cache"], st["v_cache"], ks, vs, stream=stream)
+        else:
+            pa.pa_reshape_and_cache(k, v, slots, st["k_cache"], st["v_cache"], stream=stream)
+
+    def k2(q, tables, lens):
+        if fp8:
+            pa.pa_decode_fp8(q, st["k_cache"], st["v_cache"], tables, lens, spec.scale, ks, vs, spec.num_kv_heads,
+                             st["out"], workspace=st["workspace"], partition_tokens=st["partition_tokens"],
+                             stream=stream)
+        else:
+            pa.pa_decode(q, st["k_cache"], st["v_cache"], tables, lens, spec.scale, spec.num_kv_heads, st["out"],
+                         workspace=st["workspace"], partition_tokens=st["partition_tokens"], stream=stream)
+
     def step():
-        pa.pa_reshape_and_cache(st["k"], st["v"], st["slots"], st["k_cache"], st["v_cache"], stream=stream)
-        pa.pa_decode(st["q"], st["k_cache"], st["v_cache"], st["tables"], st["lens"], spec.scale,
-                     spec.num_kv_heads, st["out"], workspace=st["workspace"],
-                     partition_tokens=st["partition_tokens"], stream=stream)
+        k1(st["k"], st["v"], st["slots"])
+        k2(st["q"], st["tables"], st["lens"])
 
     def barrier():
         if world > 1:
@@ -313,12 +338,10 @@ def run_native(args):
     start.record(stream)
     for i in range(args.steps):
         k1_ev[i][0].record(stream)
-        pa.pa_reshape_and_cache(st["k"], st["v"], st["slots"], st["k_cache"], st["v_cache"], stream=stream)
+        k1(st["k"], st["v"], st["slots"])
         k1_ev[i][1].record(stream)
         k2_ev[i][0].record(stream)
-        pa.pa_decode(st["q"], st["k_cache"], st["v_cache"], st["tables"], st["lens"], spec.scale,
-                     spec.num_kv_heads, st["out"], workspace=st["workspace"],
-                     partition_tokens=st["partition_tokens"], stream=stream)
+        k2(st["q"], st["tables"], st["lens"])
         k2_ev[i][1].record(stream)
     stop.record(stream)
     barrier()
@@ -340,11 +363,8 @@ def run_native(args):
     def e2e_step():
         for k, v in host.items():
             dev_in[k].copy_(v, non_blocking=True)
-        pa.pa_reshape_and_cache(dev_in["k"], dev_in["v"], dev_in["slots"], st["k_cache"], st["v_cache"],
-                                stream=stream)
-        pa.pa_decode(dev_in["q"], st["k_cache"], st["v_cache"], dev_in["tables"], dev_in["lens"], spec.scale,
-                     spec.num_kv_heads, st["out"], workspace=st["workspace"],
-                     partition_tokens=st["partition_tokens"], stream=stream)
+        k1(dev_in["k"], dev_in["v"], dev_in["slots"])
+        k2(dev_in["q"], dev_in["tables"], dev_in["lens"])
         out_h.copy_(st["out"], non_blocking=True)
 
     e2e_steps = max(1, min(args.steps, 500))
@@ -382,9 +402,9 @@ def run_native(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": spec.dtype,
+        "dtype": spec.dtype + ("+e4m3 cache" if fp8 else ""),
         "data": "synthetic",
-        "config": static_config(st["wl"], args, world),
+        "config": dict(static_config(st["wl"], args, world), **({"kv_cache": "fp8 e4m3, scale 1/32"} if fp8 else {})),
         "detail": {
             "kv_gbs": round(achieved, 1), "frac_of_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
             "kv_bytes_per_step": ab["unique"], "logical_kv_bytes_per_step": ab["logical"],
@@ -395,7 +415,7 @@ def run_native(args):
             "kernel": "paged_decode_mha_kernel + paged_decode_merge_kernel (timed together: one pa_decode call)",
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
             "unit": "GB/s", "frac": round(achieved / peak, 4),
-            "traffic": profiled_traffic(ab["unique_tokens"]),
+            "traffic": None if fp8 else profiled_traffic(ab["unique_tokens"]),
         },
         "e2e": {"value": round(job_throughput(world, tokens_per_step, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

@@ -180,6 +180,43 @@ int pa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, c
                       int num_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
                       int dtype, int partition_tokens, int32_t* err_word, void* stream);
 
+/* ---------------------------------------------------------------- fp8 cache */
+
+/*
+ * fp8 (E4M3) KV cache: half the bytes per token.  The pages point at quantising
+ * the cache (P1, closing note; P2 §5, memory -64% "with quantisation") without
+ * fixing a format; this library stores OCP E4M3 codes ("e4m3fn": 1 sign, 4
+ * exponent bits with bias 7, 3 fraction bits, no infinities, largest finite value
+ * 448) with one fp32 scale per cache: the stored value of an element is
+ * code * k_scale (code * v_scale).  Caches are uint8
+ * [num_blocks][block_size][num_kv_heads][head_dim]; q, k, v and out stay fp16 or bf16.
+ */
+
+/*
+ * pa_reshape_and_cache_fp8 -- pa_reshape_and_cache into fp8 caches.  Each element
+ * x of k (v) is stored as the E4M3 code nearest to x / k_scale (x / v_scale),
+ * the quotient taken in fp32 (IEEE division, round to nearest) and then rounded to
+ * nearest even, saturating at +-448 (NaN stays NaN).  Scales must be positive and
+ * finite.  head_dim must be a multiple of 16.
+ */
+int pa_reshape_and_cache_fp8(const void* k, const void* v, const int64_t* slot_mapping, void* k_cache,
+                             void* v_cache, int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                             int num_blocks, int dtype, float k_scale, float v_scale, int32_t* err_word,
+                             void* stream);
+
+/*
+ * pa_decode_fp8 -- pa_decode over fp8 caches: the same softmax(scale * q K^T) V
+ * with K = code * k_scale and V = code * v_scale, in fp32 (the codes widen
+ * exactly; k_scale is folded into q, v_scale into the result).  head_dim 128 only;
+ * every other argument, the workspace and the errors as pa_decode.  Query heads
+ * are computed on CUDA cores one per unit (a GQA group shares its K/V through L2).
+ */
+int pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                  const int32_t* context_lens, float scale, float k_scale, float v_scale, int num_kv_heads, void* out,
+                  int num_seqs, int num_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                  int dtype, int partition_tokens, void* workspace, size_t workspace_bytes, int32_t* err_word,
+                  void* stream);
+
 /* ---------------------------------------------------------- host allocator */
 
 /*

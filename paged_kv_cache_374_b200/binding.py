@@ -46,6 +46,10 @@ _sig("pa_decode", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32
      _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
 _sig("pa_decode_noalloc", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32, _i32, _i32, _i32, _i32,
      _i32, _i32, _i32, _vp, _vp)
+_sig("pa_reshape_and_cache_fp8", _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_float,
+     ctypes.c_float, _vp, _vp)
+_sig("pa_decode_fp8", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float, ctypes.c_float, _i32, _vp, _i32,
+     _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
 _sig("pa_allocator_create", _vp, _i32, _i32p)
 _sig("pa_allocator_destroy", None, _vp)
 _sig("pa_num_required_blocks", _i32, _i32, _i32)
@@ -195,6 +199,50 @@ def pa_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, nu
                                 _dev(out, "out"), s, h, d, bs, nb, block_tables.shape[1], dt,
                                 int(partition_tokens), _dev(err_word, "err_word", torch.int32), _stream(stream, q))
     _check(st, "pa_decode_noalloc")
+    return out
+
+
+def pa_reshape_and_cache_fp8(k, v, slot_mapping, k_cache, v_cache, k_scale, v_scale, err_word=None, stream=None):
+    """K1 into fp8 caches.  k, v fp16/bf16 [N, Hk, d]; caches uint8 (E4M3 codes) [NB, B, Hk, d]."""
+    import torch
+    n, hk, d = k.shape
+    nb, bs, hk2, d2 = k_cache.shape
+    if v.shape != k.shape or v_cache.shape != k_cache.shape or (hk2, d2) != (hk, d):
+        raise ValueError("shape mismatch")
+    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+        raise TypeError("fp8 caches are uint8 tensors of E4M3 codes")
+    dt = _dtype_code(k)
+    st = _lib.pa_reshape_and_cache_fp8(_dev(k, "k", k.dtype), _dev(v, "v", k.dtype),
+                                       _dev(slot_mapping, "slot_mapping", torch.int64), _dev(k_cache, "k_cache"),
+                                       _dev(v_cache, "v_cache"), n, hk, d, bs, nb, dt, float(k_scale), float(v_scale),
+                                       _dev(err_word, "err_word", torch.int32), _stream(stream, k))
+    _check(st, "pa_reshape_and_cache_fp8")
+
+
+def pa_decode_fp8(q, k_cache, v_cache, block_tables, context_lens, scale, k_scale, v_scale, num_kv_heads, out,
+                  workspace=None, partition_tokens=0, err_word=None, stream=None):
+    """K2 + K3 over fp8 caches (uint8 E4M3 codes [NB, B, Hk, d]); q / out fp16 or bf16."""
+    import torch
+    s, h, d = q.shape
+    nb, bs, hk, d2 = k_cache.shape
+    if hk != num_kv_heads or d2 != d or v_cache.shape != k_cache.shape or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+        raise TypeError("fp8 caches are uint8 tensors of E4M3 codes")
+    if out.dtype != q.dtype:
+        raise TypeError("q and out must share one dtype")
+    mb = block_tables.shape[1]
+    dt = _dtype_code(q)
+    need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = _lib.pa_decode_fp8(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                            _dev(block_tables, "block_tables", torch.int32),
+                            _dev(context_lens, "context_lens", torch.int32), float(scale), float(k_scale),
+                            float(v_scale), hk, _dev(out, "out"), s, h, d, bs, nb, mb, dt, int(partition_tokens),
+                            _dev(workspace, "workspace"), workspace.numel(), _dev(err_word, "err_word", torch.int32),
+                            _stream(stream, q))
+    _check(st, "pa_decode_fp8")
     return out
 
 

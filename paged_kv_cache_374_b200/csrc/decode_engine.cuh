@@ -47,6 +47,8 @@ struct DecodeArgs {
     int32_t* sched;   // [0] claim counter, [1] finished-warp counter; zero between launches
     int32_t* err_word;
     float scale_log2; // scale * log2(e)
+    float k_scale;    // fp8 caches: K = code * k_scale (1 for 16-bit caches)
+    float v_scale;    // fp8 caches: V = code * v_scale (1 for 16-bit caches)
     int num_seqs;     // sequences in this launch (<= kMaxSeqsPerLaunch)
     int num_heads;    // query heads
     int group;        // num_heads / num_kv_heads
@@ -68,9 +70,10 @@ struct Unit {
     int t_begin, t_end, nst, kv_head, blk0, nblk;
 };
 
-template <int D, int TOK, int NW, int R>
+// ROWB: bytes of one token's row of one kv head (head_dim * element size)
+template <int ROWB, int TOK, int NW, int R>
 struct Layout {
-    static constexpr int kTileBytes = TOK * D * 2;
+    static constexpr int kTileBytes = TOK * ROWB;
     static constexpr int kHalfBytes = TOK * 128;               // one 64-dim half tile
     static constexpr int kSlotBytes = 2 * kTileBytes;          // K tile then V tile
     static constexpr int kOffSlots = 0;
@@ -164,11 +167,13 @@ __device__ __forceinline__ void write_special_rows(const DecodeArgs& a, const Un
     if (U.kind == kUnitNaN && lane == 0) report(a.err_word, PA_DEVERR_LEN_RANGE);
 }
 
-template <class Tag, int D, int TOK, int NW, int R, class Policy>
+template <class Tag, class CTag, int D, int TOK, int NW, int R, class Policy>
 __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeArgs a,
                                                                   const __grid_constant__ CUtensorMap kmap,
                                                                   const __grid_constant__ CUtensorMap vmap) {
-    using Lay = Layout<D, TOK, NW, R>;
+    constexpr int ROWB = D * CTag::kBytes;      // bytes per token row of one kv head
+    static_assert(ROWB % 128 == 0, "rows are loaded as 128-byte swizzled boxes");
+    using Lay = Layout<ROWB, TOK, NW, R>;
     constexpr int MAXSUB = TOK / 8 > 2 ? 2 : 1;  // TMA boxes per half tile (box_rows >= TOK/2)
 
     extern __shared__ uint8_t smem_raw[];
@@ -296,7 +301,7 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
             phys[j] = __shfl_sync(kFullMask, v, e & 31);
             if (use) {
                 bad |= phys[j] < 0 || phys[j] >= a.num_blocks;
-                tx += 2u * br * D * 2;
+                tx += 2u * br * ROWB;
             }
         }
         uint8_t* dst = slots + slot * Lay::kSlotBytes;
@@ -314,10 +319,11 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
                     if (j * br < TOK && tj < I.t_end) {
                         const int row = phys[j] * bs + (tj % bs);
 #pragma unroll
-                        for (int hh = 0; hh < D / 64; ++hh) {
+                        for (int hh = 0; hh < ROWB / 128; ++hh) {
                             uint8_t* kd = dst + hh * Lay::kHalfBytes + j * br * 128;
-                            tma_load_3d(kd, &kmap, hh * 64, I.kv_head, row, &bars[slot]);
-                            tma_load_3d(kd + Lay::kTileBytes, &vmap, hh * 64, I.kv_head, row, &bars[slot]);
+                            const int x = hh * (128 / CTag::kBytes);
+                            tma_load_3d(kd, &kmap, x, I.kv_head, row, &bars[slot]);
+                            tma_load_3d(kd + Lay::kTileBytes, &vmap, x, I.kv_head, row, &bars[slot]);
                         }
                     }
                 }

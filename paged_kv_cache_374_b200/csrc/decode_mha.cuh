@@ -21,10 +21,13 @@
 
 namespace pa {
 
-template <class Tag, int D, int TOK>
+// Tag: q / out element type; CTag: cache element type (16-bit, or E4M3 codes whose
+// scales are folded into q (k_scale) and into the result (v_scale)).
+template <class Tag, class CTag, int D, int TOK>
 struct MhaPolicy {
     static constexpr int DL = D / 4;       // dims per lane
-    static constexpr int NCH = DL / 8;     // 16-byte chunks per lane per row
+    static constexpr int EPC = 16 / CTag::kBytes;  // cache elements per 16-byte chunk
+    static constexpr int NCH = DL / EPC;   // 16-byte chunks per lane per row
     static constexpr int NROW = TOK / 8;   // rows per lane per stage
     static_assert(NROW == 1 || NROW == 2 || NROW == 4, "stage shape");
     static constexpr int DUP = 4 / NROW;   // lanes that end up holding one token's score
@@ -32,7 +35,7 @@ struct MhaPolicy {
 
     int lane, r, c;
     int swz[NCH];       // offset of this lane's chunk j of row r in a tile
-    uint4 qn[NCH];      // raw q of the next unit
+    uint4 qn[DL / 8];   // raw q of the next unit
     float2 qc[DL / 2];  // q of the current unit, pre-scaled by scale * log2(e)
     float m, lsum;
     float2 o[DL / 2];
@@ -42,8 +45,9 @@ struct MhaPolicy {
         lane = lane_;
         r = lane & 7;
         c = lane >> 3;
-        const int lane_half = (D == 128) ? (c >> 1) : 0;
-        const int chunk0 = (D == 128) ? (c & 1) * 4 : c * 2;
+        const int lane_byte = c * DL * CTag::kBytes;  // this lane's first byte in a row
+        const int lane_half = lane_byte / 128;
+        const int chunk0 = (lane_byte % 128) / 16;
 #pragma unroll
         for (int j = 0; j < NCH; ++j) swz[j] = lane_half * HALF_BYTES + r * 128 + (((chunk0 + j) ^ r) << 4);
     }
@@ -52,16 +56,31 @@ struct MhaPolicy {
         if (U.kind != kUnitNormal) return;
         const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)U.s * a.num_heads + U.h) * D + c * DL);
 #pragma unroll
-        for (int j = 0; j < NCH; ++j) qn[j] = __ldg(src + j);
+        for (int j = 0; j < DL / 8; ++j) qn[j] = __ldg(src + j);
     }
 
     __device__ __forceinline__ void take_q(const DecodeArgs& a) {
+        const float sc = a.scale_log2 * a.k_scale;
 #pragma unroll
-        for (int j = 0; j < NCH; ++j) {
+        for (int j = 0; j < DL / 8; ++j) {
             float2 f[4];
             widen8<Tag>(qn[j], f);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) qc[j * 4 + k] = make_float2(f[k].x * a.scale_log2, f[k].y * a.scale_log2);
+            for (int k = 0; k < 4; ++k) qc[j * 4 + k] = make_float2(f[k].x * sc, f[k].y * sc);
+        }
+    }
+
+    // the EPC cache values of a 16-byte chunk as EPC/2 float pairs
+    static __device__ __forceinline__ void widen_chunk(const uint4& w, float2 (&f)[EPC / 2]) {
+        if constexpr (CTag::kBytes == 2) {
+            widen8<CTag>(w, f);
+        } else {
+            const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                f[2 * k] = CTag::widen2(words[k] & 0xffffu);
+                f[2 * k + 1] = CTag::widen2(words[k] >> 16);
+            }
         }
     }
 
@@ -85,10 +104,10 @@ struct MhaPolicy {
 #pragma unroll
             for (int j = 0; j < NCH; ++j) {
                 const uint4 w = *reinterpret_cast<const uint4*>(kt + i * 1024 + swz[j]);
-                float2 kf[4];
-                widen8<Tag>(w, kf);
+                float2 kf[EPC / 2];
+                widen_chunk(w, kf);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) d2 = __ffma2_rn(qc[j * 4 + k], kf[k], d2);
+                for (int k = 0; k < EPC / 2; ++k) d2 = __ffma2_rn(qc[j * (EPC / 2) + k], kf[k], d2);
             }
             acc[i] = d2.x + d2.y;
         }
@@ -136,10 +155,10 @@ struct MhaPolicy {
 #pragma unroll
                 for (int j = 0; j < NCH; ++j) {
                     const uint4 w = *reinterpret_cast<const uint4*>(vt + i * 1024 + swz[j]);
-                    float2 vf[4];
-                    widen8<Tag>(w, vf);
+                    float2 vf[EPC / 2];
+                    widen_chunk(w, vf);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) o[j * 4 + k] = __ffma2_rn(p2, vf[k], o[j * 4 + k]);
+                    for (int k = 0; k < EPC / 2; ++k) o[j * (EPC / 2) + k] = __ffma2_rn(p2, vf[k], o[j * (EPC / 2) + k]);
                 }
             }
         }
@@ -158,12 +177,16 @@ struct MhaPolicy {
         }
         float l = warp_sum(lsum) * (1.f / DUP);
         if (__any_sync(kFullMask, poisoned)) l = __int_as_float(0x7fc00000);
+        if (CTag::kBytes == 1) {
+#pragma unroll
+            for (int k = 0; k < DL / 2; ++k) o[k] = make_float2(o[k].x * a.v_scale, o[k].y * a.v_scale);
+        }
         if (U.np == 1) {
             if (r == 0) {
                 const float inv = 1.f / l;
                 uint4* dst = reinterpret_cast<uint4*>(a.out + sh * D + c * DL);
 #pragma unroll
-                for (int j = 0; j < NCH; ++j) {
+                for (int j = 0; j < DL / 8; ++j) {
                     uint4 w;
                     w.x = pack2<Tag>(o[j * 4 + 0].x * inv, o[j * 4 + 0].y * inv);
                     w.y = pack2<Tag>(o[j * 4 + 1].x * inv, o[j * 4 + 1].y * inv);

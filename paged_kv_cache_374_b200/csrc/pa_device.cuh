@@ -16,6 +16,7 @@ namespace pa {
 
 struct F16Tag {
     using T = __half;
+    static constexpr int kBytes = 2;
     // widen two packed 16-bit values (low half first) to fp32
     static __device__ __forceinline__ float2 widen2(uint32_t w) {
         return __half22float2(*reinterpret_cast<const __half2*>(&w));
@@ -28,6 +29,7 @@ struct F16Tag {
 
 struct BF16Tag {
     using T = __nv_bfloat16;
+    static constexpr int kBytes = 2;
     static __device__ __forceinline__ float2 widen2(uint32_t w) {
         // a bfloat16 is the top half of a binary32: widening is a shift
         return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
@@ -45,6 +47,25 @@ __device__ __forceinline__ float fast_exp2(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+
+// OCP FP8 E4M3 cache elements (1 byte).  Widening goes through the hardware's exact
+// e4m3x2 -> f16x2 conversion, then f16 -> f32 (both exact).
+struct E4M3Tag {
+    static constexpr int kBytes = 1;
+    // widen two packed codes (low byte first) to fp32
+    static __device__ __forceinline__ float2 widen2(uint32_t pair16) {
+        uint32_t h;
+        const unsigned short in = (unsigned short)pair16;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(in));
+        return __half22float2(*reinterpret_cast<const __half2*>(&h));
+    }
+    // nearest codes of two floats (round to nearest even, saturating at +-448), lo in the low byte
+    static __device__ __forceinline__ uint32_t encode2(float lo, float hi) {
+        unsigned short d;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+        return d;
+    }
+};
 
 // ------------------------------------------------------------------- error word
 

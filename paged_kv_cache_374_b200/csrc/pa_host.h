@@ -48,19 +48,21 @@ inline bool encode_cache_map(CUtensorMap* map, const void* base, int head_dim, i
     return r == CUDA_SUCCESS;
 }
 
-// Same view, boxes of 64 elements (128 bytes) x box_rows with the 128-byte TMA
+// Same view, boxes of 128 bytes (64 16-bit or 128 8-bit elements) x box_rows with the 128-byte TMA
 // swizzle: 16-byte chunk j of box row r lands at chunk j ^ (r % 8) of that row in
 // shared memory, so reading one chunk column of 8 consecutive rows touches all 32
 // banks once.  A head_dim of 128 is loaded as two such boxes (x = 0 and x = 64).
 inline bool encode_cache_map_swizzled(CUtensorMap* map, const void* base, int head_dim, int num_kv_heads,
-                                      int64_t total_tokens, int box_rows) {
+                                      int64_t total_tokens, int box_rows, int elem_bytes = 2) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
+    const cuuint64_t eb = (cuuint64_t)elem_bytes;
     cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads, (cuuint64_t)total_tokens};
-    cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)num_kv_heads * head_dim * 2};
-    cuuint32_t box[3] = {64u, 1u, (cuuint32_t)box_rows};
+    cuuint64_t strides[2] = {(cuuint64_t)head_dim * eb, (cuuint64_t)num_kv_heads * head_dim * eb};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / eb), 1u, (cuuint32_t)box_rows};
     cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = enc(map, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 3,
+                     const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;

@@ -162,19 +162,19 @@ int sm_count() {
     return n;
 }
 
-template <class Tag, int D, int TOK, int NW, int R, class Policy>
+template <class Tag, class CTag, int D, int TOK, int NW, int R, class Policy>
 int launch_engine(DecodeArgs args, const void* k_cache, const void* v_cache, int num_kv_heads,
                   cudaStream_t stream) {
-    using Lay = Layout<D, TOK, NW, R>;
+    using Lay = Layout<D * CTag::kBytes, TOK, NW, R>;
     static_assert(Lay::kAlloc <= 227 * 1024, "shared memory");
     static std::atomic<uint64_t> smem_done{0};
-    auto kernel = paged_decode_kernel<Tag, D, TOK, NW, R, Policy>;
+    auto kernel = paged_decode_kernel<Tag, CTag, D, TOK, NW, R, Policy>;
     if (ensure_smem_limit(kernel, Lay::kAlloc, smem_done) != cudaSuccess) return PA_ERR_CUDA;
     args.box_rows = TOK < args.block_size ? TOK : args.block_size;
     const int64_t total_tokens = (int64_t)args.num_blocks * args.block_size;
     CUtensorMap kmap, vmap;
-    if (!encode_cache_map_swizzled(&kmap, k_cache, D, num_kv_heads, total_tokens, args.box_rows) ||
-        !encode_cache_map_swizzled(&vmap, v_cache, D, num_kv_heads, total_tokens, args.box_rows))
+    if (!encode_cache_map_swizzled(&kmap, k_cache, D, num_kv_heads, total_tokens, args.box_rows, CTag::kBytes) ||
+        !encode_cache_map_swizzled(&vmap, v_cache, D, num_kv_heads, total_tokens, args.box_rows, CTag::kBytes))
         return PA_ERR_CUDA;
     const int sms = sm_count();
     if (sms <= 0) return PA_ERR_CUDA;
@@ -220,18 +220,29 @@ int launch_decode(DecodeArgs args, const void* k_cache, const void* v_cache, int
         args.unit_heads = num_kv_heads;
         args.heads_per_unit = args.group;
         if (args.group <= 8)
-            return launch_engine<Tag, D, TOK, PA_GQA_WARPS, GR, GqaPolicy<Tag, D, TOK, 1>>(args, k_cache, v_cache,
-                                                                                           num_kv_heads, stream);
+            return launch_engine<Tag, Tag, D, TOK, PA_GQA_WARPS, GR, GqaPolicy<Tag, D, TOK, 1>>(
+                args, k_cache, v_cache, num_kv_heads, stream);
         // two head tiles need more registers per thread: at most 8 warps per CTA
         constexpr int NW2 = PA_GQA_WARPS < 8 ? PA_GQA_WARPS : 8;
-        return launch_engine<Tag, D, TOK, NW2, GR, GqaPolicy<Tag, D, TOK, 2>>(args, k_cache, v_cache, num_kv_heads,
-                                                                              stream);
+        return launch_engine<Tag, Tag, D, TOK, NW2, GR, GqaPolicy<Tag, D, TOK, 2>>(args, k_cache, v_cache,
+                                                                                   num_kv_heads, stream);
     }
     constexpr int TOK = D == 128 ? PA_DECODE_TOK128 : PA_DECODE_TOK64;
     args.unit_heads = args.num_heads;
     args.heads_per_unit = 1;
-    return launch_engine<Tag, D, TOK, PA_DECODE_WARPS, R, MhaPolicy<Tag, D, TOK>>(args, k_cache, v_cache,
-                                                                                  num_kv_heads, stream);
+    return launch_engine<Tag, Tag, D, TOK, PA_DECODE_WARPS, R, MhaPolicy<Tag, Tag, D, TOK>>(args, k_cache, v_cache,
+                                                                                            num_kv_heads, stream);
+}
+
+// fp8 (E4M3) caches: CUDA cores, one query head per unit, 32-token slots (8 KiB)
+template <class Tag>
+int launch_decode_fp8(DecodeArgs args, const void* k_cache, const void* v_cache, int num_kv_heads,
+                      cudaStream_t stream) {
+    constexpr int TOK = 32;
+    args.unit_heads = args.num_heads;
+    args.heads_per_unit = 1;
+    return launch_engine<Tag, E4M3Tag, 128, TOK, PA_DECODE_WARPS, PA_DECODE_SLOTS, MhaPolicy<Tag, E4M3Tag, 128, TOK>>(
+        args, k_cache, v_cache, num_kv_heads, stream);
 }
 
 }  // namespace
@@ -258,12 +269,15 @@ extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_
     return pa::workspace_bytes_for((int64_t)num_seqs * num_heads, P, head_dim);
 }
 
-extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
-                         const int32_t* context_lens, float scale, int num_kv_heads, void* out, int num_seqs,
-                         int num_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
-                         int dtype, int partition_tokens, void* workspace, size_t workspace_bytes,
-                         int32_t* err_word, void* stream) {
-    using namespace pa;
+namespace pa {
+namespace {
+
+// Checks shared by pa_decode and pa_decode_fp8; fills args on success.
+int prepare_decode(DecodeArgs& args, const void* q, const void* k_cache, const void* v_cache,
+                   const int32_t* block_tables, const int32_t* context_lens, float scale, int num_kv_heads,
+                   void* out, int num_seqs, int num_heads, int head_dim, int block_size, int num_blocks,
+                   int max_blocks_per_seq, int dtype, int partition_tokens, void* workspace,
+                   size_t workspace_bytes, int32_t* err_word) {
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
         num_blocks <= 0 || max_blocks_per_seq <= 0 || partition_tokens < 0 || partition_tokens % 64 != 0 ||
         partition_tokens > kMaxPartitionTokens)
@@ -292,7 +306,7 @@ extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache
     const size_t need = workspace_bytes_for(SH, P, head_dim);
     if (workspace_bytes < need) return PA_ERR_INVALID_ARG;
 
-    DecodeArgs args{};
+    args = DecodeArgs{};
     args.q = static_cast<const uint16_t*>(q);
     args.out = static_cast<uint16_t*>(out);
     args.block_tables = block_tables;
@@ -306,6 +320,8 @@ extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache
     }
     args.err_word = err_word;
     args.scale_log2 = scale * 1.4426950408889634f;
+    args.k_scale = 1.f;
+    args.v_scale = 1.f;
     args.num_seqs = num_seqs;
     args.num_heads = num_heads;
     args.group = num_heads / num_kv_heads;
@@ -314,10 +330,47 @@ extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache
     args.max_blocks_per_seq = max_blocks_per_seq;
     args.partition_tokens = ptok;
     args.num_partitions = (int)P;
+    return -1;  // ready to launch
+}
+
+}  // namespace
+}  // namespace pa
+
+extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                         const int32_t* context_lens, float scale, int num_kv_heads, void* out, int num_seqs,
+                         int num_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                         int dtype, int partition_tokens, void* workspace, size_t workspace_bytes,
+                         int32_t* err_word, void* stream) {
+    using namespace pa;
+    DecodeArgs args;
+    const int rc = prepare_decode(args, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out,
+                                  num_seqs, num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype,
+                                  partition_tokens, workspace, workspace_bytes, err_word);
+    if (rc >= 0) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (head_dim == 128)
         return dtype == PA_F16 ? launch_decode<F16Tag, 128>(args, k_cache, v_cache, num_kv_heads, st)
                                : launch_decode<BF16Tag, 128>(args, k_cache, v_cache, num_kv_heads, st);
     return dtype == PA_F16 ? launch_decode<F16Tag, 64>(args, k_cache, v_cache, num_kv_heads, st)
                            : launch_decode<BF16Tag, 64>(args, k_cache, v_cache, num_kv_heads, st);
+}
+
+extern "C" int pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                             const int32_t* context_lens, float scale, float k_scale, float v_scale,
+                             int num_kv_heads, void* out, int num_seqs, int num_heads, int head_dim, int block_size,
+                             int num_blocks, int max_blocks_per_seq, int dtype, int partition_tokens,
+                             void* workspace, size_t workspace_bytes, int32_t* err_word, void* stream) {
+    using namespace pa;
+    if (head_dim != 128) return PA_ERR_UNSUPPORTED;  // 128-byte rows: one swizzled TMA box per row
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !isfinite(k_scale) || !isfinite(v_scale)) return PA_ERR_INVALID_ARG;
+    DecodeArgs args;
+    const int rc = prepare_decode(args, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out,
+                                  num_seqs, num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype,
+                                  partition_tokens, workspace, workspace_bytes, err_word);
+    if (rc >= 0) return rc;
+    args.k_scale = k_scale;
+    args.v_scale = v_scale;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return dtype == PA_F16 ? launch_decode_fp8<F16Tag>(args, k_cache, v_cache, num_kv_heads, st)
+                           : launch_decode_fp8<BF16Tag>(args, k_cache, v_cache, num_kv_heads, st);
 }
