@@ -10,6 +10,8 @@ Functions and what they follow (page titles are given in full in pa_oracle.c):
   reshape_and_cache    new K/V rows copied into their slots, bit for bit (P2 §2.1)
   copy_blocks          whole-block copies for copy-on-write after a fork (P3 §四)
   reshape_and_cache_fp8 / decode_fp8 / e4m3_*   the fp8 (E4M3) cache variant
+  prefill              causal attention of a chunk of new query tokens over the paged
+                       cache (the step before decode, P2 §2.1 steps 1-2)
   slot_mapping         slot of the newest token through the table (P3 §三)
   physical_location    token -> (table[idx // B], idx % B)  (P3 §三)
   num_required_blocks  ceil(n / B)  (P3 §三)
@@ -76,6 +78,9 @@ class Oracle:
         lib.pa_oracle_decode_fp8.restype = ctypes.c_int
         lib.pa_oracle_decode_fp8.argtypes = ([_c_u16p, _c_u8p, _c_u8p, _c_i32p, _c_i32p] + [ctypes.c_double] * 3
                                              + [ctypes.c_int] * 8 + [_c_i32p, ctypes.c_int, _c_f64p, ctypes.c_int])
+        lib.pa_oracle_prefill.restype = ctypes.c_int
+        lib.pa_oracle_prefill.argtypes = ([_c_u16p, _c_u16p, _c_u16p, _c_i32p, _c_i32p, _c_i32p, ctypes.c_double]
+                                          + [ctypes.c_int] * 8 + [_c_f64p, ctypes.c_int])
         lib.pa_oracle_mutant_id.restype = ctypes.c_int
         lib.pa_oracle_mutant_id.argtypes = []
         self._lib = lib
@@ -156,6 +161,30 @@ class Oracle:
         return self._lib.pa_oracle_reshape_and_cache_fp8(_ptr(k, _c_u16p), _ptr(v, _c_u16p), _ptr(slots, _c_i64p),
                                                          _ptr(k_cache, _c_u8p), _ptr(v_cache, _c_u8p), num_tokens,
                                                          hk, d, bs, nb, dtype, float(k_scale), float(v_scale))
+
+    def prefill(self, q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, block_tables: np.ndarray,
+                context_lens: np.ndarray, query_start: np.ndarray, scale: float, dtype: int,
+                nthreads: int = 1) -> np.ndarray:
+        """fp64 causal prefill.  q uint16 [T, H, d] packed by sequence (query_start [S+1]);
+        query row i of sequence s sits at position context_lens[s] - n_s + i.  Returns [T, H, d]."""
+        for a in (q, k_cache, v_cache):
+            assert a.dtype == np.uint16 and a.flags.c_contiguous
+        total, num_heads, d = q.shape
+        nb, bs, hk, d2 = k_cache.shape
+        assert d2 == d and v_cache.shape == k_cache.shape
+        tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+        lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+        qs = np.ascontiguousarray(query_start, dtype=np.int32)
+        num_seqs, mb = tables.shape
+        assert qs.shape == (num_seqs + 1,) and qs[-1] == total
+        out = np.zeros((total, num_heads, d), dtype=np.float64)
+        rc = self._lib.pa_oracle_prefill(_ptr(q, _c_u16p), _ptr(k_cache, _c_u16p), _ptr(v_cache, _c_u16p),
+                                         _ptr(tables, _c_i32p), _ptr(lens, _c_i32p), _ptr(qs, _c_i32p), float(scale),
+                                         num_seqs, num_heads, hk, d, bs, nb, mb, dtype, _ptr(out, _c_f64p),
+                                         int(nthreads))
+        if rc != 0:
+            raise ValueError(f"oracle prefill rejected its input (code {rc})")
+        return out
 
     def decode_fp8(self, q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, block_tables: np.ndarray,
                    context_lens: np.ndarray, scale: float, k_scale: float, v_scale: float, dtype: int, pairs=None,

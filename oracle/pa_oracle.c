@@ -296,6 +296,16 @@ typedef struct {
     int tid;
 } worker_arg;
 
+/* Prefill: query rows come from a packed [T][H][d] array; query row i of sequence
+ * s sits at absolute position context_lens[s] - n_s + i and attends to tokens
+ * 0..position (causal). */
+typedef struct {
+    decode_job base;       /* caches, tables, lengths, scale, shapes (q unused) */
+    const uint16_t* q;     /* [T][H][d] */
+    const int32_t* query_start; /* [S + 1] */
+    int total_queries;
+} prefill_job;
+
 /* Value of cache element `idx`: a 16-bit element widened, or an fp8 code times its scale. */
 static double kval(const decode_job* j, int64_t idx) {
     return j->k8 ? pa_oracle_e4m3_to_double(j->k8[idx]) * j->k_scale : widen(j->k_cache[idx], j->dtype);
@@ -314,11 +324,22 @@ static int64_t cache_row(const decode_job* j, int64_t phys, int64_t off, int kv_
 #endif
 }
 
-/* Attention of query head h of sequence s over the sequence's L tokens:
- *   x_t = scale * sum_i q_i K_t,i                for t = 0..L-1 (logical order)
+static int attend(const decode_job* j, int s, int h, const uint16_t* qrow, int64_t len, double* out, double* qd,
+                  double* x);
+
+static int decode_one(const decode_job* j, int s, int h, double* out, double* qd, double* x) {
+    const int64_t len = j->context_lens[s];
+    if (len < 0 || len > (int64_t)j->max_blocks_per_seq * j->block_size) return 1;
+    return attend(j, s, h, j->q + ((int64_t)s * j->num_heads + h) * j->head_dim, len, out, qd, x);
+}
+
+/* Attention of one query row (query head h of sequence s) over the sequence's
+ * first `len` tokens:
+ *   x_t = scale * sum_i q_i K_t,i                for t = 0..len-1 (logical order)
  *   out = sum_t exp(x_t - M) V_t / sum_t exp(x_t - M),   M = max_t x_t
  * M only keeps exp() in range; any constant gives the same value in exact math. */
-static int decode_one(const decode_job* j, int s, int h, double* out, double* qd, double* x) {
+static int attend(const decode_job* j, int s, int h, const uint16_t* qrow, int64_t len, double* out, double* qd,
+                  double* x) {
     const int d = j->head_dim, bs = j->block_size;
     const int group = j->num_heads / j->num_kv_heads;
 #if PA_ORACLE_MUTANT == 4
@@ -327,12 +348,9 @@ static int decode_one(const decode_job* j, int s, int h, double* out, double* qd
 #else
     const int kv_head = h / group; /* contiguous groups of `group` query heads */
 #endif
-    const int64_t len = j->context_lens[s];
-    if (len < 0 || len > (int64_t)j->max_blocks_per_seq * bs) return 1;
     for (int i = 0; i < d; ++i) out[i] = 0.0;
     if (len == 0) return 0; /* empty context: zeros */
 
-    const uint16_t* qrow = j->q + ((int64_t)s * j->num_heads + h) * d;
     for (int i = 0; i < d; ++i) qd[i] = widen(qrow[i], j->dtype);
 
     const int32_t* table = j->tables + (int64_t)s * j->max_blocks_per_seq;
@@ -481,6 +499,85 @@ int pa_oracle_decode_fp8(const uint16_t* q, const uint8_t* k_cache, const uint8_
                       num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
                       dtype, pairs, npairs, out, nthreads < 1 ? 1 : nthreads, 0};
     return run_decode(&job);
+}
+
+static void* prefill_worker(void* p) {
+    worker_arg* a = (worker_arg*)p;
+    prefill_job* pj = (prefill_job*)a->job;
+    decode_job* j = &pj->base;
+    const int d = j->head_dim;
+    int64_t max_len = (int64_t)j->max_blocks_per_seq * j->block_size;
+    double* qd = (double*)malloc(sizeof(double) * (size_t)d);
+    double* x = (double*)malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1));
+    if (!qd || !x) {
+        j->error = 2;
+        free(qd);
+        free(x);
+        return NULL;
+    }
+    const int64_t rows = (int64_t)pj->total_queries * j->num_heads;
+    for (int64_t w = a->tid; w < rows; w += j->nthreads) {
+        const int64_t qi = w / j->num_heads;
+        const int h = (int)(w % j->num_heads);
+        int s = 0;  /* the sequence owning packed query row qi */
+        while (s < j->num_seqs && pj->query_start[s + 1] <= qi) ++s;
+        if (s >= j->num_seqs) {
+            j->error = 1;
+            continue;
+        }
+        const int64_t n = pj->query_start[s + 1] - pj->query_start[s];
+        const int64_t len = j->context_lens[s];
+        const int64_t pos = len - n + (qi - pj->query_start[s]); /* absolute position of this query */
+        if (len > max_len || pos < 0) {
+            j->error = 1;
+            continue;
+        }
+        if (attend(j, s, h, pj->q + (qi * j->num_heads + h) * d, pos + 1, j->out + w * d, qd, x) != 0)
+            j->error = 1;
+    }
+    free(qd);
+    free(x);
+    return NULL;
+}
+
+/* Prefill attention: out[i][h] for every packed query row i (of T) and head h,
+ * causal over the paged cache (which already holds the chunk's own K/V).  Query
+ * rows of sequence s are rows query_start[s] .. query_start[s+1]-1.  out is
+ * [T][H][d].  Returns 0, 1 on a bad argument, 2 on allocation failure. */
+int pa_oracle_prefill(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                      const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
+                      double scale, int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                      int num_blocks, int max_blocks_per_seq, int dtype, double* out, int nthreads) {
+    if (bad_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype))
+        return 1;
+    for (int s = 0; s < num_seqs; ++s)
+        if (query_start[s + 1] < query_start[s]) return 1;
+    prefill_job pj;
+    decode_job base = {NULL, k_cache, v_cache, NULL, NULL, 1.0, 1.0, block_tables, context_lens, scale, num_seqs,
+                       num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype,
+                       NULL, 0, out, nthreads < 1 ? 1 : nthreads, 0};
+    pj.base = base;
+    pj.q = q;
+    pj.query_start = query_start;
+    pj.total_queries = query_start[num_seqs];
+    int n = pj.base.nthreads;
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)n);
+    worker_arg* args = (worker_arg*)malloc(sizeof(worker_arg) * (size_t)n);
+    if (!th || !args) {
+        free(th);
+        free(args);
+        return 2;
+    }
+    for (int t = 0; t < n; ++t) {
+        args[t].job = (decode_job*)&pj;
+        args[t].tid = t;
+        if (t > 0) pthread_create(&th[t], NULL, prefill_worker, &args[t]);
+    }
+    prefill_worker(&args[0]);
+    for (int t = 1; t < n; ++t) pthread_join(th[t], NULL);
+    free(th);
+    free(args);
+    return pj.base.error;
 }
 
 /* Build-time identification for the tests: which mistake (0 = none) is planted. */

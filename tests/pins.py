@@ -426,4 +426,42 @@ def pin_decode_not_per_block_sum(o):
     assert np.abs(got - blocked).max() > 0.1
 
 
+# ------------------------------------------------------------------- prefill
+
+def _packed_queries(c, n_new, rng):
+    """Query rows of the last n_new[s] tokens of each sequence, packed by sequence."""
+    qs = np.concatenate([[0], np.cumsum(n_new)]).astype(np.int32)
+    q = to_bits(rng.normal(0, 1, (int(qs[-1]), c.H, c.d)), c.dtype)
+    return q, qs
+
+
+def pin_prefill_single_query_is_decode(o):
+    """A chunk of one query token per sequence is exactly a decode step."""
+    rng = np.random.default_rng(27)
+    c = PagedCase(rng, [9, 40, 130], 4, 2, 64, 16, F16, 0.125)
+    got = o.prefill(c.q.reshape(3, 4, 64).copy(), c.k_cache, c.v_cache, c.tables, c.lens,
+                    np.arange(4, dtype=np.int32), c.scale, F16)
+    assert np.array_equal(got, c.run(o))
+
+
+def pin_prefill_matches_masked_sdpa(o):
+    """Against torch's scaled_dot_product_attention on the contiguous K/V with the
+    causal mask of the chunk: query i of a chunk of n over L tokens sees t <= L-n+i
+    (a whole-prompt chunk, n = L, is the plain causal case)."""
+    rng = np.random.default_rng(28)
+    for lens, n_new, h, hk, bs in (([37, 80], [37, 80], 4, 4, 16), ([50, 129, 64], [5, 33, 64], 6, 2, 16),
+                                   ([70], [19], 2, 1, 64)):
+        c = PagedCase(rng, lens, h, hk, 64, bs, BF16, 0.13)
+        q, qs = _packed_queries(c, n_new, rng)
+        got = o.prefill(q, c.k_cache, c.v_cache, c.tables, c.lens, qs, c.scale, BF16)
+        for s, (L, n) in enumerate(zip(lens, n_new)):
+            qq = torch.from_numpy(from_bits(q[qs[s]:qs[s + 1]], BF16)).permute(1, 0, 2)[None]   # [1,H,n,d]
+            k = torch.from_numpy(from_bits(c.seq_k[s], BF16)).permute(1, 0, 2)[None]           # [1,Hk,L,d]
+            v = torch.from_numpy(from_bits(c.seq_v[s], BF16)).permute(1, 0, 2)[None]
+            mask = torch.arange(L)[None, :] <= (L - n + torch.arange(n))[:, None]
+            ref = torch.nn.functional.scaled_dot_product_attention(qq, k, v, attn_mask=mask, scale=c.scale,
+                                                                   enable_gqa=h != hk)
+            assert np.allclose(got[qs[s]:qs[s + 1]], ref[0].permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
