@@ -54,7 +54,7 @@ def parse():
                    help="fp8: the cache is stored as E4M3 codes (pa_reshape_and_cache_fp8 / pa_decode_fp8)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
-    p.add_argument("--row", default="decode", choices=["decode", "copy_blocks", "swap"],
+    p.add_argument("--row", default="decode", choices=["decode", "copy_blocks", "swap", "prefill"],
                    help="decode: the hot path (default); copy_blocks: copy-on-write block copies alone; "
                         "swap: swap-out / swap-in of blocks to pinned host memory")
     return p.parse_args()
@@ -593,8 +593,61 @@ def run_swap(args):
                       "bytes_per_call": moved, "blocks_per_call": n, **res}), flush=True)
 
 
+def run_prefill(args):
+    """Paged prefill at the 7B layer shape (32 heads, head_dim 128, block size 16,
+    fp16): (a) 8 whole 2048-token prompts, (b) 8 chunks of 512 tokens after 3584
+    cached ones.  Attention FLOPs = 4 * d * H * (attended tokens summed over rows)."""
+    import torch
+    from paged_kv_cache_374_b200 import binding as pa
+    h = hk = 32
+    d, bs = 128, 16
+    peak = 1713.1
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak = float(json.load(f)["bf16_tflops"])
+    except Exception:
+        pass
+    res = {}
+    for name, prior, chunk in (("prompt_2048", 0, 2048), ("chunk_512_after_3584", 3584, 512)):
+        s = 8
+        L = prior + chunk
+        nblk = L // bs
+        nb = s * nblk + 8
+        g = torch.Generator(device="cuda").manual_seed(7)
+        kc = torch.randn(nb, bs, hk, d, generator=g, device="cuda").to(torch.float16)
+        vc = torch.randn(nb, bs, hk, d, generator=g, device="cuda").to(torch.float16)
+        perm = torch.randperm(nb, generator=torch.Generator().manual_seed(8))[: s * nblk]
+        tables = perm.view(s, nblk).to(torch.int32).cuda()
+        lens = torch.full((s,), L, dtype=torch.int32, device="cuda")
+        qs = (torch.arange(s + 1, dtype=torch.int32) * chunk).cuda()
+        q = torch.randn(s * chunk, h, d, generator=g, device="cuda").to(torch.float16)
+        out = torch.empty_like(q)
+        call = lambda: pa.pa_prefill(q, kc, vc, tables, lens, qs, 1 / math.sqrt(d), hk, out, chunk)
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        steps = min(args.steps, 50)
+        e0.record()
+        for _ in range(steps):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        attended = s * sum(prior + i + 1 for i in range(chunk))
+        flops = 4 * d * h * attended
+        tf = flops / (ms / 1e3) / 1e12
+        res[name] = {"TFLOP/s": round(tf, 1), "ms_per_call": round(ms, 4), "tokens_per_s": round(s * chunk / ms * 1e3),
+                     "frac_of_bf16_peak": round(tf / peak, 4)}
+    print(json.dumps({"row": "prefill", "metric": "paged prefill attention TFLOP/s (7B layer shape, fp16)",
+                      "peak_tflops": peak, **res}), flush=True)
+
+
 def main():
     args = parse()
+    if args.row == "prefill":
+        run_prefill(args)
+        return
     if args.row == "copy_blocks":
         run_copy_blocks(args)
         return

@@ -217,6 +217,34 @@ int pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const
                   int dtype, int partition_tokens, void* workspace, size_t workspace_bytes, int32_t* err_word,
                   void* stream);
 
+/* ----------------------------------------------------------------- prefill */
+
+/*
+ * pa_prefill -- causal attention of a chunk of new query tokens over the paged
+ * cache: the step before decode (P2 §2.1: the prompt's K/V enter the cache and
+ * each position attends to the ones before it; with prefix reuse, P3 §三, the
+ * chunk starts after tokens already cached).
+ *
+ * Sequence s contributes n_s = query_start[s+1] - query_start[s] query rows, packed
+ * by sequence; its cache already holds all L_s = context_lens[s] tokens, the
+ * chunk's own K/V included (written by pa_reshape_and_cache with the slots of
+ * pa_prefill_slots).  Query row i of sequence s sits at position L_s - n_s + i and
+ * attends, with one softmax, to tokens 0 .. L_s - n_s + i through the block table:
+ *     out[row][h] = softmax(scale * q[row][h] K[0..pos]^T) V[0..pos]   (h_kv = h / g)
+ *
+ *   q, out        [T][num_heads][head_dim], T = query_start[num_seqs], dtype, device
+ *   query_start   int32 [num_seqs + 1], device; n_s <= context_lens[s]
+ *   max_query_len the largest n_s (sizes the grid)
+ * Caches, tables, lengths, dtype and supported sizes as pa_decode;
+ * max_blocks_per_seq at most 4096.  Tensor cores (mma.sync m16n8k16, fp32
+ * accumulation); p enters P.V as two 16-bit terms.  Bad lengths or table entries
+ * give NaN rows and PA_DEVERR_* bits.
+ */
+int pa_prefill(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+               const int32_t* context_lens, const int32_t* query_start, float scale, int num_kv_heads, void* out,
+               int num_seqs, int num_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+               int max_query_len, int dtype, int32_t* err_word, void* stream);
+
 /* ---------------------------------------------------------- host allocator */
 
 /*
@@ -273,6 +301,21 @@ double pa_usage(const pa_allocator* a);                             /* allocated
  */
 int pa_append_slots(pa_allocator* a, int32_t* block_tables, int max_blocks_per_seq, int32_t* context_lens,
                     int num_seqs, int block_size, int64_t* slot_mapping);
+
+/*
+ * pa_prefill_slots -- slot resolution for a chunk of new tokens per sequence
+ * (host; the prefill analogue of pa_append_slots).
+ *
+ * Sequence s holds n = context_lens[s] tokens and appends m = new_tokens[s]: its
+ * new tokens take positions n .. n+m-1, a block being allocated each time a
+ * position opens one (P3 §三, allocate_for_request / append_slot), and
+ *     slot_mapping[k] = block_tables[s][pos / block_size] * block_size + pos % block_size
+ * for the k-th new token overall, sequences in order.  context_lens[s] becomes
+ * n + m.  All or nothing (PA_ERR_OUT_OF_BLOCKS, PA_ERR_INVALID_ARG).
+ *   slot_mapping  host int64 [sum of new_tokens], out
+ */
+int pa_prefill_slots(pa_allocator* a, int32_t* block_tables, int max_blocks_per_seq, int32_t* context_lens,
+                     const int32_t* new_tokens, int num_seqs, int block_size, int64_t* slot_mapping);
 
 /* ------------------------------------------------------------ copy-on-write */
 

@@ -50,6 +50,8 @@ _sig("pa_reshape_and_cache_fp8", _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32
      ctypes.c_float, _vp, _vp)
 _sig("pa_decode_fp8", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float, ctypes.c_float, _i32, _vp, _i32,
      _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
+_sig("pa_prefill", _i32, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+     _i32, _i32, _vp, _vp)
 _sig("pa_allocator_create", _vp, _i32, _i32p)
 _sig("pa_allocator_destroy", None, _vp)
 _sig("pa_num_required_blocks", _i32, _i32, _i32)
@@ -64,6 +66,7 @@ _sig("pa_num_free", _i32, _vp)
 _sig("pa_num_blocks", _i32, _vp)
 _sig("pa_usage", ctypes.c_double, _vp)
 _sig("pa_append_slots", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32, _i64p)
+_sig("pa_prefill_slots", _i32, _vp, _i32p, _i32, _i32p, _i32p, _i32, _i32, _i64p)
 _sig("pa_cow_prepare", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32, _i32p, ctypes.POINTER(ctypes.c_int))
 _sig("pa_copy_blocks", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp)
 _sig("pa_swap_plan", _i32, _vp, _vp, _i32p, _i32, _i32p)
@@ -246,6 +249,31 @@ def pa_decode_fp8(q, k_cache, v_cache, block_tables, context_lens, scale, k_scal
     return out
 
 
+def pa_prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, scale, num_kv_heads, out,
+               max_query_len, err_word=None, stream=None):
+    """Causal chunk attention.  q / out [T, H, d] packed by sequence; query_start int32 [S+1] (CUDA)."""
+    import torch
+    total, h, d = q.shape
+    nb, bs, hk, d2 = k_cache.shape
+    s = context_lens.shape[0]
+    if hk != num_kv_heads or d2 != d or v_cache.shape != k_cache.shape or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if query_start.shape != (s + 1,) or block_tables.shape[0] != s:
+        raise ValueError("query_start must be [S+1] and block_tables [S, MB]")
+    dt = _dtype_code(q)
+    for t in (k_cache, v_cache, out):
+        if t.dtype != q.dtype:
+            raise TypeError("q, the caches and out must share one dtype")
+    st = _lib.pa_prefill(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                         _dev(block_tables, "block_tables", torch.int32),
+                         _dev(context_lens, "context_lens", torch.int32),
+                         _dev(query_start, "query_start", torch.int32), float(scale), hk, _dev(out, "out"), s, h, d,
+                         bs, nb, block_tables.shape[1], int(max_query_len), dt, _dev(err_word, "err_word", torch.int32),
+                         _stream(stream, q))
+    _check(st, "pa_prefill")
+    return out
+
+
 # --------------------------------------------------------------- allocator
 
 def _np_i32(a, name):
@@ -332,6 +360,20 @@ def pa_append_slots(handle, block_tables: np.ndarray, context_lens: np.ndarray, 
     _check(_lib.pa_append_slots(handle, tables.ctypes.data_as(_i32p), mb, lens.ctypes.data_as(_i32p), s,
                                 block_size, slots.ctypes.data_as(_i64p)), "pa_append_slots")
     return slots
+
+
+def pa_prefill_slots(handle, block_tables: np.ndarray, context_lens: np.ndarray, new_tokens,
+                     block_size: int) -> np.ndarray:
+    """In place on block_tables and context_lens (int32); returns the new tokens' slots, int64 [sum(new)]."""
+    tables = _np_i32(block_tables, "block_tables")
+    lens = _np_i32(context_lens, "context_lens")
+    new = np.ascontiguousarray(new_tokens, dtype=np.int32)
+    s, mb = tables.shape
+    slots = np.empty(max(int(new.sum()), 1), dtype=np.int64)
+    _check(_lib.pa_prefill_slots(handle, tables.ctypes.data_as(_i32p), mb, lens.ctypes.data_as(_i32p),
+                                 new.ctypes.data_as(_i32p), s, block_size, slots.ctypes.data_as(_i64p)),
+           "pa_prefill_slots")
+    return slots[:int(new.sum())]
 
 
 def pa_cow_prepare(handle, block_tables: np.ndarray, context_lens: np.ndarray, block_size: int) -> np.ndarray:
@@ -438,6 +480,9 @@ class BlockAllocator:
 
     def append_slots(self, block_tables: np.ndarray, context_lens: np.ndarray, block_size: int) -> np.ndarray:
         return pa_append_slots(self.handle, block_tables, context_lens, block_size)
+
+    def prefill_slots(self, block_tables: np.ndarray, context_lens: np.ndarray, new_tokens, block_size: int):
+        return pa_prefill_slots(self.handle, block_tables, context_lens, new_tokens, block_size)
 
     def cow_prepare(self, block_tables: np.ndarray, context_lens: np.ndarray, block_size: int) -> np.ndarray:
         return pa_cow_prepare(self.handle, block_tables, context_lens, block_size)

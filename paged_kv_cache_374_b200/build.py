@@ -13,7 +13,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIBRARY = os.path.join(PKG, "libpa.so")
-SOURCES = ["allocator.cpp", "reshape_and_cache.cu", "paged_decode.cu", "paged_decode_noalloc.cu", "copy_blocks.cu"]
+SOURCES = ["allocator.cpp", "reshape_and_cache.cu", "paged_decode.cu", "paged_decode_noalloc.cu", "copy_blocks.cu",
+           "paged_prefill.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-Xcompiler", "-fPIC,-O2,-Wall", "-shared", "-cudart", "static"]
 

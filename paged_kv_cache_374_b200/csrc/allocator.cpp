@@ -190,6 +190,43 @@ int pa_append_slots(pa_allocator* a, int32_t* block_tables, int max_blocks_per_s
     return PA_OK;
 }
 
+int pa_prefill_slots(pa_allocator* a, int32_t* block_tables, int max_blocks_per_seq, int32_t* context_lens,
+                     const int32_t* new_tokens, int num_seqs, int block_size, int64_t* slot_mapping) {
+    if (!a || num_seqs < 0 || max_blocks_per_seq < 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
+    if (num_seqs > 0 && (!block_tables || !context_lens || !new_tokens || !slot_mapping)) return PA_ERR_INVALID_ARG;
+    // Pass 1: validate and count the blocks the chunks open.
+    int64_t need = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        const int64_t n = context_lens[s], m = new_tokens[s];
+        if (n < 0 || m < 0 || n + m > INT32_MAX) return PA_ERR_INVALID_ARG;
+        const int64_t have = (n + block_size - 1) / block_size;
+        const int64_t want = (n + m + block_size - 1) / block_size;
+        if (want > max_blocks_per_seq) return PA_ERR_INVALID_ARG;  // the table row is too short
+        if (n % block_size != 0 && m > 0) {  // the chunk starts inside the last held block
+            const int32_t id = block_tables[(int64_t)s * max_blocks_per_seq + n / block_size];
+            if (!a->valid(id) || a->ref[id] == 0) return PA_ERR_INVALID_ARG;
+        }
+        need += want - have;
+    }
+    if (a->count < need) return PA_ERR_OUT_OF_BLOCKS;
+    // Pass 2: open the blocks in sequence order and resolve every new token's slot.
+    int64_t k = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        const int64_t n = context_lens[s], m = new_tokens[s];
+        int32_t* row = block_tables + (int64_t)s * max_blocks_per_seq;
+        for (int64_t pos = n; pos < n + m; ++pos) {
+            if (pos % block_size == 0) {
+                const int32_t id = a->pop_front();
+                a->ref[id] = 1;
+                row[pos / block_size] = id;
+            }
+            slot_mapping[k++] = (int64_t)row[pos / block_size] * block_size + pos % block_size;
+        }
+        context_lens[s] = (int32_t)(n + m);
+    }
+    return PA_OK;
+}
+
 int pa_cow_prepare(pa_allocator* a, int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
                    int num_seqs, int block_size, int32_t* copy_pairs, int* num_copies) {
     if (!a || num_seqs < 0 || max_blocks_per_seq < 0 || block_size <= 0 || !num_copies) return PA_ERR_INVALID_ARG;

@@ -249,3 +249,33 @@ def test_swap_plan_matches_model(pa):
         got = pa.pa_swap_plan(host.handle, dev.handle, row, k)
         assert [tuple(x) for x in got.tolist()] == back and list(row) == mrow
         assert host.num_free() == mhost.num_free()
+
+
+def test_prefill_slots_match_model_and_oracle(pa, oracle):
+    """A chunk of new tokens per sequence: blocks open exactly as repeated appends
+    would open them (the model), and every new token's slot is the oracle's
+    physical location of its position."""
+    rng = np.random.default_rng(13)
+    for bs in (16, 64):
+        nb, s, mb = 300, 6, 40
+        order = rng.permutation(nb).astype(np.int32)
+        a = pa.BlockAllocator(nb, order)
+        mgr = ManagerModel(nb, bs, order)
+        lens = rng.integers(0, 3 * bs, size=s).astype(np.int32)
+        tables = np.full((s, mb), -1, dtype=np.int32)
+        for i in range(s):
+            n = pa.pa_num_required_blocks(int(lens[i]), bs)
+            tables[i, :n] = a.alloc_n(n)
+            mgr.allocate_for_request(i, int(lens[i]))
+        new = rng.integers(0, 5 * bs, size=s).astype(np.int32)
+        before = lens.copy()
+        slots = a.prefill_slots(tables, lens, new, bs)
+        k = 0
+        for i in range(s):
+            for pos in range(int(before[i]), int(before[i] + new[i])):
+                mgr.append_slot(i, pos)
+                phys, off = oracle.physical_location(tables[i], pos, bs)
+                assert slots[k] == phys * bs + off
+                k += 1
+            assert list(tables[i, :len(mgr.tables[i])]) == mgr.tables[i]
+        assert np.array_equal(lens, before + new) and a.num_free() == mgr.pool.num_free()
