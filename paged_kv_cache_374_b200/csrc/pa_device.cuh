@@ -17,6 +17,7 @@ namespace pa {
 struct F16Tag {
     using T = __half;
     static constexpr int kBytes = 2;
+    static constexpr bool kIsBF16 = false;
     // widen two packed 16-bit values (low half first) to fp32
     static __device__ __forceinline__ float2 widen2(uint32_t w) {
         return __half22float2(*reinterpret_cast<const __half2*>(&w));
@@ -30,6 +31,7 @@ struct F16Tag {
 struct BF16Tag {
     using T = __nv_bfloat16;
     static constexpr int kBytes = 2;
+    static constexpr bool kIsBF16 = true;
     static __device__ __forceinline__ float2 widen2(uint32_t w) {
         // a bfloat16 is the top half of a binary32: widening is a shift
         return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));

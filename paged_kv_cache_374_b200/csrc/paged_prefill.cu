@@ -5,26 +5,40 @@
 // cached tokens).  Query row i of sequence s (chunk of n rows over L tokens) sits
 // at position L - n + i and attends to tokens 0 .. L - n + i through the table.
 //
-// A real dense contraction, run on tensor cores (mma.sync m16n8k16, 16-bit inputs,
-// fp32 accumulation): one CTA = 64 query rows of one head (4 warps x 16 rows),
-// streaming 64-token K/V tiles of its kv head through a two-stage TMA ring (the
-// 128-byte-swizzled tensor maps of the decode path, one mbarrier per stage).  Per
-// tile: S = Q K^T (K via ldmatrix), causal mask, online softmax per row in base 2,
-// O += P V (V via ldmatrix.trans; P taken straight from the S accumulators and
-// fed as two 16-bit terms, hi + lo, so p keeps about 16 significant bits).
-// Tokens past the sequence end are zeroed in the V fragments (0 * NaN is NaN in an
-// MMA); table entries are checked once, up front.
+// A real dense contraction, run on the 5th-generation tensor cores (tcgen05, fp32
+// accumulators in tensor memory).  One CTA = 128 query rows of one head (the MMA's
+// M), two CTAs per SM:
+//   - warp 4 streams the kv head's K and V in 64-token tiles through two-stage
+//     TMA rings (the 128-byte-swizzled tensor maps of the decode path; a tile's
+//     table entries are read as it is issued, after one up-front range check);
+//   - warp 5 owns the tensor memory and issues every MMA from one thread:
+//       S_j = Q K_j^T   (A = Q, B = K, both K-major in shared memory; M 128 x N 64)
+//       O  += P_j V_j   (A = P_j in tensor memory, B = V_j MN-major; M 128 x N d)
+//     in the order S_0, S_1, PV_0, S_2, PV_1, ... with S double-buffered, so the
+//     softmax of tile j+1 overlaps the tensor core's work on tile j;
+//   - warps 0-3 own one query row per thread (tensor-memory lane = row): read
+//     S_j, apply the causal mask and the online softmax in base 2, write P_j over
+//     S_j as two 16-bit terms (hi + lo, about 16 significant bits, so the result
+//     keeps the decode path's accuracy), and at the end normalise O and store it.
+// The running max used for the exponentials only moves when a row's max grows
+// by more than 2^8 (then O and the row sum are rescaled in tensor memory); the
+// result is the same softmax, p stays <= 256.  V rows past the sequence end are
+// zeroed in shared memory before PV (0 * NaN is NaN in an MMA).  Every wait is
+// bounded; a timeout reports PA_DEVERR_TIMEOUT and the CTA drains its copies and
+// MMAs before freeing tensor memory.
 #include <cmath>
 
-#include "decode_gqa.cuh"
+#include "decode_engine.cuh"
 #include "pa_host.h"
+#include "tcgen05.cuh"
 
 namespace pa {
 
-constexpr int kPfRows = 64;          // query rows per CTA
+constexpr int kPfRows = 128;         // query rows per CTA
 constexpr int kPfTok = 64;           // tokens per K/V tile
-constexpr int kPfThreads = 128;
-constexpr int kPfMaxEntries = 4096;  // table entries a CTA can hold
+constexpr int kPfThreads = 192;      // softmax warps 0-3, load warp 4, MMA warp 5
+constexpr uint32_t kPfTmemCols = 256;  // O at column 0, S/P buffers at 128 and 192
+constexpr float kPfRescaleLog2 = 8.f;
 
 struct PrefillArgs {
     const uint16_t* q;    // [T][H][D]
@@ -39,30 +53,45 @@ struct PrefillArgs {
 
 template <int D>
 struct PfLayout {
-    static constexpr int kTile = kPfTok * D * 2;       // one K or V tile
-    static constexpr int kHalf = kPfTok * 128;         // one 64-dim half of a tile
-    static constexpr int kStage = 2 * kTile;           // K then V
-    static constexpr int kOffBars = 2 * kStage;
-    static constexpr int kOffTab = kOffBars + 16;
-    static constexpr int kBytes = kOffTab + kPfMaxEntries * 4;
+    static constexpr int kQHalf = kPfRows * 128;  // 64 dims of every query row
+    static constexpr int kTHalf = kPfTok * 128;   // 64 dims of every token of a tile
+    static constexpr int kTile = (D / 64) * kTHalf;
+    static constexpr int kOffK = (D / 64) * kQHalf;
+    static constexpr int kOffV = kOffK + 2 * kTile;
+    static constexpr int kOffBars = kOffV + 2 * kTile;
+    static constexpr int kNumBars = 16;
+    static constexpr int kBytes = kOffBars + kNumBars * 8 + 16;
     static constexpr int kAlloc = kBytes + 1024;
 };
 
+// mbarrier slots
+enum : int {
+    kBarKFull = 0,    // [2] TMA landed a K tile
+    kBarKEmpty = 2,   // [2] the S MMAs reading a K stage are done
+    kBarVFull = 4,    // [2]
+    kBarVEmpty = 6,   // [2] the PV MMAs reading a V stage are done
+    kBarSFull = 8,    // [2] S_j is in its buffer
+    kBarPFull = 10,   // [2] the 128 row threads wrote P_j
+    kBarOFull = 12,   // [2] PV_j has landed in O (alternating by tile parity)
+    kBarOLast = 14,   // the last PV has landed
+    kBarDrain = 15,   // every MMA issued has completed
+};
+
 template <class Tag, int D>
-__global__ void __launch_bounds__(kPfThreads) paged_prefill_kernel(const PrefillArgs a,
-                                                                   const __grid_constant__ CUtensorMap kmap,
-                                                                   const __grid_constant__ CUtensorMap vmap) {
+__global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const PrefillArgs a,
+                                                                      const __grid_constant__ CUtensorMap kmap,
+                                                                      const __grid_constant__ CUtensorMap vmap) {
     using Lay = PfLayout<D>;
-    using Ops = MmaOps<Tag>;
-    constexpr int KS = D / 16;  // k-steps of q K^T
-    constexpr int DN = D / 8;   // 8-dim output tiles
-    constexpr int NT = kPfTok / 8;  // 8-token score tiles per K tile
+    constexpr bool kBF16 = Tag::kIsBF16;
+    constexpr uint32_t kIdS = umma::idesc_f16(kBF16, false, kPfRows, kPfTok);
+    constexpr uint32_t kIdO = umma::idesc_f16(kBF16, true, kPfRows, D);
     constexpr unsigned FULL = 0xffffffffu;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBars);
-    int32_t* s_tab = reinterpret_cast<int32_t*>(smem + Lay::kOffTab);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + Lay::kNumBars);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
     const int s = blockIdx.z, h = blockIdx.y;
     const int qt = gridDim.x - 1 - blockIdx.x;  // tiles with the most context first
@@ -70,39 +99,28 @@ __global__ void __launch_bounds__(kPfThreads) paged_prefill_kernel(const Prefill
     const int n = a.query_start[s + 1] - q0;
     if (qt * kPfRows >= n) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t = lane & 3;
     const int L = a.context_lens[s];
     const int bs = a.block_size;
     const int q_first = qt * kPfRows;
-    const int q_last = min(n, q_first + kPfRows) - 1;
+    const int nrows = min(n - q_first, kPfRows);
     auto write_rows = [&](float value) {
-        for (int i = tid; i < (q_last - q_first + 1) * D; i += kPfThreads) {
-            const int r = q_first + i / D;
-            a.out[((int64_t)(q0 + r) * a.num_heads + h) * D + i % D] = Tag::round1(value);
-        }
+        for (int i = tid; i < nrows * D; i += kPfThreads)
+            a.out[((int64_t)(q0 + q_first + i / D) * a.num_heads + h) * D + i % D] = Tag::round1(value);
     };
     if (L < 0 || L > a.max_blocks_per_seq * bs || n > L) {
         write_rows(__int_as_float(0x7fc00000));
         if (tid == 0) report(a.err_word, PA_DEVERR_LEN_RANGE);
         return;
     }
-    const int base_pos = L - n;
-    const int pos_last = base_pos + q_last;
-    const int ntiles = pos_last / kPfTok + 1;
+    const int base_pos = L - n + q_first;  // position of this CTA's first row
+    const int ntiles = (base_pos + nrows - 1) / kPfTok + 1;
     const int kv_head = h / a.group;
+    const int32_t* tab = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
     const int nent = (min(ntiles * kPfTok, L) + bs - 1) / bs;  // table entries the tiles read
-
-    // table entries, checked once
     bool bad = false;
     for (int i = tid; i < nent; i += kPfThreads) {
-        const int id = a.block_tables[(int64_t)s * a.max_blocks_per_seq + i];
-        s_tab[i] = id;
+        const int id = __ldg(tab + i);
         bad |= id < 0 || id >= a.num_blocks;
-    }
-    if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        fence_mbar_init();
     }
     if (__syncthreads_or(bad)) {
         write_rows(__int_as_float(0x7fc00000));
@@ -110,174 +128,242 @@ __global__ void __launch_bounds__(kPfThreads) paged_prefill_kernel(const Prefill
         return;
     }
 
-    const int br = a.box_rows;
-    auto issue = [&](int tile, int st) {  // thread 0 only
-        uint8_t* kd = smem + st * Lay::kStage;
-        uint32_t tx = 0;
-        for (int j = 0; j * br < kPfTok; ++j)
-            if (tile * kPfTok + j * br < L) tx += 2u * (D / 64) * br * 128;
-        mbar_arrive_expect_tx(&bars[st], tx);
-        for (int j = 0; j * br < kPfTok; ++j) {
-            const int tj = tile * kPfTok + j * br;
-            if (tj >= L) break;
-            const int row = s_tab[tj / bs] * bs + tj % bs;
+    // Q rows -> K-major swizzled tile; rows past the chunk are zero
+    if (tid < kPfRows) {
+        const bool live = tid < nrows;
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)(q0 + q_first + (live ? tid : 0)) * a.num_heads + h) * D);
 #pragma unroll
-            for (int hh = 0; hh < D / 64; ++hh) {
-                uint8_t* dst = kd + hh * Lay::kHalf + j * br * 128;
-                tma_load_3d(dst, &kmap, hh * 64, kv_head, row, &bars[st]);
-                tma_load_3d(dst + Lay::kTile, &vmap, hh * 64, kv_head, row, &bars[st]);
-            }
+        for (int c = 0; c < D / 8; ++c) {
+            const uint4 v = live ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(smem + (c >> 3) * Lay::kQHalf + tid * 128 + (((c & 7) ^ (tid & 7)) << 4)) = v;
         }
-    };
+        fence_proxy_async_shared();
+    }
     if (tid == 0) {
-        issue(0, 0);
-        if (ntiles > 1) issue(1, 1);
+        for (int i = 0; i < Lay::kNumBars; ++i) mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? kPfRows : 1);
+        *abort_flag = 0;
+        fence_mbar_init();
     }
+    if (warp == 5) umma::alloc(tslot, kPfTmemCols);
+    umma::fence_before_sync();
+    __syncthreads();
+    umma::fence_after_sync();
+    const uint32_t tmem = *tslot;
+    const uint32_t tO = tmem, tS = tmem + 128;  // S/P buffer b at tS + 64 b
 
-    // this warp's 16 query rows: g and g + 8; rows past the chunk act as its last row
-    const int row0 = q_first + warp * 16 + g, row1 = row0 + 8;
-    const int pos0 = base_pos + min(row0, n - 1), pos1 = base_pos + min(row1, n - 1);
-    uint32_t qa[KS][4];
-    {
-        const uint32_t* p0 = reinterpret_cast<const uint32_t*>(a.q + ((int64_t)(q0 + min(row0, n - 1)) * a.num_heads + h) * D);
-        const uint32_t* p1 = reinterpret_cast<const uint32_t*>(a.q + ((int64_t)(q0 + min(row1, n - 1)) * a.num_heads + h) * D);
+    if (warp == 4) {
+        // ---------------------------------------------------------------- loads
+        if (lane == 0) {
+            const int br = a.box_rows;
+            auto load = [&](const CUtensorMap* map, uint8_t* dst0, uint64_t* bar, int tile) {
+                const int t0 = tile * kPfTok;
+                uint32_t tx = 0;
+                for (int j = 0; j * br < kPfTok; ++j)
+                    if (t0 + j * br < L) tx += (uint32_t)(D / 64) * br * 128;
+                mbar_arrive_expect_tx(bar, tx);
+                for (int j = 0; j * br < kPfTok; ++j) {
+                    const int tj = t0 + j * br;
+                    if (tj >= L) break;
+                    const int row = __ldg(tab + tj / bs) * bs + tj % bs;
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            qa[ks][0] = __ldg(p0 + ks * 8 + t);
-            qa[ks][1] = __ldg(p1 + ks * 8 + t);
-            qa[ks][2] = __ldg(p0 + ks * 8 + 4 + t);
-            qa[ks][3] = __ldg(p1 + ks * 8 + 4 + t);
+                    for (int hh = 0; hh < D / 64; ++hh)
+                        tma_load_3d(dst0 + hh * Lay::kTHalf + j * br * 128, map, hh * 64, kv_head, row, bar);
+                }
+            };
+            bool ok = true;
+            int issued_k = 0, issued_v = 0;
+            for (int j = 0; j < ntiles; ++j) {
+                const int st = j & 1;
+                if (j >= 2) ok = mbar_wait(&bars[kBarKEmpty + st], ((j >> 1) + 1) & 1) && !*abort_flag;
+                if (!ok) break;
+                load(&kmap, smem + Lay::kOffK + st * Lay::kTile, &bars[kBarKFull + st], j);
+                issued_k = j + 1;
+                if (j >= 2) ok = mbar_wait(&bars[kBarVEmpty + st], ((j >> 1) + 1) & 1) && !*abort_flag;
+                if (!ok) break;
+                load(&vmap, smem + Lay::kOffV + st * Lay::kTile, &bars[kBarVFull + st], j);
+                issued_v = j + 1;
+            }
+            if (!ok) {
+                report(a.err_word, PA_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+            // every copy still in flight lands before the CTA may exit
+            for (int j = max(0, issued_k - 2); j < issued_k; ++j) mbar_wait(&bars[kBarKFull + (j & 1)], (j >> 1) & 1);
+            for (int j = max(0, issued_v - 2); j < issued_v; ++j) mbar_wait(&bars[kBarVFull + (j & 1)], (j >> 1) & 1);
         }
-    }
-    float o[DN][4];
+    } else if (warp == 5) {
+        // ----------------------------------------------------------------- MMAs
+        const uint32_t qa = smem_u32(smem);
+        auto issue_s = [&](int j) {  // lane 0: S_j = Q K_j^T into buffer j & 1
+            const uint32_t ka = smem_u32(smem + Lay::kOffK + (j & 1) * Lay::kTile);
 #pragma unroll
-    for (int dn = 0; dn < DN; ++dn) o[dn][0] = o[dn][1] = o[dn][2] = o[dn][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    int stopped_at = -1;  // tile whose wait gave up (the decision is CTA-uniform)
-
-    for (int it = 0; it < ntiles; ++it) {
-        const int st = it & 1;
-        const bool ok = __all_sync(FULL, mbar_wait(&bars[st], (it >> 1) & 1));
-        if (__syncthreads_or(!ok)) {
-            stopped_at = it;
-            break;
-        }
-        const uint8_t* kt = smem + st * Lay::kStage;
-        const uint8_t* vt = kt + Lay::kTile;
-        const int tile_base = it * kPfTok;
-        // ---- S = Q K^T
-        float sc[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-#pragma unroll
-            for (int np = 0; np < NT / 2; ++np) {
-                const int tok = np * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-                const int ch = ks * 2 + ((lane >> 3) & 1);
-                uint32_t b[4];
-                ldsm_x4(b, kt + (ch >> 3) * Lay::kHalf + tok * 128 + (((ch & 7) ^ (lane & 7)) << 4));
-                Ops::mma(sc[2 * np], qa[ks], b[0], b[1]);
-                Ops::mma(sc[2 * np + 1], qa[ks], b[2], b[3]);
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t da = umma::desc_sw128(qa + (kk >> 2) * Lay::kQHalf + (kk & 3) * 32, 16, 1024);
+                const uint64_t db = umma::desc_sw128(ka + (kk >> 2) * Lay::kTHalf + (kk & 3) * 32, 16, 1024);
+                umma::mma_ss(tS + (j & 1) * 64, da, db, kIdS, kk > 0 ? 1u : 0u);
+            }
+            umma::commit(&bars[kBarSFull + (j & 1)]);
+            umma::commit(&bars[kBarKEmpty + (j & 1)]);
+        };
+        auto wait = [&](int bar, uint32_t parity) {  // whole warp
+            const bool ok = mbar_wait(&bars[bar], parity) && !*abort_flag;
+            return __all_sync(FULL, ok);
+        };
+        bool ok = true;
+        for (int j = 0; j < 2 && j < ntiles && ok; ++j) {
+            ok = wait(kBarKFull + j, 0);
+            if (ok) {
+                umma::fence_after_sync();
+                if (lane == 0) issue_s(j);
+                __syncwarp();
             }
         }
-        // ---- causal mask, online softmax (rows g and g+8)
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int st = j & 1;
+            ok = wait(kBarVFull + st, (j >> 1) & 1);
+            if (!ok) break;
+            const int t0 = j * kPfTok;
+            if (t0 + kPfTok > L) {  // zero the V rows past the sequence end
+                uint8_t* vt = smem + Lay::kOffV + st * Lay::kTile;
+                const int r0 = L - t0;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int tk = tile_base + nt * 8 + 2 * t;
-            sc[nt][0] = tk <= pos0 ? sc[nt][0] * a.scale_log2 : -INFINITY;
-            sc[nt][1] = tk + 1 <= pos0 ? sc[nt][1] * a.scale_log2 : -INFINITY;
-            sc[nt][2] = tk <= pos1 ? sc[nt][2] * a.scale_log2 : -INFINITY;
-            sc[nt][3] = tk + 1 <= pos1 ? sc[nt][3] * a.scale_log2 : -INFINITY;
-            mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
-            mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
-        }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: token 0 is always visible
-        const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
-        m0 = mn0;
-        m1 = mn1;
-        l0 *= al0;
-        l1 *= al1;
-#pragma unroll
-        for (int dn = 0; dn < DN; ++dn) {
-            o[dn][0] *= al0;
-            o[dn][1] *= al0;
-            o[dn][2] *= al1;
-            o[dn][3] *= al1;
-        }
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            sc[nt][0] = fast_exp2(sc[nt][0] - m0);
-            sc[nt][1] = fast_exp2(sc[nt][1] - m0);
-            sc[nt][2] = fast_exp2(sc[nt][2] - m1);
-            sc[nt][3] = fast_exp2(sc[nt][3] - m1);
-            l0 += sc[nt][0] + sc[nt][1];
-            l1 += sc[nt][2] + sc[nt][3];
-        }
-        // ---- O += P V, 16 tokens at a time
-        const bool tail = tile_base + kPfTok > L;  // some tokens of this tile are past the sequence end
-#pragma unroll
-        for (int kk = 0; kk < kPfTok / 16; ++kk) {
-            uint32_t ph[4], pl[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float* src = &sc[2 * kk + (j >> 1)][(j & 1) * 2];
-                ph[j] = Ops::pack(src[0], src[1]);
-                const float2 hv = Tag::widen2(ph[j]);
-                pl[j] = Ops::pack(src[0] - hv.x, src[1] - hv.y);
+                for (int hh = 0; hh < D / 64; ++hh)
+                    for (int i = r0 * 8 + lane; i < kPfTok * 8; i += 32)
+                        *reinterpret_cast<uint4*>(vt + hh * Lay::kTHalf + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+                fence_proxy_async_shared();
+                __syncwarp();
             }
-            const int tk = tile_base + kk * 16 + 2 * t;
-            const uint32_t mlo = tail ? ((tk < L ? 0x0000ffffu : 0u) | (tk + 1 < L ? 0xffff0000u : 0u)) : FULL;
-            const uint32_t mhi = tail ? ((tk + 8 < L ? 0x0000ffffu : 0u) | (tk + 9 < L ? 0xffff0000u : 0u)) : FULL;
+            ok = wait(kBarPFull + st, (j >> 1) & 1);
+            if (!ok) break;
+            umma::fence_after_sync();
+            if (lane == 0) {
+                const uint32_t va = smem_u32(smem + Lay::kOffV + st * Lay::kTile);
+                const uint32_t tp = tS + st * 64;
 #pragma unroll
-            for (int dp = 0; dp < DN / 2; ++dp) {
-                const int tok = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int ch = dp * 2 + ((lane >> 4) & 1);
-                uint32_t b[4];
-                ldsm_x4_trans(b, vt + (ch >> 3) * Lay::kHalf + tok * 128 + (((ch & 7) ^ (lane & 7)) << 4));
-                b[0] &= mlo;
-                b[1] &= mhi;
-                b[2] &= mlo;
-                b[3] &= mhi;
-                Ops::mma(o[2 * dp], ph, b[0], b[1]);
-                Ops::mma(o[2 * dp], pl, b[0], b[1]);
-                Ops::mma(o[2 * dp + 1], ph, b[2], b[3]);
-                Ops::mma(o[2 * dp + 1], pl, b[2], b[3]);
+                for (int kk = 0; kk < kPfTok / 16; ++kk) {
+                    const uint64_t db = umma::desc_sw128(va + kk * 2048, Lay::kTHalf, 1024);
+                    umma::mma_ts(tO, tp + kk * 8, db, kIdO, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma::mma_ts(tO, tp + 32 + kk * 8, db, kIdO, 1u);
+                }
+                umma::commit(&bars[kBarVEmpty + st]);
+                umma::commit(&bars[kBarOFull + st]);
+                if (j == ntiles - 1) umma::commit(&bars[kBarOLast]);
+            }
+            __syncwarp();
+            if (j + 2 < ntiles) {
+                ok = wait(kBarKFull + st, ((j + 2) >> 1) & 1);
+                if (!ok) break;
+                umma::fence_after_sync();
+                if (lane == 0) issue_s(j + 2);
+                __syncwarp();
             }
         }
-        __syncthreads();  // every warp is done with this stage
-        if (tid == 0 && it + 2 < ntiles) {
-            fence_proxy_async_shared();
-            issue(it + 2, st);
+        if (lane == 0) {
+            if (!ok) {
+                report(a.err_word, PA_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+            umma::commit(&bars[kBarDrain]);  // every MMA issued completes before TMEM is freed
+            mbar_wait(&bars[kBarDrain], 0);
         }
-    }
-    if (stopped_at >= 0) {
-        if (tid == 0) {
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ softmax, one row per thread
+        const int r = tid;
+        const int pos = base_pos + min(r, nrows - 1);
+        const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+        const float c = a.scale_log2;
+        float m_used = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < ntiles; ++j) {
+            const int b = j & 1;
+            ok = __all_sync(FULL, mbar_wait(&bars[kBarSFull + b], (j >> 1) & 1) && !*abort_flag);
+            if (!ok) break;
+            umma::fence_after_sync();
+            uint32_t sv[2][32];
+            umma::ld32(tS + b * 64 + lrow, sv[0]);
+            umma::ld32(tS + b * 64 + 32 + lrow, sv[1]);
+            umma::wait_ld();
+            const int t0 = j * kPfTok;
+            float x[kPfTok];
+            float mt = -INFINITY;
+#pragma unroll
+            for (int t = 0; t < kPfTok; ++t) {
+                x[t] = t0 + t <= pos ? __uint_as_float(sv[t >> 5][t & 31]) * c : -INFINITY;
+                mt = fmaxf(mt, x[t]);
+            }
+            const bool need = mt > m_used + kPfRescaleLog2;  // always on the first tile
+            if (__any_sync(FULL, need)) {
+                const float m_new = need ? mt : m_used;
+                if (j > 0) {
+                    const float alpha = fast_exp2(m_used - m_new);
+                    // PV_{j-1} must have landed in O before it is rescaled
+                    ok = __all_sync(FULL, mbar_wait(&bars[kBarOFull + ((j - 1) & 1)], ((j - 1) >> 1) & 1) &&
+                                              !*abort_flag);
+                    if (!ok) break;
+                    umma::fence_after_sync();
+#pragma unroll 1
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t o[32];
+                        umma::ld32(tO + lrow + cc * 32, o);
+                        umma::wait_ld();
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                        umma::st32(tO + lrow + cc * 32, o);
+                    }
+                    umma::wait_st();
+                    l *= alpha;
+                }
+                m_used = m_new;
+            }
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {  // 32 tokens -> 16 hi and 16 lo columns
+                uint32_t ph[16], pl[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const float p0 = fast_exp2(x[32 * half + 2 * k] - m_used);
+                    const float p1 = fast_exp2(x[32 * half + 2 * k + 1] - m_used);
+                    l += p0 + p1;
+                    ph[k] = pack2<Tag>(p0, p1);
+                    const float2 hv = Tag::widen2(ph[k]);
+                    pl[k] = pack2<Tag>(p0 - hv.x, p1 - hv.y);
+                }
+                umma::st16(tS + b * 64 + 16 * half + lrow, ph);
+                umma::st16(tS + b * 64 + 32 + 16 * half + lrow, pl);
+            }
+            umma::wait_st();
+            umma::fence_before_sync();
+            mbar_arrive(&bars[kBarPFull + b]);
+        }
+        if (ok) ok = __all_sync(FULL, mbar_wait(&bars[kBarOLast], 0) && !*abort_flag);
+        if (ok) {
+            umma::fence_after_sync();
+            const float inv = 1.f / l;
+            uint4* dst = reinterpret_cast<uint4*>(a.out + ((int64_t)(q0 + q_first + min(r, nrows - 1)) * a.num_heads + h) * D);
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                umma::ld32(tO + lrow + cc * 32, o);
+                umma::wait_ld();
+                if (r < nrows) {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const float* f = reinterpret_cast<const float*>(o + 8 * v);
+                        dst[cc * 4 + v] = make_uint4(pack2<Tag>(f[0] * inv, f[1] * inv), pack2<Tag>(f[2] * inv, f[3] * inv),
+                                                     pack2<Tag>(f[4] * inv, f[5] * inv), pack2<Tag>(f[6] * inv, f[7] * inv));
+                    }
+                }
+            }
+        } else if (lane == 0) {
             report(a.err_word, PA_DEVERR_TIMEOUT);
-            // tiles stopped_at and stopped_at + 1 may still be in flight: let them land
-            for (int k = stopped_at; k < ntiles && k < stopped_at + 2; ++k) mbar_wait(&bars[k & 1], (k >> 1) & 1);
+            *abort_flag = 1;
         }
-        return;
     }
-    l0 += __shfl_xor_sync(FULL, l0, 1);
-    l0 += __shfl_xor_sync(FULL, l0, 2);
-    l1 += __shfl_xor_sync(FULL, l1, 1);
-    l1 += __shfl_xor_sync(FULL, l1, 2);
-    const float inv0 = 1.f / l0, inv1 = 1.f / l1;
-    if (row0 < n) {
-        uint32_t* dst = reinterpret_cast<uint32_t*>(a.out + ((int64_t)(q0 + row0) * a.num_heads + h) * D);
-#pragma unroll
-        for (int dn = 0; dn < DN; ++dn) dst[dn * 4 + t] = pack2<Tag>(o[dn][0] * inv0, o[dn][1] * inv0);
-    }
-    if (row1 < n) {
-        uint32_t* dst = reinterpret_cast<uint32_t*>(a.out + ((int64_t)(q0 + row1) * a.num_heads + h) * D);
-#pragma unroll
-        for (int dn = 0; dn < DN; ++dn) dst[dn * 4 + t] = pack2<Tag>(o[dn][2] * inv1, o[dn][3] * inv1);
+    umma::fence_before_sync();
+    __syncthreads();
+    if (warp == 5) {
+        umma::fence_after_sync();
+        umma::dealloc(tmem, kPfTmemCols);
     }
 }
 
@@ -317,7 +403,7 @@ extern "C" int pa_prefill(const void* q, const void* k_cache, const void* v_cach
     if (block_size != 16 && block_size != 32 && block_size != 64) return PA_ERR_UNSUPPORTED;
     if ((int64_t)num_blocks * block_size > INT32_MAX || (int64_t)max_blocks_per_seq * block_size > INT32_MAX)
         return PA_ERR_UNSUPPORTED;
-    if (max_blocks_per_seq > kPfMaxEntries || num_seqs > 65535 || num_heads > 65535) return PA_ERR_UNSUPPORTED;
+    if (num_seqs > 65535 || num_heads > 65535) return PA_ERR_UNSUPPORTED;
     if (num_seqs == 0 || max_query_len == 0) return PA_OK;
     if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start || !out)
         return PA_ERR_INVALID_ARG;
