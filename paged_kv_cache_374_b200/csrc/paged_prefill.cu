@@ -28,7 +28,7 @@
 // MMAs before freeing tensor memory.
 #include <cmath>
 
-#include "decode_engine.cuh"
+#include "decode_gqa.cuh"
 #include "pa_host.h"
 #include "tcgen05.cuh"
 
@@ -39,6 +39,83 @@ constexpr int kPfTok = 64;           // tokens per K/V tile
 constexpr int kPfThreads = 192;      // softmax warps 0-3, load warp 4, MMA warp 5
 constexpr uint32_t kPfTmemCols = 256;  // O at column 0, S/P buffers at 128 and 192
 constexpr float kPfRescaleLog2 = 8.f;
+
+#ifndef PA_PF_SPIN
+#define PA_PF_SPIN 1
+#endif
+
+// Bounded wait on an mbarrier phase: the suspending try_wait of the library, or
+// (PA_PF_SPIN) a poll of test_wait bounded by 2 s of the global timer.
+__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity) {
+#if PA_PF_SPIN
+    uint64_t t0;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    for (uint32_t i = 0;; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if ((i & 255u) == 255u) {
+            uint64_t t1;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
+            if (t1 - t0 > 2000000000ull) return false;
+        }
+    }
+#else
+    return mbar_wait(bar, parity);
+#endif
+}
+
+// The largest visible raw score of a row's tile (8 independent max chains).
+template <bool kDiag>
+__device__ __forceinline__ float tile_row_max(const float (&x)[kPfTok], int vis) {
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = (!kDiag || i <= vis) ? x[i] : -INFINITY;
+#pragma unroll
+    for (int t = 8; t < kPfTok; ++t)
+        if (!kDiag || t <= vis) m[t & 7] = fmaxf(m[t & 7], x[t]);
+#pragma unroll
+    for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+    return m[0];
+}
+
+// p_t = 2^(x_t c - m) for the row's tile (0 past the diagonal when kDiag), written
+// to tensor memory at `taddr` as P_hi (columns 0-31) and P_lo (32-63), two tokens
+// per column; returns the sum of the fp32 p_t.  Packed fp32x2 arithmetic.
+template <class Tag, bool kDiag>
+__device__ __forceinline__ float tile_row_p(const float (&x)[kPfTok], int vis, float c, float m, uint32_t taddr) {
+    const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m), neg1 = make_float2(-1.f, -1.f);
+    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {  // 32 tokens -> 16 hi and 16 lo columns
+        uint32_t ph[16], pl[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int t = 32 * half + 2 * k;
+            const float2 e = __ffma2_rn(make_float2(x[t], x[t + 1]), c2, nm2);
+            float2 p = make_float2(fast_exp2(e.x), fast_exp2(e.y));
+            if (kDiag) {
+                p.x = t <= vis ? p.x : 0.f;
+                p.y = t + 1 <= vis ? p.y : 0.f;
+            }
+            acc[k & 3] = __fadd2_rn(acc[k & 3], p);
+            ph[k] = MmaOps<Tag>::pack(p.x, p.y);
+            const float2 lo = __ffma2_rn(Tag::widen2(ph[k]), neg1, p);  // p - hi, exact
+            pl[k] = MmaOps<Tag>::pack(lo.x, lo.y);
+        }
+        umma::st16(taddr + 16 * half, ph);
+        umma::st16(taddr + 32 + 16 * half, pl);
+    }
+    acc[0] = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+    return acc[0].x + acc[0].y;
+}
 
 struct PrefillArgs {
     const uint16_t* q;    // [T][H][D]
@@ -128,13 +205,19 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
         return;
     }
 
-    // Q rows -> K-major swizzled tile; rows past the chunk are zero
+    // Q rows -> K-major swizzled tile; rows past the chunk are zero.  A negative
+    // scale is moved into the sign of q (exact), so the softmax sees scale >= 0.
     if (tid < kPfRows) {
         const bool live = tid < nrows;
+        const uint32_t flip = a.scale_log2 < 0.f ? 0x80008000u : 0u;
         const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)(q0 + q_first + (live ? tid : 0)) * a.num_heads + h) * D);
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) {
-            const uint4 v = live ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            uint4 v = live ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            v.x ^= flip;
+            v.y ^= flip;
+            v.z ^= flip;
+            v.w ^= flip;
             *reinterpret_cast<uint4*>(smem + (c >> 3) * Lay::kQHalf + tid * 128 + (((c & 7) ^ (tid & 7)) << 4)) = v;
         }
         fence_proxy_async_shared();
@@ -153,44 +236,52 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
 
     if (warp == 4) {
         // ---------------------------------------------------------------- loads
-        if (lane == 0) {
-            const int br = a.box_rows;
-            auto load = [&](const CUtensorMap* map, uint8_t* dst0, uint64_t* bar, int tile) {
-                const int t0 = tile * kPfTok;
-                uint32_t tx = 0;
-                for (int j = 0; j * br < kPfTok; ++j)
-                    if (t0 + j * br < L) tx += (uint32_t)(D / 64) * br * 128;
-                mbar_arrive_expect_tx(bar, tx);
-                for (int j = 0; j * br < kPfTok; ++j) {
-                    const int tj = t0 + j * br;
-                    if (tj >= L) break;
-                    const int row = __ldg(tab + tj / bs) * bs + tj % bs;
+        // Lane i < 64 / box_rows owns box i of every tile: it reads that box's table
+        // entry (all lanes at once, ahead of the wait for the free stage) and issues
+        // the box's copies; lane 0 posts the byte count first.
+        const int br = a.box_rows;
+        const int nbox = kPfTok / br;
+        const uint32_t box_bytes = (uint32_t)(D / 64) * br * 128;
+        bool ok = true;
+        int issued_k = 0, issued_v = 0;
+        auto row_of = [&](int tile) {  // this lane's cache row for `tile`, or -1
+            const int tj = tile * kPfTok + lane * br;
+            return (lane < nbox && tj < L) ? __ldg(tab + tj / bs) * bs + tj % bs : -1;
+        };
+        auto load = [&](const CUtensorMap* map, uint8_t* dst0, uint64_t* bar, int row) {
+            const uint32_t n = __popc(__ballot_sync(FULL, row >= 0));
+            if (lane == 0) mbar_arrive_expect_tx(bar, n * box_bytes);
+            __syncwarp();
+            if (row >= 0) {
 #pragma unroll
-                    for (int hh = 0; hh < D / 64; ++hh)
-                        tma_load_3d(dst0 + hh * Lay::kTHalf + j * br * 128, map, hh * 64, kv_head, row, bar);
-                }
-            };
-            bool ok = true;
-            int issued_k = 0, issued_v = 0;
-            for (int j = 0; j < ntiles; ++j) {
-                const int st = j & 1;
-                if (j >= 2) ok = mbar_wait(&bars[kBarKEmpty + st], ((j >> 1) + 1) & 1) && !*abort_flag;
-                if (!ok) break;
-                load(&kmap, smem + Lay::kOffK + st * Lay::kTile, &bars[kBarKFull + st], j);
-                issued_k = j + 1;
-                if (j >= 2) ok = mbar_wait(&bars[kBarVEmpty + st], ((j >> 1) + 1) & 1) && !*abort_flag;
-                if (!ok) break;
-                load(&vmap, smem + Lay::kOffV + st * Lay::kTile, &bars[kBarVFull + st], j);
-                issued_v = j + 1;
+                for (int hh = 0; hh < D / 64; ++hh)
+                    tma_load_3d(dst0 + hh * Lay::kTHalf + lane * br * 128, map, hh * 64, kv_head, row, bar);
             }
+        };
+        int row = row_of(0);
+        for (int j = 0; j < ntiles; ++j) {
+            const int st = j & 1;
+            if (j >= 2) ok = __all_sync(FULL, pf_wait(&bars[kBarKEmpty + st], ((j >> 1) + 1) & 1) && !*abort_flag);
+            if (!ok) break;
+            load(&kmap, smem + Lay::kOffK + st * Lay::kTile, &bars[kBarKFull + st], row);
+            issued_k = j + 1;
+            const int next = j + 1 < ntiles ? row_of(j + 1) : -1;  // in flight during the wait below
+            if (j >= 2) ok = __all_sync(FULL, pf_wait(&bars[kBarVEmpty + st], ((j >> 1) + 1) & 1) && !*abort_flag);
+            if (!ok) break;
+            load(&vmap, smem + Lay::kOffV + st * Lay::kTile, &bars[kBarVFull + st], row);
+            issued_v = j + 1;
+            row = next;
+        }
+        if (lane == 0) {
             if (!ok) {
                 report(a.err_word, PA_DEVERR_TIMEOUT);
                 *abort_flag = 1;
             }
             // every copy still in flight lands before the CTA may exit
-            for (int j = max(0, issued_k - 2); j < issued_k; ++j) mbar_wait(&bars[kBarKFull + (j & 1)], (j >> 1) & 1);
-            for (int j = max(0, issued_v - 2); j < issued_v; ++j) mbar_wait(&bars[kBarVFull + (j & 1)], (j >> 1) & 1);
+            for (int j = max(0, issued_k - 2); j < issued_k; ++j) pf_wait(&bars[kBarKFull + (j & 1)], (j >> 1) & 1);
+            for (int j = max(0, issued_v - 2); j < issued_v; ++j) pf_wait(&bars[kBarVFull + (j & 1)], (j >> 1) & 1);
         }
+        __syncwarp();
     } else if (warp == 5) {
         // ----------------------------------------------------------------- MMAs
         const uint32_t qa = smem_u32(smem);
@@ -206,7 +297,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             umma::commit(&bars[kBarKEmpty + (j & 1)]);
         };
         auto wait = [&](int bar, uint32_t parity) {  // whole warp
-            const bool ok = mbar_wait(&bars[bar], parity) && !*abort_flag;
+            const bool ok = pf_wait(&bars[bar], parity) && !*abort_flag;
             return __all_sync(FULL, ok);
         };
         bool ok = true;
@@ -242,8 +333,8 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
 #pragma unroll
                 for (int kk = 0; kk < kPfTok / 16; ++kk) {
                     const uint64_t db = umma::desc_sw128(va + kk * 2048, Lay::kTHalf, 1024);
-                    umma::mma_ts(tO, tp + kk * 8, db, kIdO, (j > 0 || kk > 0) ? 1u : 0u);
-                    umma::mma_ts(tO, tp + 32 + kk * 8, db, kIdO, 1u);
+                    umma::mma_ts(tO, tp + kk * 8, db, kIdO, (j > 0 || kk > 0) ? 1u : 0u);  // P_hi V
+                    umma::mma_ts(tO, tp + 32 + kk * 8, db, kIdO, 1u);                      // P_lo V
                 }
                 umma::commit(&bars[kBarVEmpty + st]);
                 umma::commit(&bars[kBarOFull + st]);
@@ -264,7 +355,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
                 *abort_flag = 1;
             }
             umma::commit(&bars[kBarDrain]);  // every MMA issued completes before TMEM is freed
-            mbar_wait(&bars[kBarDrain], 0);
+            pf_wait(&bars[kBarDrain], 0);
         }
         __syncwarp();
     } else {
@@ -272,12 +363,12 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
         const int r = tid;
         const int pos = base_pos + min(r, nrows - 1);
         const uint32_t lrow = (uint32_t)(warp * 32) << 16;
-        const float c = a.scale_log2;
+        const float c = fabsf(a.scale_log2);
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < ntiles; ++j) {
             const int b = j & 1;
-            ok = __all_sync(FULL, mbar_wait(&bars[kBarSFull + b], (j >> 1) & 1) && !*abort_flag);
+            ok = __all_sync(FULL, pf_wait(&bars[kBarSFull + b], (j >> 1) & 1) && !*abort_flag);
             if (!ok) break;
             umma::fence_after_sync();
             uint32_t sv[2][32];
@@ -285,20 +376,21 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             umma::ld32(tS + b * 64 + 32 + lrow, sv[1]);
             umma::wait_ld();
             const int t0 = j * kPfTok;
-            float x[kPfTok];
-            float mt = -INFINITY;
+            // every row of the CTA sees the whole tile unless it reaches the diagonal
+            const bool diag = t0 + kPfTok - 1 > base_pos;
+            const int vis = diag ? pos - t0 : kPfTok - 1;  // last visible token of the tile, this row
+            float x[kPfTok];  // raw scores
 #pragma unroll
-            for (int t = 0; t < kPfTok; ++t) {
-                x[t] = t0 + t <= pos ? __uint_as_float(sv[t >> 5][t & 31]) * c : -INFINITY;
-                mt = fmaxf(mt, x[t]);
-            }
+            for (int t = 0; t < kPfTok; ++t) x[t] = __uint_as_float(sv[t >> 5][t & 31]);
+            float mt = diag ? tile_row_max<true>(x, vis) : tile_row_max<false>(x, vis);
+            mt = mt == -INFINITY ? -INFINITY : mt * c;  // the tile max in log2 units
             const bool need = mt > m_used + kPfRescaleLog2;  // always on the first tile
             if (__any_sync(FULL, need)) {
                 const float m_new = need ? mt : m_used;
                 if (j > 0) {
                     const float alpha = fast_exp2(m_used - m_new);
                     // PV_{j-1} must have landed in O before it is rescaled
-                    ok = __all_sync(FULL, mbar_wait(&bars[kBarOFull + ((j - 1) & 1)], ((j - 1) >> 1) & 1) &&
+                    ok = __all_sync(FULL, pf_wait(&bars[kBarOFull + ((j - 1) & 1)], ((j - 1) >> 1) & 1) &&
                                               !*abort_flag);
                     if (!ok) break;
                     umma::fence_after_sync();
@@ -316,26 +408,13 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
                 }
                 m_used = m_new;
             }
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {  // 32 tokens -> 16 hi and 16 lo columns
-                uint32_t ph[16], pl[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float p0 = fast_exp2(x[32 * half + 2 * k] - m_used);
-                    const float p1 = fast_exp2(x[32 * half + 2 * k + 1] - m_used);
-                    l += p0 + p1;
-                    ph[k] = pack2<Tag>(p0, p1);
-                    const float2 hv = Tag::widen2(ph[k]);
-                    pl[k] = pack2<Tag>(p0 - hv.x, p1 - hv.y);
-                }
-                umma::st16(tS + b * 64 + 16 * half + lrow, ph);
-                umma::st16(tS + b * 64 + 32 + 16 * half + lrow, pl);
-            }
+            l += diag ? tile_row_p<Tag, true>(x, vis, c, m_used, tS + b * 64 + lrow)
+                      : tile_row_p<Tag, false>(x, vis, c, m_used, tS + b * 64 + lrow);
             umma::wait_st();
             umma::fence_before_sync();
             mbar_arrive(&bars[kBarPFull + b]);
         }
-        if (ok) ok = __all_sync(FULL, mbar_wait(&bars[kBarOLast], 0) && !*abort_flag);
+        if (ok) ok = __all_sync(FULL, pf_wait(&bars[kBarOLast], 0) && !*abort_flag);
         if (ok) {
             umma::fence_after_sync();
             const float inv = 1.f / l;
@@ -349,8 +428,9 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         const float* f = reinterpret_cast<const float*>(o + 8 * v);
-                        dst[cc * 4 + v] = make_uint4(pack2<Tag>(f[0] * inv, f[1] * inv), pack2<Tag>(f[2] * inv, f[3] * inv),
-                                                     pack2<Tag>(f[4] * inv, f[5] * inv), pack2<Tag>(f[6] * inv, f[7] * inv));
+                        dst[cc * 4 + v] = make_uint4(
+                            MmaOps<Tag>::pack(f[0] * inv, f[1] * inv), MmaOps<Tag>::pack(f[2] * inv, f[3] * inv),
+                            MmaOps<Tag>::pack(f[4] * inv, f[5] * inv), MmaOps<Tag>::pack(f[6] * inv, f[7] * inv));
                     }
                 }
             }
