@@ -284,14 +284,21 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
         __syncwarp();
     } else if (warp == 5) {
         // ----------------------------------------------------------------- MMAs
-        const uint32_t qa = smem_u32(smem);
+        // Operand descriptors, built once: an MMA's descriptor is its stage's plus
+        // the byte offset / 16 in the start-address field (no carry: shared
+        // addresses stay below 2^18).
+        const uint64_t dq = umma::desc_sw128(smem_u32(smem), 16, 1024);
+        const uint64_t dk0 = umma::desc_sw128(smem_u32(smem + Lay::kOffK), 16, 1024);
+        const uint64_t dv0 = umma::desc_sw128(smem_u32(smem + Lay::kOffV), Lay::kTHalf, 1024);
+        constexpr uint64_t kStageStep = Lay::kTile >> 4;  // the second stage of a ring
         auto issue_s = [&](int j) {  // lane 0: S_j = Q K_j^T into buffer j & 1
-            const uint32_t ka = smem_u32(smem + Lay::kOffK + (j & 1) * Lay::kTile);
+            const uint64_t bk = dk0 + (j & 1) * kStageStep;
+            const uint32_t d = tS + (j & 1) * 64;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                const uint64_t da = umma::desc_sw128(qa + (kk >> 2) * Lay::kQHalf + (kk & 3) * 32, 16, 1024);
-                const uint64_t db = umma::desc_sw128(ka + (kk >> 2) * Lay::kTHalf + (kk & 3) * 32, 16, 1024);
-                umma::mma_ss(tS + (j & 1) * 64, da, db, kIdS, kk > 0 ? 1u : 0u);
+                constexpr int kQStep = Lay::kQHalf >> 4, kTStep = Lay::kTHalf >> 4;
+                umma::mma_ss(d, dq + (uint64_t)((kk >> 2) * kQStep + (kk & 3) * 2),
+                             bk + (uint64_t)((kk >> 2) * kTStep + (kk & 3) * 2), kIdS, kk > 0 ? 1u : 0u);
             }
             umma::commit(&bars[kBarSFull + (j & 1)]);
             umma::commit(&bars[kBarKEmpty + (j & 1)]);
@@ -328,11 +335,11 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             if (!ok) break;
             umma::fence_after_sync();
             if (lane == 0) {
-                const uint32_t va = smem_u32(smem + Lay::kOffV + st * Lay::kTile);
+                const uint64_t bv = dv0 + st * kStageStep;
                 const uint32_t tp = tS + st * 64;
 #pragma unroll
                 for (int kk = 0; kk < kPfTok / 16; ++kk) {
-                    const uint64_t db = umma::desc_sw128(va + kk * 2048, Lay::kTHalf, 1024);
+                    const uint64_t db = bv + (uint64_t)(kk * (2048 >> 4));  // 16 tokens further
                     umma::mma_ts(tO, tp + kk * 8, db, kIdO, (j > 0 || kk > 0) ? 1u : 0u);  // P_hi V
                     umma::mma_ts(tO, tp + 32 + kk * 8, db, kIdO, 1u);                      // P_lo V
                 }
