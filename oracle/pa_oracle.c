@@ -532,7 +532,12 @@ static void* prefill_worker(void* p) {
             j->error = 1;
             continue;
         }
-        if (attend(j, s, h, pj->q + (qi * j->num_heads + h) * d, pos + 1, j->out + w * d, qd, x) != 0)
+#if PA_ORACLE_MUTANT == 12
+        const int64_t nvis = pos + 2 < len ? pos + 2 : len; /* planted: sees one token past its position */
+#else
+        const int64_t nvis = pos + 1; /* tokens 0 .. pos */
+#endif
+        if (attend(j, s, h, pj->q + (qi * j->num_heads + h) * d, nvis, j->out + w * d, qd, x) != 0)
             j->error = 1;
     }
     free(qd);

@@ -6,14 +6,14 @@ The mistakes are compiled into copies of the C oracle with PA_ORACLE_MUTANT=n:
   5 per-block softmax sum (unnormalised)               6 softmax denominator left out
   7 fp16 exponent bias off by one                      8 cache write to the neighbouring slot
   9 newest-token slot one position late                10 floor instead of ceil for block counts
- 11 fp8 codes rounded toward zero
+ 11 fp8 codes rounded toward zero              12 causal mask one token late (prefill)
 """
 import pytest
 
 import oracle as oracle_pkg
 import pins
 
-MUTANTS = list(range(1, 12))
+MUTANTS = list(range(1, 13))
 
 
 @pytest.fixture(scope="module")
