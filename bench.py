@@ -52,6 +52,9 @@ def parse():
     p.add_argument("--num-seqs", type=int, default=None, help="truncate the batch (smaller profiling case)")
     p.add_argument("--kv-dtype", default="native", choices=["native", "fp8"],
                    help="fp8: the cache is stored as E4M3 codes (pa_reshape_and_cache_fp8 / pa_decode_fp8)")
+    p.add_argument("--shared-prefix", default="auto", choices=["auto", "off"],
+                   help="auto: sequences sharing prompt blocks (the beam workload) run through "
+                        "pa_decode_shared_prefix; off: plain pa_decode")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
     p.add_argument("--row", default="decode", choices=["decode", "copy_blocks", "swap", "prefill"],
@@ -194,7 +197,7 @@ def gpu_uuid(torch, device):
 FP8_INV_SCALE = 32.0  # fp8 caches: stored value = code / 32 (N(0,1) values use codes up to ~150)
 
 
-def build_step(name, device, partition_tokens, num_seqs=None, kv_dtype="native"):
+def build_step(name, device, partition_tokens, num_seqs=None, kv_dtype="native", shared=False):
     """Tables from the library's allocator, one step's slots via a1, tensors on
     the device.  Returns a dict of everything the timed loop needs."""
     import torch
@@ -229,12 +232,20 @@ def build_step(name, device, partition_tokens, num_seqs=None, kv_dtype="native")
             t[key] = (t[key].float() * FP8_INV_SCALE).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
     ws_bytes = pa.pa_decode_workspace_size(s, spec.num_heads, spec.num_kv_heads, spec.head_dim, bs,
                                            wl.max_blocks_per_seq, partition_tokens)
+    ptok = partition_tokens or pa.pa_decode_partition_tokens(s, spec.num_heads, spec.num_kv_heads, spec.head_dim, bs,
+                                                             wl.max_blocks_per_seq)
+    groups = None
+    if shared and kv_dtype == "native":
+        groups = pa.pa_find_shared_prefixes(tables, lens, bs, ptok)
+        if groups.num_groups == 0:
+            groups = None
     d = dict(
         wl=wl, spec=spec, alloc=alloc, tables_h=tables, lens_h=lens, slots_h=slots, a1_us=a1_us,
         tables=torch.from_numpy(tables).to(device), lens=torch.from_numpy(lens).to(device),
         slots=torch.from_numpy(slots).to(device), out=torch.empty_like(t["q"]),
         workspace=torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=device), ws_bytes=ws_bytes,
-        partition_tokens=partition_tokens, **t)
+        partition_tokens=partition_tokens, ptok=ptok, groups=groups,
+        group_dev=groups.to(device) if groups is not None else None, **t)
     return d
 
 
@@ -293,7 +304,8 @@ def run_native(args):
                                 timeout=__import__("datetime").timedelta(seconds=120))
     device = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(device)
-    st = build_step(args.workload, device, args.partition_tokens, args.num_seqs, args.kv_dtype)
+    st = build_step(args.workload, device, args.partition_tokens, args.num_seqs, args.kv_dtype,
+                    shared=args.shared_prefix == "auto")
     fp8 = args.kv_dtype == "fp8"
     ks = vs = 1.0 / FP8_INV_SCALE
     spec = st["spec"]
@@ -305,8 +317,15 @@ def run_native(args):
         else:
             pa.pa_reshape_and_cache(k, v, slots, st["k_cache"], st["v_cache"], stream=stream)
 
-    def k2(q, tables, lens):
-        if fp8:
+    def k2(q, tables, lens, groups=None):
+        g = st["groups"]
+        if g is not None:
+            start, offs, mem = groups if groups is not None else st["group_dev"]
+            pa.pa_decode_shared_prefix(q, st["k_cache"], st["v_cache"], tables, lens, spec.scale, spec.num_kv_heads,
+                                       st["out"], start, offs, mem, g.num_groups, g.max_group_size,
+                                       g.max_shared_tokens, workspace=st["workspace"],
+                                       partition_tokens=st["partition_tokens"], stream=stream)
+        elif fp8:
             pa.pa_decode_fp8(q, st["k_cache"], st["v_cache"], tables, lens, spec.scale, ks, vs, spec.num_kv_heads,
                              st["out"], workspace=st["workspace"], partition_tokens=st["partition_tokens"],
                              stream=stream)
@@ -360,11 +379,26 @@ def run_native(args):
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = out_h.numel() * out_h.element_size()
 
+    grp_dev = None
+    if st["groups"] is not None:  # the grouping is redone from the host tables every step
+        grp_dev = [torch.empty(st["spec"].num_seqs + 1, dtype=torch.int32, device=device) for _ in range(3)]
+        grp_h = [torch.empty(st["spec"].num_seqs + 1, dtype=torch.int32).pin_memory() for _ in range(3)]
+        h2d += 4 * (2 * st["spec"].num_seqs + 1 + st["groups"].num_groups + 1)
+
     def e2e_step():
         for k, v in host.items():
             dev_in[k].copy_(v, non_blocking=True)
+        groups = None
+        if grp_dev is not None:
+            g = pa.pa_find_shared_prefixes(st["tables_h"], st["lens_h"], spec.block_size, st["ptok"])
+            groups = []
+            for hbuf, dbuf, arr in zip(grp_h, grp_dev, (g.seq_start, g.group_offsets, g.group_members)):
+                n = len(arr)
+                hbuf[:n].copy_(torch.from_numpy(arr))
+                dbuf[:n].copy_(hbuf[:n], non_blocking=True)
+                groups.append(dbuf[:n])
         k1(dev_in["k"], dev_in["v"], dev_in["slots"])
-        k2(dev_in["q"], dev_in["tables"], dev_in["lens"])
+        k2(dev_in["q"], dev_in["tables"], dev_in["lens"], groups)
         out_h.copy_(st["out"], non_blocking=True)
 
     e2e_steps = max(1, min(args.steps, 500))
@@ -390,7 +424,7 @@ def run_native(args):
         st["partition_tokens"] or pa.pa_decode_partition_tokens(spec.num_seqs, spec.num_heads, spec.num_kv_heads,
                                                                  spec.head_dim, spec.block_size,
                                                                  st["wl"].max_blocks_per_seq)))
-    launches_per_step = 2 + (1 if nparts_max > 1 else 0)
+    launches_per_step = 2 + (1 if nparts_max > 1 else 0) + (1 if st["groups"] is not None else 0)
     result = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -404,7 +438,10 @@ def run_native(args):
         "vs_baseline": None,
         "dtype": spec.dtype + ("+e4m3 cache" if fp8 else ""),
         "data": "synthetic",
-        "config": dict(static_config(st["wl"], args, world), **({"kv_cache": "fp8 e4m3, scale 1/32"} if fp8 else {})),
+        "config": dict(static_config(st["wl"], args, world), **({"kv_cache": "fp8 e4m3, scale 1/32"} if fp8 else {}),
+                       **({"shared_prefix": "pa_decode_shared_prefix: %d group(s), %d shared tokens" % (
+                           st["groups"].num_groups, st["groups"].max_shared_tokens)} if st["groups"] is not None
+                          else {})),
         "detail": {
             "kv_gbs": round(achieved, 1), "frac_of_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
             "kv_bytes_per_step": ab["unique"], "logical_kv_bytes_per_step": ab["logical"],
@@ -412,10 +449,12 @@ def run_native(args):
             "e2e_ms_per_step": round(e2e_ms, 4),
         },
         "roofline": {
-            "kernel": "paged_decode_mha_kernel + paged_decode_merge_kernel (timed together: one pa_decode call)",
+            "kernel": ("shared-prefix kernel + paged_decode_kernel + paged_decode_merge_kernel (timed together: one "
+                       "pa_decode_shared_prefix call)" if st["groups"] is not None else
+                       "paged_decode_kernel + paged_decode_merge_kernel (timed together: one pa_decode call)"),
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
             "unit": "GB/s", "frac": round(achieved / peak, 4),
-            "traffic": None if fp8 else profiled_traffic(ab["unique_tokens"]),
+            "traffic": None if (fp8 or st["groups"] is not None) else profiled_traffic(ab["unique_tokens"]),
         },
         "e2e": {"value": round(job_throughput(world, tokens_per_step, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

@@ -180,6 +180,61 @@ int pa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, c
                       int num_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
                       int dtype, int partition_tokens, int32_t* err_word, void* stream);
 
+/* ------------------------------------------------------- shared prefixes */
+
+/*
+ * pa_decode_shared_prefix -- pa_decode for batches whose sequences share a
+ * prefix through the same physical blocks (a beam fork holding the prompt's
+ * blocks by reference, P3 §四; requests reusing a cached prompt, P3 §三).  The
+ * result is pa_decode's, to rounding: the shared part is attended once per kv
+ * head for the whole group (on the tensor cores, the group's queries as the rows
+ * of one matrix) instead of once per sequence, and merged with each sequence's
+ * own suffix by the same partial-softmax merge that joins split partitions.
+ *
+ * Arguments as pa_decode, plus (all device arrays):
+ *   seq_start      [num_seqs] int32: 0, or the tokens sequence s shares with
+ *                  its group -- a multiple of the partition size below
+ *                  context_lens[s].  Tokens below it must use the same physical
+ *                  blocks as every other member of the group.
+ *   num_groups     groups of sequences sharing a prefix (host int; 0 = pa_decode)
+ *   group_offsets  [num_groups + 1] int32: group g is
+ *   group_members  group_members[group_offsets[g] .. group_offsets[g+1]) (sequence
+ *                  indices); every member has the same seq_start
+ *   max_group_size, max_shared_tokens  host ints bounding the arrays (launch sizes)
+ * pa_find_shared_prefixes builds these from host block tables.  partition_tokens
+ * must be the one the workspace was sized with (0 = default).  A seq_start that
+ * is not a multiple of the partition below the length is ignored (the whole
+ * sequence runs in the per-sequence kernel) and reported as
+ * PA_DEVERR_LEN_RANGE; a member whose seq_start differs from its group's gets no
+ * shared partials and is reported the same way (its output is then undefined).
+ */
+int pa_decode_shared_prefix(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                            const int32_t* context_lens, float scale, int num_kv_heads, void* out, int num_seqs,
+                            int num_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                            int dtype, const int32_t* seq_start, int num_groups, const int32_t* group_offsets,
+                            const int32_t* group_members, int max_group_size, int max_shared_tokens,
+                            int partition_tokens, void* workspace, size_t workspace_bytes, int32_t* err_word,
+                            void* stream);
+
+/*
+ * pa_find_shared_prefixes -- host-side grouping for pa_decode_shared_prefix.
+ * Sequences whose first partition (partition_tokens tokens) maps to the same
+ * physical blocks form a group; the group shares the longest run of whole
+ * partitions that all members map to the same blocks and that lies strictly
+ * below every member's length.  Groups of one sequence are not formed.
+ *   block_tables  [num_seqs][max_blocks_per_seq] int32, host;  context_lens host
+ *   seq_start     [num_seqs] out (0 outside groups)
+ *   group_offsets [num_seqs + 1] out;  group_members [num_seqs] out
+ *   num_groups, max_group_size, max_shared_tokens  out
+ * partition_tokens must be a positive multiple of block_size (the value passed
+ * to the decode call, or pa_decode_partition_tokens(...)).  Table entries are
+ * compared, not range-checked (the device kernels check them).
+ */
+int pa_find_shared_prefixes(const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                            int max_blocks_per_seq, int block_size, int partition_tokens, int32_t* seq_start,
+                            int32_t* group_offsets, int32_t* group_members, int* num_groups, int* max_group_size,
+                            int* max_shared_tokens);
+
 /* ---------------------------------------------------------------- fp8 cache */
 
 /*

@@ -52,6 +52,10 @@ _sig("pa_decode_fp8", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_fl
      _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
 _sig("pa_prefill", _i32, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
      _i32, _i32, _vp, _vp)
+_sig("pa_decode_shared_prefix", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32, _i32, _i32, _i32, _i32,
+     _i32, _i32, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
+_sig("pa_find_shared_prefixes", _i32, _i32p, _i32p, _i32, _i32, _i32, _i32, _i32p, _i32p, _i32p,
+     ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int))
 _sig("pa_allocator_create", _vp, _i32, _i32p)
 _sig("pa_allocator_destroy", None, _vp)
 _sig("pa_num_required_blocks", _i32, _i32, _i32)
@@ -110,6 +114,12 @@ def _dev(t, name, dtype=None):
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _h32(a: np.ndarray):
+    """Host pointer of a C-contiguous int32 numpy array."""
+    assert a.dtype == np.int32 and a.flags.c_contiguous
+    return a.ctypes.data_as(_i32p)
 
 
 def _stream(stream, like):
@@ -178,6 +188,77 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_hea
                         s, h, d, bs, nb, mb, dt, int(partition_tokens), ws_ptr, ws_bytes,
                         _dev(err_word, "err_word", torch.int32), _stream(stream, q))
     _check(st, "pa_decode")
+    return out
+
+
+class SharedPrefixes:
+    """Result of pa_find_shared_prefixes (host numpy arrays)."""
+
+    def __init__(self, seq_start, group_offsets, group_members, num_groups, max_group_size, max_shared_tokens):
+        self.seq_start = seq_start
+        self.group_offsets = group_offsets
+        self.group_members = group_members
+        self.num_groups = num_groups
+        self.max_group_size = max_group_size
+        self.max_shared_tokens = max_shared_tokens
+
+    def to(self, device):
+        """The three arrays as int32 tensors on ``device`` (a tuple)."""
+        import torch
+        return tuple(torch.from_numpy(np.ascontiguousarray(x)).to(device)
+                     for x in (self.seq_start, self.group_offsets, self.group_members))
+
+
+def pa_find_shared_prefixes(block_tables: np.ndarray, context_lens: np.ndarray, block_size: int,
+                            partition_tokens: int) -> SharedPrefixes:
+    """Host grouping of sequences that share whole partitions through the same blocks."""
+    tb = np.ascontiguousarray(block_tables, dtype=np.int32)
+    ln = np.ascontiguousarray(context_lens, dtype=np.int32)
+    s, mb = tb.shape
+    start = np.zeros(s, dtype=np.int32)
+    offs = np.zeros(s + 1, dtype=np.int32)
+    members = np.zeros(max(s, 1), dtype=np.int32)
+    ng, mg, mt = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    st = _lib.pa_find_shared_prefixes(_h32(tb), _h32(ln), s, mb, block_size, partition_tokens, _h32(start),
+                                      _h32(offs), _h32(members), ctypes.byref(ng), ctypes.byref(mg),
+                                      ctypes.byref(mt))
+    _check(st, "pa_find_shared_prefixes")
+    n = int(ng.value)
+    return SharedPrefixes(start, offs[: n + 1].copy(), members[: int(offs[n])].copy(), n, int(mg.value),
+                          int(mt.value))
+
+
+def pa_decode_shared_prefix(q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out, seq_start,
+                            group_offsets, group_members, num_groups, max_group_size, max_shared_tokens,
+                            workspace=None, partition_tokens=0, err_word=None, stream=None):
+    """pa_decode with the shared prefixes of groups attended once per group
+    (seq_start / group_offsets / group_members: int32 device tensors, e.g. from
+    ``pa_find_shared_prefixes(...).to(device)``).  Returns ``out``."""
+    import torch
+    s, h, d = q.shape
+    nb, bs, hk, d2 = k_cache.shape
+    if hk != num_kv_heads or d2 != d or v_cache.shape != k_cache.shape or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [S, MB] and context_lens [S]")
+    mb = block_tables.shape[1]
+    dt = _dtype_code(q)
+    for t in (k_cache, v_cache, out):
+        if t.dtype != q.dtype:
+            raise TypeError("q, the caches and out must share one dtype")
+    need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _lib.pa_decode_shared_prefix(
+        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), _dev(context_lens, "context_lens", torch.int32),
+        float(scale), hk, _dev(out, "out"), s, h, d, bs, nb, mb, dt, _dev(seq_start, "seq_start", torch.int32),
+        int(num_groups), _dev(group_offsets, "group_offsets", torch.int32),
+        _dev(group_members, "group_members", torch.int32), int(max_group_size), int(max_shared_tokens),
+        int(partition_tokens), _dev(workspace, "workspace"), ws_bytes, _dev(err_word, "err_word", torch.int32),
+        _stream(stream, q))
+    _check(st, "pa_decode_shared_prefix")
     return out
 
 

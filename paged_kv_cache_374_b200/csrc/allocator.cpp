@@ -6,6 +6,8 @@
 // ring has exactly num_blocks slots, enough because a block sits in the queue only
 // while its count is zero.  Every operation validates first and mutates second, so
 // a failing call leaves the allocator as it was.
+#include <algorithm>
+#include <climits>
 #include <cstdint>
 #include <cstdlib>
 #include <new>
@@ -299,6 +301,76 @@ int pa_swap_plan(pa_allocator* from, pa_allocator* to, int32_t* table_row, int n
         pairs[2 * i + 1] = fresh;
         table_row[i] = fresh;
     }
+    return PA_OK;
+}
+
+int pa_find_shared_prefixes(const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                            int max_blocks_per_seq, int block_size, int partition_tokens, int32_t* seq_start,
+                            int32_t* group_offsets, int32_t* group_members, int* num_groups, int* max_group_size,
+                            int* max_shared_tokens) {
+    if (num_seqs < 0 || max_blocks_per_seq < 0 || block_size <= 0 || partition_tokens <= 0 ||
+        partition_tokens % block_size != 0 || !num_groups || !max_group_size || !max_shared_tokens)
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs > 0 && (!block_tables || !context_lens || !seq_start || !group_offsets || !group_members))
+        return PA_ERR_INVALID_ARG;
+    const int P = partition_tokens, epp = partition_tokens / block_size;  // table entries per partition
+    const int64_t maxlen = (int64_t)max_blocks_per_seq * block_size;
+    auto row = [&](int s) { return block_tables + (int64_t)s * max_blocks_per_seq; };
+    auto same = [&](int x, int y, int k) {  // partition k of x and y uses the same blocks
+        return std::equal(row(x) + (int64_t)k * epp, row(x) + (int64_t)(k + 1) * epp, row(y) + (int64_t)k * epp);
+    };
+    // candidates: at least one whole partition strictly below the length
+    std::vector<int> cand;
+    for (int s = 0; s < num_seqs; ++s) {
+        seq_start[s] = 0;
+        if (context_lens[s] > P && context_lens[s] <= maxlen) cand.push_back(s);
+    }
+    int ng = 0, pos = 0, maxg = 0, maxtok = 0;
+    group_offsets[0] = 0;
+    auto kmax = [&](int x) { return (context_lens[x] - 1) / P; };  // whole partitions below the length
+    auto emit = [&](std::vector<int>& mem, int k) {
+        std::sort(mem.begin(), mem.end());
+        for (int x : mem) {
+            seq_start[x] = k * P;
+            group_members[pos++] = x;
+        }
+        group_offsets[++ng] = pos;
+        maxg = std::max(maxg, (int)mem.size());
+        maxtok = std::max(maxtok, k * P);
+    };
+    // `mem` (two or more) share partitions [0, k).  Members that also share
+    // partition k with at least one other member split off with a longer prefix;
+    // the rest form a group sharing k partitions.
+    std::vector<std::pair<std::vector<int>, int>> work;
+    auto split = [&](std::vector<int> mem, int k) {
+        std::vector<int> rest, ext;
+        for (int x : mem) (kmax(x) > k ? ext : rest).push_back(x);
+        std::sort(ext.begin(), ext.end(), [&](int x, int y) {
+            const int32_t *a = row(x) + (int64_t)k * epp, *b = row(y) + (int64_t)k * epp;
+            for (int i = 0; i < epp; ++i)
+                if (a[i] != b[i]) return a[i] < b[i];
+            return x < y;
+        });
+        for (size_t i = 0; i < ext.size();) {
+            size_t j = i + 1;
+            while (j < ext.size() && same(ext[i], ext[j], k)) ++j;
+            if (j - i >= 2)
+                work.emplace_back(std::vector<int>(ext.begin() + i, ext.begin() + j), k + 1);
+            else
+                rest.push_back(ext[i]);
+            i = j;
+        }
+        if (rest.size() >= 2 && k > 0) emit(rest, k);
+    };
+    work.emplace_back(cand, 0);
+    while (!work.empty()) {
+        auto item = std::move(work.back());
+        work.pop_back();
+        split(std::move(item.first), item.second);
+    }
+    *num_groups = ng;
+    *max_group_size = maxg;
+    *max_shared_tokens = maxtok;
     return PA_OK;
 }
 

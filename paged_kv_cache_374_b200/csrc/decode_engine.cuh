@@ -60,6 +60,10 @@ struct DecodeArgs {
     int max_blocks_per_seq;
     int partition_tokens;
     int num_partitions;  // Pmax: partitions allotted per (s, h) in the workspace
+    // Nullable.  seq_start[s] > 0: the partitions of sequence s below token
+    // seq_start[s] (a multiple of partition_tokens below context_lens[s]) are
+    // already in the workspace (a shared prefix); this launch runs the rest.
+    const int32_t* seq_start;
 };
 
 enum UnitKind { kUnitNone = 0, kUnitNormal = 1, kUnitZero = 2, kUnitNaN = 3 };
@@ -111,6 +115,14 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 }
 
 // Decode claim index u into a unit (warp-uniform; reads the schedule in smem).
+// First partition this launch runs for sequence s (0 unless a valid seq_start).
+__device__ __forceinline__ int first_partition(const DecodeArgs& a, int s, int L) {
+    if (!a.seq_start) return 0;
+    const int st = __ldg(a.seq_start + s);
+    const int P = a.partition_tokens;
+    return (st > 0 && st < L && L <= a.max_blocks_per_seq * a.block_size && st % P == 0) ? st / P : 0;
+}
+
 __device__ __forceinline__ Unit decode_unit(int u, const DecodeArgs& a, const int* s_cum, const uint32_t* s_key,
                                             const int* s_len, int TOK) {
     Unit U;
@@ -139,15 +151,16 @@ __device__ __forceinline__ Unit decode_unit(int u, const DecodeArgs& a, const in
         s = (int)(s_key[idx] & 0xfffu);
         p = s_cum[s + 1] - s_cum[s];
     }
+    const int L = s_len[s];
+    const int p0 = first_partition(a, s, L);
     U.s = s;
     U.h = h;
-    U.p = p;
-    U.np = s_cum[s + 1] - s_cum[s] + 1;
-    const int L = s_len[s];
+    U.p = p0 + p;
+    U.np = p0 + s_cum[s + 1] - s_cum[s] + 1;
     const int maxlen = a.max_blocks_per_seq * a.block_size;
     U.kind = (L < 0 || L > maxlen) ? kUnitNaN : (L == 0 ? kUnitZero : kUnitNormal);
     const int P = a.partition_tokens;
-    U.t_begin = p * P;
+    U.t_begin = U.p * P;
     U.t_end = U.kind == kUnitNormal ? min(L, U.t_begin + P) : U.t_begin;
     U.nst = (U.t_end - U.t_begin + TOK - 1) / TOK;
     U.kv_head = (h * a.heads_per_unit) / a.group;
@@ -201,7 +214,10 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
             const bool normal = L > 0 && L <= maxlen;
             const int np = normal ? (L + P - 1) / P : 1;
             const int last = normal ? L - (np - 1) * P : 0;
-            s_cum[s] = np - 1;  // full partitions, scanned below
+            const int p0 = first_partition(a, s, L);
+            if (a.seq_start && blockIdx.x == 0 && p0 == 0 && a.seq_start[s] != 0)
+                report(a.err_word, PA_DEVERR_LEN_RANGE);  // unusable start: every partition runs here
+            s_cum[s] = np - 1 - p0;  // full partitions this launch runs, scanned below
             s_key[s] = ((uint32_t)(P - last) << 12) | (uint32_t)s;
         } else {
             s_key[s] = 0xffffffffu;

@@ -81,4 +81,25 @@ inline cudaError_t ensure_smem_limit(Kernel kernel, int bytes, std::atomic<uint6
     return e;
 }
 
+// The prefix half of a two-level decode (paged_prefill.cu): partials of the
+// shared partitions of every group member, written into the decode workspace.
+struct SharedPrefixLaunch {
+    const void* q;
+    const void* k_cache;
+    const void* v_cache;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    const int32_t* seq_start;
+    const int32_t* group_offsets;
+    const int32_t* group_members;
+    float* ws_m;
+    float* ws_l;
+    float* ws_o;
+    int32_t* err_word;
+    float scale;
+    int num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype;
+    int partition_tokens, num_partitions, num_groups, max_group_size, max_shared_tokens;
+};
+int launch_shared_prefix(const SharedPrefixLaunch& l, cudaStream_t stream);
+
 }  // namespace pa

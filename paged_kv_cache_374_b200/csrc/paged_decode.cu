@@ -187,6 +187,7 @@ int launch_engine(DecodeArgs args, const void* k_cache, const void* v_cache, int
         c.out += shoff * D;
         c.block_tables += (int64_t)s0 * args.max_blocks_per_seq;
         c.context_lens += s0;
+        if (c.seq_start) c.seq_start += s0;
         if (args.num_partitions > 1) {
             c.ws_m += shoff * args.num_partitions;
             c.ws_l += shoff * args.num_partitions;
@@ -373,4 +374,62 @@ extern "C" int pa_decode_fp8(const void* q, const void* k_cache, const void* v_c
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return dtype == PA_F16 ? launch_decode_fp8<F16Tag>(args, k_cache, v_cache, num_kv_heads, st)
                            : launch_decode_fp8<BF16Tag>(args, k_cache, v_cache, num_kv_heads, st);
+}
+
+extern "C" int pa_decode_shared_prefix(const void* q, const void* k_cache, const void* v_cache,
+                                       const int32_t* block_tables, const int32_t* context_lens, float scale,
+                                       int num_kv_heads, void* out, int num_seqs, int num_heads, int head_dim,
+                                       int block_size, int num_blocks, int max_blocks_per_seq, int dtype,
+                                       const int32_t* seq_start, int num_groups, const int32_t* group_offsets,
+                                       const int32_t* group_members, int max_group_size, int max_shared_tokens,
+                                       int partition_tokens, void* workspace, size_t workspace_bytes,
+                                       int32_t* err_word, void* stream) {
+    using namespace pa;
+    if (num_groups < 0 || max_group_size < 0 || max_shared_tokens < 0) return PA_ERR_INVALID_ARG;
+    DecodeArgs args;
+    const int rc = prepare_decode(args, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out,
+                                  num_seqs, num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype,
+                                  partition_tokens, workspace, workspace_bytes, err_word);
+    if (rc >= 0) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool shared = num_groups > 0 && max_shared_tokens > 0 && args.num_partitions > 1;
+    if (shared) {
+        if (!seq_start || !group_offsets || !group_members || !aligned4(seq_start) || !aligned4(group_offsets) ||
+            !aligned4(group_members) || max_group_size <= 0 || max_shared_tokens % args.partition_tokens != 0)
+            return PA_ERR_INVALID_ARG;
+        SharedPrefixLaunch l{};
+        l.q = q;
+        l.k_cache = k_cache;
+        l.v_cache = v_cache;
+        l.block_tables = block_tables;
+        l.context_lens = context_lens;
+        l.seq_start = seq_start;
+        l.group_offsets = group_offsets;
+        l.group_members = group_members;
+        l.ws_m = args.ws_m;
+        l.ws_l = args.ws_l;
+        l.ws_o = args.ws_o;
+        l.err_word = err_word;
+        l.scale = scale;
+        l.num_heads = num_heads;
+        l.num_kv_heads = num_kv_heads;
+        l.head_dim = head_dim;
+        l.block_size = block_size;
+        l.num_blocks = num_blocks;
+        l.max_blocks_per_seq = max_blocks_per_seq;
+        l.dtype = dtype;
+        l.partition_tokens = args.partition_tokens;
+        l.num_partitions = args.num_partitions;
+        l.num_groups = num_groups;
+        l.max_group_size = max_group_size;
+        l.max_shared_tokens = max_shared_tokens;
+        const int r = launch_shared_prefix(l, st);
+        if (r != PA_OK) return r;
+        args.seq_start = seq_start;
+    }
+    if (head_dim == 128)
+        return dtype == PA_F16 ? launch_decode<F16Tag, 128>(args, k_cache, v_cache, num_kv_heads, st)
+                               : launch_decode<BF16Tag, 128>(args, k_cache, v_cache, num_kv_heads, st);
+    return dtype == PA_F16 ? launch_decode<F16Tag, 64>(args, k_cache, v_cache, num_kv_heads, st)
+                           : launch_decode<BF16Tag, 64>(args, k_cache, v_cache, num_kv_heads, st);
 }

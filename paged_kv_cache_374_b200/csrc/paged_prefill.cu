@@ -126,6 +126,17 @@ struct PrefillArgs {
     int32_t* err_word;
     float scale_log2;
     int num_heads, group, block_size, box_rows, num_blocks, max_blocks_per_seq;
+    // shared-prefix mode (the prefix half of a two-level decode): group g's member
+    // sequences group_members[group_offsets[g] .. group_offsets[g+1]) share the
+    // partitions below seq_start[member]; each CTA computes one partition of one
+    // kv head for up to 128 (member, query head) rows and leaves partials
+    const int32_t* group_offsets;
+    const int32_t* group_members;
+    const int32_t* seq_start;
+    float* ws_m;
+    float* ws_l;
+    float* ws_o;
+    int partition_tokens, num_partitions, max_shared_partitions;
 };
 
 template <int D>
@@ -154,7 +165,7 @@ enum : int {
     kBarDrain = 15,   // every MMA issued has completed
 };
 
-template <class Tag, int D>
+template <class Tag, int D, bool kShared>
 __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const PrefillArgs a,
                                                                       const __grid_constant__ CUtensorMap kmap,
                                                                       const __grid_constant__ CUtensorMap vmap) {
@@ -169,38 +180,89 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBars);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + Lay::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-
-    const int s = blockIdx.z, h = blockIdx.y;
-    const int qt = gridDim.x - 1 - blockIdx.x;  // tiles with the most context first
-    const int q0 = a.query_start[s];
-    const int n = a.query_start[s + 1] - q0;
-    if (qt * kPfRows >= n) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int L = a.context_lens[s];
     const int bs = a.block_size;
-    const int q_first = qt * kPfRows;
-    const int nrows = min(n - q_first, kPfRows);
-    auto write_rows = [&](float value) {
-        for (int i = tid; i < nrows * D; i += kPfThreads)
-            a.out[((int64_t)(q0 + q_first + i / D) * a.num_heads + h) * D + i % D] = Tag::round1(value);
-    };
-    if (L < 0 || L > a.max_blocks_per_seq * bs || n > L) {
-        write_rows(__int_as_float(0x7fc00000));
-        if (tid == 0) report(a.err_word, PA_DEVERR_LEN_RANGE);
-        return;
+
+    // The job of this CTA: nrows query rows (row r at position base_pos + r sees
+    // tokens 0 .. base_pos + r), K/V tiles tile0 .. tile0 + ntiles - 1 of the table
+    // row `tab`, of a sequence of L tokens.
+    int nrows, L, base_pos, tile0, ntiles, kv_head;
+    const int32_t* tab;
+    // prefill: rows q_first .. of sequence s, head h
+    int s = 0, h = 0, q0 = 0, q_first = 0;
+    // shared prefix: rows q_first .. of the group's (member, query head) list, partition p
+    int m0 = 0, p = 0;
+    if constexpr (!kShared) {
+        s = blockIdx.z;
+        h = blockIdx.y;
+        const int qt = gridDim.x - 1 - blockIdx.x;  // tiles with the most context first
+        q0 = a.query_start[s];
+        const int n = a.query_start[s + 1] - q0;
+        if (qt * kPfRows >= n) return;
+        L = a.context_lens[s];
+        q_first = qt * kPfRows;
+        nrows = min(n - q_first, kPfRows);
+        if (L < 0 || L > a.max_blocks_per_seq * bs || n > L) {
+            for (int i = tid; i < nrows * D; i += kPfThreads)
+                a.out[((int64_t)(q0 + q_first + i / D) * a.num_heads + h) * D + i % D] =
+                    Tag::round1(__int_as_float(0x7fc00000));
+            if (tid == 0) report(a.err_word, PA_DEVERR_LEN_RANGE);
+            return;
+        }
+        base_pos = L - n + q_first;
+        tile0 = 0;
+        ntiles = (base_pos + nrows - 1) / kPfTok + 1;
+        kv_head = h / a.group;
+        tab = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
+    } else {
+        const int g = blockIdx.z / a.max_shared_partitions;
+        p = blockIdx.z - g * a.max_shared_partitions;
+        kv_head = blockIdx.y;
+        m0 = a.group_offsets[g];
+        const int rows = (a.group_offsets[g + 1] - m0) * a.group;
+        q_first = blockIdx.x * kPfRows;
+        if (q_first >= rows) return;
+        nrows = min(rows - q_first, kPfRows);
+        const int lead = a.group_members[m0];
+        L = a.seq_start[lead];  // tokens shared by the group
+        const int P = a.partition_tokens;
+        if (L <= 0 || L % P != 0 || L > a.max_blocks_per_seq * bs) {  // the group's start is unusable
+            if (tid == 0 && p == 0 && blockIdx.x == 0 && blockIdx.y == 0) report(a.err_word, PA_DEVERR_LEN_RANGE);
+            return;
+        }
+        if ((p + 1) * P > L) return;  // past this group's prefix
+        base_pos = 1 << 29;  // no causal mask: every row sees the whole prefix
+        tile0 = p * (P / kPfTok);
+        ntiles = P / kPfTok;
+        tab = a.block_tables + (int64_t)lead * a.max_blocks_per_seq;
     }
-    const int base_pos = L - n + q_first;  // position of this CTA's first row
-    const int ntiles = (base_pos + nrows - 1) / kPfTok + 1;
-    const int kv_head = h / a.group;
-    const int32_t* tab = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
-    const int nent = (min(ntiles * kPfTok, L) + bs - 1) / bs;  // table entries the tiles read
+    // (member sequence, query head) of CTA row r in shared-prefix mode
+    auto shared_row = [&](int r, int& seq, int& head) {
+        const int gr = q_first + r;
+        seq = a.group_members[m0 + gr / a.group];
+        head = kv_head * a.group + gr % a.group;
+    };
+    const int e0 = tile0 * kPfTok / bs;
+    const int nent = (min((tile0 + ntiles) * kPfTok, L) + bs - 1) / bs;  // table entries the tiles read
     bool bad = false;
-    for (int i = tid; i < nent; i += kPfThreads) {
+    for (int i = e0 + tid; i < nent; i += kPfThreads) {
         const int id = __ldg(tab + i);
         bad |= id < 0 || id >= a.num_blocks;
     }
     if (__syncthreads_or(bad)) {
-        write_rows(__int_as_float(0x7fc00000));
+        if constexpr (!kShared) {
+            for (int i = tid; i < nrows * D; i += kPfThreads)
+                a.out[((int64_t)(q0 + q_first + i / D) * a.num_heads + h) * D + i % D] =
+                    Tag::round1(__int_as_float(0x7fc00000));
+        } else {
+            for (int r = tid; r < nrows; r += kPfThreads) {
+                int seq, head;
+                shared_row(r, seq, head);
+                const int64_t pi = ((int64_t)seq * a.num_heads + head) * a.num_partitions + p;
+                a.ws_m[pi] = __int_as_float(0x7fc00000);
+                a.ws_l[pi] = __int_as_float(0x7fc00000);
+            }
+        }
         if (tid == 0) report(a.err_word, PA_DEVERR_TABLE_RANGE);
         return;
     }
@@ -210,7 +272,15 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
     if (tid < kPfRows) {
         const bool live = tid < nrows;
         const uint32_t flip = a.scale_log2 < 0.f ? 0x80008000u : 0u;
-        const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)(q0 + q_first + (live ? tid : 0)) * a.num_heads + h) * D);
+        int64_t qrow;  // row of q in [rows][num_heads * D] units of D
+        if constexpr (!kShared) {
+            qrow = (int64_t)(q0 + q_first + (live ? tid : 0)) * a.num_heads + h;
+        } else {
+            int seq, head;
+            shared_row(live ? tid : 0, seq, head);
+            qrow = (int64_t)seq * a.num_heads + head;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + qrow * D);
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) {
             uint4 v = live ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
@@ -258,14 +328,14 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
                     tma_load_3d(dst0 + hh * Lay::kTHalf + lane * br * 128, map, hh * 64, kv_head, row, bar);
             }
         };
-        int row = row_of(0);
+        int row = row_of(tile0);
         for (int j = 0; j < ntiles; ++j) {
             const int st = j & 1;
             if (j >= 2) ok = __all_sync(FULL, pf_wait(&bars[kBarKEmpty + st], ((j >> 1) + 1) & 1) && !*abort_flag);
             if (!ok) break;
             load(&kmap, smem + Lay::kOffK + st * Lay::kTile, &bars[kBarKFull + st], row);
             issued_k = j + 1;
-            const int next = j + 1 < ntiles ? row_of(j + 1) : -1;  // in flight during the wait below
+            const int next = j + 1 < ntiles ? row_of(tile0 + j + 1) : -1;  // in flight during the wait below
             if (j >= 2) ok = __all_sync(FULL, pf_wait(&bars[kBarVEmpty + st], ((j >> 1) + 1) & 1) && !*abort_flag);
             if (!ok) break;
             load(&vmap, smem + Lay::kOffV + st * Lay::kTile, &bars[kBarVFull + st], row);
@@ -320,7 +390,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             const int st = j & 1;
             ok = wait(kBarVFull + st, (j >> 1) & 1);
             if (!ok) break;
-            const int t0 = j * kPfTok;
+            const int t0 = (tile0 + j) * kPfTok;
             if (t0 + kPfTok > L) {  // zero the V rows past the sequence end
                 uint8_t* vt = smem + Lay::kOffV + st * Lay::kTile;
                 const int r0 = L - t0;
@@ -382,7 +452,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             umma::ld32(tS + b * 64 + lrow, sv[0]);
             umma::ld32(tS + b * 64 + 32 + lrow, sv[1]);
             umma::wait_ld();
-            const int t0 = j * kPfTok;
+            const int t0 = (tile0 + j) * kPfTok;
             // every row of the CTA sees the whole tile unless it reaches the diagonal
             const bool diag = t0 + kPfTok - 1 > base_pos;
             const int vis = diag ? pos - t0 : kPfTok - 1;  // last visible token of the tile, this row
@@ -422,7 +492,41 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             mbar_arrive(&bars[kBarPFull + b]);
         }
         if (ok) ok = __all_sync(FULL, pf_wait(&bars[kBarOLast], 0) && !*abort_flag);
-        if (ok) {
+        if (ok && kShared) {
+            // partial of this partition for the row's (sequence, head): running max
+            // (base-2 units, scores scaled by scale * log2 e), sum, unnormalised o
+            umma::fence_after_sync();
+            bool write = r < nrows;
+            int64_t pi = 0;
+            if (write) {
+                int seq, head;
+                shared_row(r, seq, head);
+                const int Ls = a.context_lens[seq];
+                // a member must share the group's prefix length and extend past it
+                if (a.seq_start[seq] != L || Ls <= L || Ls > a.max_blocks_per_seq * bs) {
+                    report(a.err_word, PA_DEVERR_LEN_RANGE);
+                    write = false;
+                }
+                pi = ((int64_t)seq * a.num_heads + head) * a.num_partitions + p;
+            }
+            float4* dst = reinterpret_cast<float4*>(a.ws_o + pi * D);
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                umma::ld32(tO + lrow + cc * 32, o);
+                umma::wait_ld();
+                if (write) {
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        dst[cc * 8 + v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                                      __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+                }
+            }
+            if (write) {
+                a.ws_m[pi] = m_used;
+                a.ws_l[pi] = l;
+            }
+        } else if (ok) {
             umma::fence_after_sync();
             const float inv = 1.f / l;
             uint4* dst = reinterpret_cast<uint4*>(a.out + ((int64_t)(q0 + q_first + min(r, nrows - 1)) * a.num_heads + h) * D);
@@ -461,7 +565,7 @@ int launch_prefill(PrefillArgs args, const void* k_cache, const void* v_cache, i
                    int max_query_len, cudaStream_t stream) {
     using Lay = PfLayout<D>;
     static std::atomic<uint64_t> smem_done{0};
-    auto kernel = paged_prefill_kernel<Tag, D>;
+    auto kernel = paged_prefill_kernel<Tag, D, false>;
     if (ensure_smem_limit(kernel, Lay::kAlloc, smem_done) != cudaSuccess) return PA_ERR_CUDA;
     args.box_rows = kPfTok < args.block_size ? kPfTok : args.block_size;
     const int64_t total_tokens = (int64_t)args.num_blocks * args.block_size;
@@ -474,7 +578,64 @@ int launch_prefill(PrefillArgs args, const void* k_cache, const void* v_cache, i
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+template <class Tag, int D>
+int launch_shared(PrefillArgs args, const void* k_cache, const void* v_cache, int num_kv_heads, int num_groups,
+                  int max_group_size, cudaStream_t stream) {
+    using Lay = PfLayout<D>;
+    static std::atomic<uint64_t> smem_done{0};
+    auto kernel = paged_prefill_kernel<Tag, D, true>;
+    if (ensure_smem_limit(kernel, Lay::kAlloc, smem_done) != cudaSuccess) return PA_ERR_CUDA;
+    args.box_rows = kPfTok < args.block_size ? kPfTok : args.block_size;
+    const int64_t total_tokens = (int64_t)args.num_blocks * args.block_size;
+    CUtensorMap kmap, vmap;
+    if (!encode_cache_map_swizzled(&kmap, k_cache, D, num_kv_heads, total_tokens, args.box_rows) ||
+        !encode_cache_map_swizzled(&vmap, v_cache, D, num_kv_heads, total_tokens, args.box_rows))
+        return PA_ERR_CUDA;
+    const int64_t rows = (int64_t)max_group_size * args.group;
+    dim3 grid((unsigned)((rows + kPfRows - 1) / kPfRows), (unsigned)num_kv_heads,
+              (unsigned)(num_groups * args.max_shared_partitions));
+    kernel<<<grid, kPfThreads, Lay::kAlloc, stream>>>(args, kmap, vmap);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 }  // namespace
+
+int launch_shared_prefix(const SharedPrefixLaunch& l, cudaStream_t stream) {
+    if (l.partition_tokens % kPfTok != 0 || l.max_shared_tokens % l.partition_tokens != 0) return PA_ERR_INVALID_ARG;
+    const int64_t maxpp = l.max_shared_tokens / l.partition_tokens;
+    if (maxpp == 0 || l.num_groups == 0) return PA_OK;
+    if (maxpp * l.num_groups > 65535 || l.num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    PrefillArgs args{};
+    args.q = static_cast<const uint16_t*>(l.q);
+    args.block_tables = l.block_tables;
+    args.context_lens = l.context_lens;
+    args.err_word = l.err_word;
+    args.scale_log2 = l.scale * 1.4426950408889634f;
+    args.num_heads = l.num_heads;
+    args.group = l.num_heads / l.num_kv_heads;
+    args.block_size = l.block_size;
+    args.num_blocks = l.num_blocks;
+    args.max_blocks_per_seq = l.max_blocks_per_seq;
+    args.group_offsets = l.group_offsets;
+    args.group_members = l.group_members;
+    args.seq_start = l.seq_start;
+    args.ws_m = l.ws_m;
+    args.ws_l = l.ws_l;
+    args.ws_o = l.ws_o;
+    args.partition_tokens = l.partition_tokens;
+    args.num_partitions = l.num_partitions;
+    args.max_shared_partitions = (int)maxpp;
+    if (l.head_dim == 128)
+        return l.dtype == PA_F16 ? launch_shared<F16Tag, 128>(args, l.k_cache, l.v_cache, l.num_kv_heads, l.num_groups,
+                                                              l.max_group_size, stream)
+                                 : launch_shared<BF16Tag, 128>(args, l.k_cache, l.v_cache, l.num_kv_heads,
+                                                               l.num_groups, l.max_group_size, stream);
+    return l.dtype == PA_F16 ? launch_shared<F16Tag, 64>(args, l.k_cache, l.v_cache, l.num_kv_heads, l.num_groups,
+                                                         l.max_group_size, stream)
+                             : launch_shared<BF16Tag, 64>(args, l.k_cache, l.v_cache, l.num_kv_heads, l.num_groups,
+                                                          l.max_group_size, stream);
+}
+
 }  // namespace pa
 
 extern "C" int pa_prefill(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,

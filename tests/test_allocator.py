@@ -279,3 +279,73 @@ def test_prefill_slots_match_model_and_oracle(pa, oracle):
                 k += 1
             assert list(tables[i, :len(mgr.tables[i])]) == mgr.tables[i]
         assert np.array_equal(lens, before + new) and a.num_free() == mgr.pool.num_free()
+
+
+# ------------------------------------------------------------- shared prefixes
+
+def _check_groups(tables, lens, bs, P, g):
+    """Invariants of pa_find_shared_prefixes' result."""
+    S = len(lens)
+    seen = set()
+    for k in range(g.num_groups):
+        mem = list(g.group_members[g.group_offsets[k]:g.group_offsets[k + 1]])
+        assert len(mem) >= 2 and not (set(mem) & seen)
+        seen |= set(mem)
+        st = {int(g.seq_start[m]) for m in mem}
+        assert len(st) == 1
+        st = st.pop()
+        assert st > 0 and st % P == 0 and all(st < lens[m] for m in mem)
+        for m in mem:  # same physical blocks below the start
+            assert np.array_equal(tables[m, :st // bs], tables[mem[0], :st // bs])
+    for s in range(S):
+        if s not in seen:
+            assert g.seq_start[s] == 0
+    assert g.max_shared_tokens == max([int(x) for x in g.seq_start] + [0])
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_find_shared_prefixes_on_random_forks(pa, seed):
+    rng = np.random.default_rng(seed)
+    bs = int(rng.choice([16, 32, 64]))
+    P = bs * int(rng.choice([1, 2, 4]))
+    S, MB = 40, 40
+    tables = np.full((S, MB), -1, np.int32)
+    lens = np.zeros(S, np.int32)
+    nxt = 0
+    for s in range(S):
+        L = int(rng.integers(1, MB * bs + 1))
+        nb = -(-L // bs)
+        if s > 0 and rng.random() < 0.7:  # fork from an earlier sequence: share a random number of its blocks
+            src = int(rng.integers(0, s))
+            k = int(rng.integers(0, -(-int(lens[src]) // bs) + 1))
+            k = min(k, nb)
+            tables[s, :k] = tables[src, :k]
+        else:
+            k = 0
+        tables[s, k:nb] = np.arange(nxt, nxt + nb - k)
+        nxt += nb - k
+        lens[s] = L
+    g = pa.pa_find_shared_prefixes(tables, lens, bs, P)
+    _check_groups(tables, lens, bs, P, g)
+
+
+def test_find_shared_prefixes_beam_fork(pa):
+    """Every beam holds the prompt's blocks: one group sharing the whole prompt."""
+    bs, P = 64, 256
+    prompt = np.arange(8, dtype=np.int32)       # 512 tokens
+    tables = np.full((12, 16), -1, np.int32)
+    lens = np.zeros(12, np.int32)
+    for s in range(12):
+        tables[s, :8] = prompt
+        tables[s, 8:10] = [100 + 2 * s, 101 + 2 * s]
+        lens[s] = 512 + 1 + 7 * s
+    g = pa.pa_find_shared_prefixes(tables, lens, bs, P)
+    assert g.num_groups == 1 and list(g.group_members) == list(range(12))
+    assert list(g.seq_start) == [512] * 12 and g.max_group_size == 12 and g.max_shared_tokens == 512
+    _check_groups(tables, lens, bs, P, g)
+    lens[3] = 512  # its last token sits in the prompt: it can share only 256 tokens, the others keep 512
+    g = pa.pa_find_shared_prefixes(tables, lens, bs, P)
+    assert g.seq_start[3] == 0 and g.num_groups == 1
+    _check_groups(tables, lens, bs, P, g)
+    with pytest.raises(pa.PAError):
+        pa.pa_find_shared_prefixes(tables, lens, bs, 100)  # not a multiple of the block size

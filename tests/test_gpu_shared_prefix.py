@@ -1,0 +1,125 @@
+"""Two-level decode of sequences that share a prefix through the same blocks
+(pa_decode_shared_prefix), on the GPU against the oracle: the shared part is
+attended once per group, the suffix per sequence, and the result must be the
+oracle's decode of every sequence over all of its tokens."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_cases import Step, assert_close, bits
+from pins import BF16, F16, PagedCase
+import oracle as oracle_pkg
+from paged_kv_cache_374_b200 import binding as pa
+
+pytestmark = pytest.mark.gpu
+
+TDT = {F16: torch.float16, BF16: torch.bfloat16}
+WK = {F16: "f16", BF16: "bf16"}
+
+
+def dev(a, dtype):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(TDT[dtype]).cuda()
+
+
+def share(c: PagedCase, members, tokens):
+    """Members of a group use the lead's blocks (and data) for their first ``tokens``."""
+    lead, nb = members[0], tokens // c.bs
+    for s in members[1:]:
+        c.tables[s, :nb] = c.tables[lead, :nb]
+        c.seq_k[s][:tokens] = c.seq_k[lead][:tokens]
+        c.seq_v[s][:tokens] = c.seq_v[lead][:tokens]
+    c._assemble()
+
+
+def run_both(c, P, err=None, groups=None):
+    q = dev(c.q, c.dtype)
+    kc, vc = dev(c.k_cache, c.dtype), dev(c.v_cache, c.dtype)
+    tb, ln = torch.from_numpy(c.tables).cuda(), torch.from_numpy(c.lens).cuda()
+    g = groups or pa.pa_find_shared_prefixes(c.tables, c.lens, c.bs, P)
+    start, offs, mem = g.to("cuda")
+    out = torch.empty_like(q)
+    pa.pa_decode_shared_prefix(q, kc, vc, tb, ln, c.scale, c.Hk, out, start, offs, mem, g.num_groups,
+                               g.max_group_size, g.max_shared_tokens, partition_tokens=P, err_word=err)
+    ref = torch.empty_like(q)
+    pa.pa_decode(q, kc, vc, tb, ln, c.scale, c.Hk, ref, partition_tokens=P)
+    torch.cuda.synchronize()
+    return out, ref, g
+
+
+CASES = [(128, 16, 1, F16), (128, 32, 4, BF16), (64, 64, 1, BF16), (64, 16, 8, F16), (128, 64, 2, F16)]
+
+
+@pytest.mark.parametrize("d,bs,g,dtype", CASES)
+def test_shared_prefix_matches_oracle(d, bs, g, dtype):
+    rng = np.random.default_rng(70 + d + bs + g)
+    P = 64
+    lens = [300, 200, 193, 257, 140, 129, 130, 400, 90, 1]
+    hk = 2
+    c = PagedCase(rng, lens, hk * g, hk, d, bs, dtype, 1 / math.sqrt(d), extra_blocks=4)
+    share(c, [0, 1, 2, 3], 192)        # three partitions
+    share(c, [0, 4], 64)               # 4 shares only the first with 0
+    share(c, [5, 6, 7], 128)           # two partitions
+    out, ref_gpu, grp = run_both(c, P)
+    assert grp.num_groups == 2
+    assert list(grp.seq_start) == [192, 192, 192, 192, 0, 128, 128, 128, 0, 0]
+    ref = oracle_pkg.get().decode(c.q, c.k_cache, c.v_cache, c.tables, c.lens, c.scale, dtype, nthreads=8)
+    assert_close(out, ref, WK[dtype], f"shared d{d} bs{bs} g{g}")
+    assert_close(ref_gpu, ref, WK[dtype], "pa_decode")
+
+
+def test_no_groups_is_pa_decode():
+    rng = np.random.default_rng(71)
+    c = PagedCase(rng, [100, 300, 64], 4, 4, 128, 16, F16, 0.1)
+    out, ref, grp = run_both(c, 64)
+    assert grp.num_groups == 0
+    assert torch.equal(out, ref)
+
+
+def test_bad_start_is_reported_and_ignored():
+    """A member whose start is not a multiple of the partition runs whole in the
+    per-sequence kernel (and gets no shared partials): still the oracle's result."""
+    rng = np.random.default_rng(72)
+    c = PagedCase(rng, [300, 280, 290], 8, 8, 128, 16, BF16, 1 / math.sqrt(128))
+    share(c, [0, 1, 2], 256)
+    grp = pa.pa_find_shared_prefixes(c.tables, c.lens, c.bs, 64)
+    assert list(grp.seq_start) == [256, 256, 256]
+    grp.seq_start = grp.seq_start.copy()
+    grp.seq_start[2] = 200
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, _, _ = run_both(c, 64, err=err, groups=grp)
+    assert err.item() & pa.PA_DEVERR_LEN_RANGE
+    ref = oracle_pkg.get().decode(c.q, c.k_cache, c.v_cache, c.tables, c.lens, c.scale, BF16)
+    assert_close(out, ref, "bf16", "bad start")
+
+
+def test_beam_full_size():
+    """The beam workload (128 sequences forked from one 512-token prompt, block
+    size 64): one group sharing the prompt; compared with the oracle on sampled
+    (sequence, head) pairs and with pa_decode everywhere."""
+    step = Step("beam")
+    t = step.tensors()
+    P = pa.pa_decode_partition_tokens(step.spec.num_seqs, 32, 32, 128, step.bs, step.tables.shape[1])
+    grp = pa.pa_find_shared_prefixes(step.tables, step.lens, step.bs, P)
+    assert grp.num_groups >= 1 and grp.max_shared_tokens == step.spec.prefix_tokens // P * P
+    start, offs, mem = grp.to("cuda")
+    tb, ln = torch.from_numpy(step.tables).cuda(), torch.from_numpy(step.lens).cuda()
+    pa.pa_reshape_and_cache(t["k"], t["v"], torch.from_numpy(step.slots).cuda(), t["k_cache"], t["v_cache"])
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty_like(t["q"])
+    pa.pa_decode_shared_prefix(t["q"], t["k_cache"], t["v_cache"], tb, ln, step.spec.scale, 32, out, start, offs,
+                               mem, grp.num_groups, grp.max_group_size, grp.max_shared_tokens, err_word=err)
+    ref_gpu = torch.empty_like(out)
+    pa.pa_decode(t["q"], t["k_cache"], t["v_cache"], tb, ln, step.spec.scale, 32, ref_gpu)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert (out.float() - ref_gpu.float()).abs().max().item() <= 2e-3
+    o = oracle_pkg.get()
+    kh, vh = bits(t["k_cache"]), bits(t["v_cache"])
+    rng = np.random.default_rng(73)
+    pairs = np.array([(int(rng.integers(0, step.spec.num_seqs)), int(rng.integers(0, 32))) for _ in range(64)],
+                     dtype=np.int32)
+    ref = o.decode(bits(t["q"]), kh, vh, step.tables, step.lens, step.spec.scale, F16, pairs=pairs, nthreads=8)
+    got = out[torch.from_numpy(pairs[:, 0]).long(), torch.from_numpy(pairs[:, 1]).long()]
+    assert_close(got, ref, "f16", "beam shared")
