@@ -426,6 +426,11 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
             __threadfence();
         }
     }
+    // Launched behind the shared-prefix kernel (programmatic dependent launch),
+    // this launch may run beside it but must not complete before it: the merge
+    // kernel, which waits for this one, reads its partials too.  (A no-op for a
+    // plain launch.)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace pa

@@ -193,8 +193,23 @@ int launch_engine(DecodeArgs args, const void* k_cache, const void* v_cache, int
             c.ws_l += shoff * args.num_partitions;
             c.ws_o += shoff * args.num_partitions * D;
         }
-        kernel<<<sms, NW * 32, Lay::kAlloc, stream>>>(c, kmap, vmap);
-        if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+        if (c.seq_start && s0 == 0) {
+            // behind the shared-prefix kernel: start on the SMs it leaves free
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)sms);
+            cfg.blockDim = dim3(NW * 32);
+            cfg.dynamicSmemBytes = Lay::kAlloc;
+            cfg.stream = stream;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[0].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaLaunchKernelEx(&cfg, kernel, c, kmap, vmap) != cudaSuccess) return PA_ERR_CUDA;
+        } else {
+            kernel<<<sms, NW * 32, Lay::kAlloc, stream>>>(c, kmap, vmap);
+            if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+        }
         if (args.num_partitions > 1) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3((unsigned)((int64_t)c.num_seqs * args.num_heads));

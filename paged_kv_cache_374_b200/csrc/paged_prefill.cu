@@ -215,6 +215,8 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
         kv_head = h / a.group;
         tab = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
     } else {
+        // the decode engine that follows may start on the SMs this grid leaves free
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
         const int g = blockIdx.z / a.max_shared_partitions;
         p = blockIdx.z - g * a.max_shared_partitions;
         kv_head = blockIdx.y;
