@@ -39,6 +39,9 @@ FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "paged_decode_llama7b.md")
 DECODE_SOURCES = [os.path.join(ROOT, "paged_kv_cache_374_b200", "csrc", f) for f in
                   ("paged_decode.cu", "decode_engine.cuh", "decode_mha.cuh", "decode_gqa.cuh", "pa_device.cuh")]
+SHARED_PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "shared_prefix_beam.md")
+SHARED_SOURCES = DECODE_SOURCES + [os.path.join(ROOT, "paged_kv_cache_374_b200", "csrc", f) for f in
+                                   ("paged_prefill.cu", "tcgen05.cuh")]
 
 
 def parse():
@@ -107,18 +110,18 @@ def source_digest(paths):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(units_now: int):
-    """DRAM bytes per launch of K2 from the committed ncu summary, scaled to this
-    launch's tokens; None when the summary is missing or the kernel source has
-    changed since the counters were taken."""
+def profiled_traffic(units_now: int, summary=PROFILE_SUMMARY, sources=DECODE_SOURCES):
+    """DRAM bytes per launch of the decode kernels from a committed ncu summary,
+    scaled to this launch's (unique) tokens; None when the summary is missing or
+    a kernel source has changed since the counters were taken."""
     try:
         fields = {}
-        with open(PROFILE_SUMMARY) as f:
+        with open(summary) as f:
             for line in f:
                 if line.startswith("- ") and ": " in line:
                     k, v = line[2:].split(": ", 1)
                     fields[k.strip()] = v.strip().strip("`")
-        if fields.get("source_sha256_16") != source_digest(DECODE_SOURCES):
+        if fields.get("source_sha256_16") != source_digest(sources):
             return None
         per_token = float(fields["dram_bytes_per_launch"]) / float(fields["tokens_per_launch"])
         return per_token * units_now
@@ -454,7 +457,9 @@ def run_native(args):
                        "paged_decode_kernel + paged_decode_merge_kernel (timed together: one pa_decode call)"),
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
             "unit": "GB/s", "frac": round(achieved / peak, 4),
-            "traffic": None if (fp8 or st["groups"] is not None) else profiled_traffic(ab["unique_tokens"]),
+            "traffic": (None if fp8 else
+                        profiled_traffic(ab["unique_tokens"], SHARED_PROFILE_SUMMARY, SHARED_SOURCES)
+                        if st["groups"] is not None else profiled_traffic(ab["unique_tokens"])),
         },
         "e2e": {"value": round(job_throughput(world, tokens_per_step, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
