@@ -123,3 +123,20 @@ def test_beam_full_size():
     ref = o.decode(bits(t["q"]), kh, vh, step.tables, step.lens, step.spec.scale, F16, pairs=pairs, nthreads=8)
     got = out[torch.from_numpy(pairs[:, 0]).long(), torch.from_numpy(pairs[:, 1]).long()]
     assert_close(got, ref, "f16", "beam shared")
+
+
+def test_more_sequences_than_one_launch():
+    """1100 sequences in four groups: the engine runs in two launches (at most
+    1024 sequences each); every sequence's start and partials must line up."""
+    rng = np.random.default_rng(74)
+    S, P, bs = 1100, 64, 16
+    lens = rng.integers(65, 400, size=S).astype(np.int32)
+    c = PagedCase(rng, lens, 2, 2, 64, bs, F16, 0.125, extra_blocks=2)
+    groups = [list(range(0, 300)), list(range(300, 700)), list(range(700, 1050, 2)), [1098, 1099]]
+    for g in groups:
+        share(c, g, 64 * int(min(-(-int(min(lens[g])) // 64) - 1, 3)))
+    out, ref_gpu, grp = run_both(c, P)
+    assert grp.num_groups >= 4
+    assert torch.equal(torch.isnan(out), torch.isnan(ref_gpu))
+    ref = oracle_pkg.get().decode(c.q, c.k_cache, c.v_cache, c.tables, c.lens, c.scale, F16, nthreads=8)
+    assert_close(out, ref, "f16", "1100 sequences shared")
