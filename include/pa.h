@@ -200,7 +200,9 @@ int pa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, c
  *   group_offsets  [num_groups + 1] int32: group g is
  *   group_members  group_members[group_offsets[g] .. group_offsets[g+1]) (sequence
  *                  indices); every member has the same seq_start
- *   max_group_size, max_shared_tokens  host ints bounding the arrays (launch sizes)
+ *   max_group_size, max_shared_tokens  host ints bounding the group sizes and the
+ *                  seq_start values (the launch sizes); a group beyond them is
+ *                  reported as PA_DEVERR_LEN_RANGE and its output is undefined
  * pa_find_shared_prefixes builds these from host block tables.  partition_tokens
  * must be the one the workspace was sized with (0 = default).  A seq_start that
  * is not a multiple of the partition below the length is ignored (the whole

@@ -232,6 +232,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             if (tid == 0 && p == 0 && blockIdx.x == 0 && blockIdx.y == 0) report(a.err_word, PA_DEVERR_LEN_RANGE);
             return;
         }
+        // the launch bounds (max_group_size, max_shared_tokens) must cover every group
+        if (tid == 0 && ((p == a.max_shared_partitions - 1 && L > a.max_shared_partitions * P) ||
+                         (blockIdx.x == gridDim.x - 1 && rows > (int)gridDim.x * kPfRows)))
+            report(a.err_word, PA_DEVERR_LEN_RANGE);
         if ((p + 1) * P > L) return;  // past this group's prefix
         base_pos = 1 << 29;  // no causal mask: every row sees the whole prefix
         tile0 = p * (P / kPfTok);

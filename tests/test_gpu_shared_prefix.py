@@ -140,3 +140,21 @@ def test_more_sequences_than_one_launch():
     assert torch.equal(torch.isnan(out), torch.isnan(ref_gpu))
     ref = oracle_pkg.get().decode(c.q, c.k_cache, c.v_cache, c.tables, c.lens, c.scale, F16, nthreads=8)
     assert_close(out, ref, "f16", "1100 sequences shared")
+
+
+def test_launch_bounds_too_small_are_reported():
+    rng = np.random.default_rng(75)
+    c = PagedCase(rng, [300] * 6, 4, 4, 128, 16, F16, 0.1)
+    share(c, list(range(6)), 256)
+    g = pa.pa_find_shared_prefixes(c.tables, c.lens, c.bs, 64)
+    assert g.max_shared_tokens == 256 and g.max_group_size == 6
+    for mg, mt in ((6, 128), (6, 256)):
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        q = dev(c.q, F16)
+        out = torch.empty_like(q)
+        start, offs, mem = g.to("cuda")
+        pa.pa_decode_shared_prefix(q, dev(c.k_cache, F16), dev(c.v_cache, F16), torch.from_numpy(c.tables).cuda(),
+                                   torch.from_numpy(c.lens).cuda(), c.scale, 4, out, start, offs, mem,
+                                   g.num_groups, mg, mt, partition_tokens=64, err_word=err)
+        torch.cuda.synchronize()
+        assert bool(err.item() & pa.PA_DEVERR_LEN_RANGE) == (mt < 256)
