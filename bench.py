@@ -38,7 +38,8 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "paged_decode_llama7b.md")
 DECODE_SOURCES = [os.path.join(ROOT, "paged_kv_cache_374_b200", "csrc", f) for f in
-                  ("paged_decode.cu", "decode_engine.cuh", "decode_mha.cuh", "decode_gqa.cuh", "pa_device.cuh")]
+                  ("paged_decode.cu", "decode_engine.cuh", "decode_mha.cuh", "decode_gqa.cuh", "decode_fp8tc.cuh",
+                   "pa_device.cuh")]
 SHARED_PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "shared_prefix_beam.md")
 SHARED_SOURCES = DECODE_SOURCES + [os.path.join(ROOT, "paged_kv_cache_374_b200", "csrc", f) for f in
                                    ("paged_prefill.cu", "tcgen05.cuh")]

@@ -74,14 +74,16 @@ struct Unit {
     int t_begin, t_end, nst, kv_head, blk0, nblk;
 };
 
-// ROWB: bytes of one token's row of one kv head (head_dim * element size)
-template <int ROWB, int TOK, int NW, int R>
+// ROWB: bytes of one token's row of one kv head (head_dim * element size);
+// SCR: shared scratch bytes a compute policy keeps per warp (a multiple of 1 KiB)
+template <int ROWB, int TOK, int NW, int R, int SCR = 0>
 struct Layout {
     static constexpr int kTileBytes = TOK * ROWB;
-    static constexpr int kHalfBytes = TOK * 128;               // one 64-dim half tile
+    static constexpr int kHalfBytes = TOK * 128;               // one 128-byte-wide box column of a tile
     static constexpr int kSlotBytes = 2 * kTileBytes;          // K tile then V tile
     static constexpr int kOffSlots = 0;
-    static constexpr int kOffBars = NW * R * kSlotBytes;
+    static constexpr int kOffScratch = NW * R * kSlotBytes;
+    static constexpr int kOffBars = kOffScratch + NW * SCR;
     static constexpr int kOffCum = kOffBars + NW * R * 8;         // int[S + 1]
     static constexpr int kOffKey = kOffCum + (kMaxSeqsPerLaunch + 1) * 4 + 12;  // uint32[S_pow2]
     static constexpr int kOffLen = kOffKey + kMaxSeqsPerLaunch * 4;            // int[S]
@@ -186,7 +188,7 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
                                                                   const __grid_constant__ CUtensorMap vmap) {
     constexpr int ROWB = D * CTag::kBytes;      // bytes per token row of one kv head
     static_assert(ROWB % 128 == 0, "rows are loaded as 128-byte swizzled boxes");
-    using Lay = Layout<ROWB, TOK, NW, R>;
+    using Lay = Layout<ROWB, TOK, NW, R, Policy::kScratchBytes>;
     constexpr int MAXSUB = TOK / 8 > 2 ? 2 : 1;  // TMA boxes per half tile (box_rows >= TOK/2)
 
     extern __shared__ uint8_t smem_raw[];
@@ -267,7 +269,7 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
 
     // ------------------------------------------------------------ warp engine
     Policy pol;
-    pol.setup(lane);
+    pol.setup(lane, smem + Lay::kOffScratch + warp * Policy::kScratchBytes);
     int32_t* claim_ctr = a.sched;
     auto claim = [&]() -> int { return lane == 0 ? atomicAdd(claim_ctr, 1) : 0; };
     auto load_tab = [&](const Unit& U, int chunk) -> int {

@@ -93,7 +93,9 @@ struct GqaPolicy {
     float o[NT][MT][4];             // O^T fragments: dims mt*16 + g (+8), heads 2t, 2t+1
     bool poisoned;
 
-    __device__ __forceinline__ void setup(int lane_) {
+    static constexpr int kScratchBytes = 0;
+
+    __device__ __forceinline__ void setup(int lane_, uint8_t* /*scratch*/) {
         lane = lane_;
         g = lane >> 2;
         t = lane & 3;
@@ -170,11 +172,12 @@ struct GqaPolicy {
                 for (int nt = 0; nt < NT; ++nt) Ops::mma(x[nt], af, qb[nt][ks][0], qb[nt][ks][1]);
             }
             const bool v0 = g < nv, v1 = g + 8 < nv;
+            const float sc = a.scale_log2 * a.k_scale;  // k_scale: 1, or the fp8 cache's K scale
             bool up = false;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) x[nt][j] *= a.scale_log2;
+                for (int j = 0; j < 4; ++j) x[nt][j] *= sc;
                 if (!v0) x[nt][0] = x[nt][1] = -INFINITY;
                 if (!v1) x[nt][2] = x[nt][3] = -INFINITY;
                 up |= x[nt][0] > m[nt][0] || x[nt][2] > m[nt][0] || x[nt][1] > m[nt][1] || x[nt][3] > m[nt][1];
@@ -254,6 +257,13 @@ struct GqaPolicy {
                 l += __shfl_xor_sync(kFullMask, l, 8);
                 l += __shfl_xor_sync(kFullMask, l, 16);
                 if (bad) l = __int_as_float(0x7fc00000);
+                if (a.v_scale != 1.f) {  // fp8 cache: V = code * v_scale
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        o[nt][mt][j] *= a.v_scale;
+                        o[nt][mt][j + 2] *= a.v_scale;
+                    }
+                }
                 const int head = nt * 8 + 2 * t + j;
                 if (head >= a.heads_per_unit) continue;
                 const int64_t sh = (int64_t)U.s * a.num_heads + U.h * a.heads_per_unit + head;

@@ -41,7 +41,9 @@ struct MhaPolicy {
     float2 o[DL / 2];
     bool poisoned;
 
-    __device__ __forceinline__ void setup(int lane_) {
+    static constexpr int kScratchBytes = 0;
+
+    __device__ __forceinline__ void setup(int lane_, uint8_t* /*scratch*/) {
         lane = lane_;
         r = lane & 7;
         c = lane >> 3;

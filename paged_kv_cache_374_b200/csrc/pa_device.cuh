@@ -61,6 +61,13 @@ struct E4M3Tag {
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(in));
         return __half22float2(*reinterpret_cast<const __half2*>(&h));
     }
+    // two packed codes (low byte first) as an exact f16x2 pair (low half first)
+    static __device__ __forceinline__ uint32_t to_f16x2(uint32_t pair16) {
+        uint32_t h;
+        const unsigned short in = (unsigned short)pair16;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(in));
+        return h;
+    }
     // nearest codes of two floats (round to nearest even, saturating at +-448), lo in the low byte
     static __device__ __forceinline__ uint32_t encode2(float lo, float hi) {
         unsigned short d;

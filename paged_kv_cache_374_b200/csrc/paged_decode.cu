@@ -11,6 +11,7 @@
 // one query head, tensor cores per kv head (decode_gqa.cuh) when a group of query
 // heads shares each kv head.  K3 (below) merges the partials of split sequences.
 #include "decode_engine.cuh"
+#include "decode_fp8tc.cuh"
 #include "decode_gqa.cuh"
 #include "decode_mha.cuh"
 #include "pa_host.h"
@@ -165,7 +166,7 @@ int sm_count() {
 template <class Tag, class CTag, int D, int TOK, int NW, int R, class Policy>
 int launch_engine(DecodeArgs args, const void* k_cache, const void* v_cache, int num_kv_heads,
                   cudaStream_t stream) {
-    using Lay = Layout<D * CTag::kBytes, TOK, NW, R>;
+    using Lay = Layout<D * CTag::kBytes, TOK, NW, R, Policy::kScratchBytes>;
     static_assert(Lay::kAlloc <= 227 * 1024, "shared memory");
     static std::atomic<uint64_t> smem_done{0};
     auto kernel = paged_decode_kernel<Tag, CTag, D, TOK, NW, R, Policy>;
@@ -250,15 +251,29 @@ int launch_decode(DecodeArgs args, const void* k_cache, const void* v_cache, int
                                                                                             num_kv_heads, stream);
 }
 
-// fp8 (E4M3) caches: CUDA cores, one query head per unit, 32-token slots (8 KiB)
+// fp8 (E4M3) caches.  GQA groups of 2-16: tensor cores, one kv head with its whole
+// query group per unit (one fetch of the codes serves the group), 16-token slots
+// widened into per-warp 16-bit tiles.  MHA (and larger groups): CUDA cores, one
+// query head per unit, 32-token slots (8 KiB): with a single head the tensor-core
+// stage carries too little work per byte to keep up.
 template <class Tag>
 int launch_decode_fp8(DecodeArgs args, const void* k_cache, const void* v_cache, int num_kv_heads,
                       cudaStream_t stream) {
-    constexpr int TOK = 32;
+    constexpr int TOK = 16;
+    if (args.group >= 2 && args.group <= PA_GQA_MAX_GROUP) {
+        args.unit_heads = num_kv_heads;
+        args.heads_per_unit = args.group;
+        if (args.group <= 8)
+            return launch_engine<Tag, E4M3Tag, 128, TOK, 12, 2, Fp8TcPolicy<Tag, TOK, 1>>(args, k_cache, v_cache,
+                                                                                            num_kv_heads, stream);
+        return launch_engine<Tag, E4M3Tag, 128, TOK, 8, 2, Fp8TcPolicy<Tag, TOK, 2>>(args, k_cache, v_cache,
+                                                                                       num_kv_heads, stream);
+    }
+    constexpr int TOK32 = 32;
     args.unit_heads = args.num_heads;
     args.heads_per_unit = 1;
-    return launch_engine<Tag, E4M3Tag, 128, TOK, PA_DECODE_WARPS, PA_DECODE_SLOTS, MhaPolicy<Tag, E4M3Tag, 128, TOK>>(
-        args, k_cache, v_cache, num_kv_heads, stream);
+    return launch_engine<Tag, E4M3Tag, 128, TOK32, PA_DECODE_WARPS, PA_DECODE_SLOTS,
+                         MhaPolicy<Tag, E4M3Tag, 128, TOK32>>(args, k_cache, v_cache, num_kv_heads, stream);
 }
 
 }  // namespace
