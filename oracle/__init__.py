@@ -5,7 +5,11 @@ import this package.  It shares no code with the CUDA library and never imports
 it.  The arithmetic lives in ``pa_oracle.c`` (plain C, double precision); this
 module is argument marshalling over numpy arrays of raw 16-bit patterns.
 
-Functions and what they follow (page titles are given in full in pa_oracle.c):
+Pages cited: P1 "大模型部署中的PagedAttention：KV Cache显存管理突破"; P2 "大模型推理优化：KV
+Cache与PagedAttention技术详解"; P3 "LLM 推理中的 PageAttention 实现原理：虚拟内存管理在 KV
+Cache 中的创新应用".
+
+Functions and what they follow:
   decode               softmax(q K^T * scale) V, one softmax over all tokens (P1 §1)
   reshape_and_cache    new K/V rows copied into their slots, bit for bit (P2 §2.1)
   copy_blocks          whole-block copies for copy-on-write after a fork (P3 §四)

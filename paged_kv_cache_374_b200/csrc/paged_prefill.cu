@@ -1,7 +1,8 @@
 // Paged prefill: causal attention of a chunk of new query tokens over the paged
 // cache -- the step before decode (P2 "大模型推理优化：KV Cache与PagedAttention技术详解",
 // §2.1: the prompt's K/V enter the cache, then every position attends to the ones
-// before it; prefix reuse across requests, P3 §三, makes the chunk start after
+// before it; prefix reuse across requests, P3 "LLM 推理中的 PageAttention 实现原理：虚拟内存管理在 KV Cache
+// 中的创新应用" §三, makes the chunk start after
 // cached tokens).  Query row i of sequence s (chunk of n rows over L tokens) sits
 // at position L - n + i and attends to tokens 0 .. L - n + i through the table.
 //

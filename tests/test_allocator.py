@@ -1,4 +1,5 @@
-"""The C++ host allocator against the Python model of the pages' block pool, id for id."""
+"""The C++ host allocator against the Python model of the pages' block pool, id for id
+(P3 = "LLM 推理中的 PageAttention 实现原理：虚拟内存管理在 KV Cache 中的创新应用")."""
 import json
 import os
 

@@ -1,4 +1,5 @@
-"""The allocator model against the demo program of P3 §三 (main) and its own rules."""
+"""The allocator model against the demo program of P3 ("LLM 推理中的 PageAttention 实现原理：虚拟内存管理在
+KV Cache 中的创新应用") §三 (main) and its own rules."""
 import json
 import os
 
