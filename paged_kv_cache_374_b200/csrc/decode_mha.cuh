@@ -33,10 +33,15 @@ struct MhaPolicy {
     static constexpr int DUP = 4 / NROW;   // lanes that end up holding one token's score
     static constexpr int HALF_BYTES = TOK * 128;
 
+    // fp8 codes with fp16 q: q K^T as f32 += f16 * f16 (sm_100 mixed-precision fma) on
+    // the raw q pairs and the exactly widened codes; the scale is applied to the sum
+    static constexpr bool kMixed = CTag::kBytes == 1 && !Tag::kIsBF16;
+
     int lane, r, c;
     int swz[NCH];       // offset of this lane's chunk j of row r in a tile
     uint4 qn[DL / 8];   // raw q of the next unit
     float2 qc[DL / 2];  // q of the current unit, pre-scaled by scale * log2(e)
+    uint32_t qh[DL / 2];  // kMixed: raw q of the current unit as f16 pairs
     float m, lsum;
     float2 o[DL / 2];
     bool poisoned;
@@ -62,6 +67,16 @@ struct MhaPolicy {
     }
 
     __device__ __forceinline__ void take_q(const DecodeArgs& a) {
+        if constexpr (kMixed) {
+#pragma unroll
+            for (int j = 0; j < DL / 8; ++j) {
+                qh[4 * j] = qn[j].x;
+                qh[4 * j + 1] = qn[j].y;
+                qh[4 * j + 2] = qn[j].z;
+                qh[4 * j + 3] = qn[j].w;
+            }
+            return;
+        }
         const float sc = a.scale_log2 * a.k_scale;
 #pragma unroll
         for (int j = 0; j < DL / 8; ++j) {
@@ -96,8 +111,17 @@ struct MhaPolicy {
 
     __device__ __forceinline__ void poison() { poisoned = true; }
 
+    // acc + lo(a) lo(b) + hi(a) hi(b) for two f16 pairs, accumulated in f32
+    static __device__ __forceinline__ float2 fma_f16x2(uint32_t a2, uint32_t b2, float2 acc) {
+        float2 d;
+        asm("{\n\t.reg .f16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %2;\n\tmov.b32 {bl, bh}, %3;\n\t"
+            "fma.rn.f32.f16 %0, al, bl, %4;\n\tfma.rn.f32.f16 %1, ah, bh, %5;\n\t}"
+            : "=f"(d.x), "=f"(d.y)
+            : "r"(a2), "r"(b2), "f"(acc.x), "f"(acc.y));
+        return d;
+    }
+
     __device__ __forceinline__ void stage(const DecodeArgs& a, const uint8_t* kt, const uint8_t* vt, int ntok) {
-        (void)a;
         // partial dot products of rows i*8 + r over this lane's dims
         float acc[NROW];
 #pragma unroll
@@ -106,12 +130,22 @@ struct MhaPolicy {
 #pragma unroll
             for (int j = 0; j < NCH; ++j) {
                 const uint4 w = *reinterpret_cast<const uint4*>(kt + i * 1024 + swz[j]);
-                float2 kf[EPC / 2];
-                widen_chunk(w, kf);
+                if constexpr (kMixed) {
+                    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int k = 0; k < EPC / 2; ++k) d2 = __ffma2_rn(qc[j * (EPC / 2) + k], kf[k], d2);
+                    for (int k = 0; k < 4; ++k) {
+                        d2 = fma_f16x2(qh[j * 8 + 2 * k], E4M3Tag::to_f16x2(words[k] & 0xffffu), d2);
+                        d2 = fma_f16x2(qh[j * 8 + 2 * k + 1], E4M3Tag::to_f16x2(words[k] >> 16), d2);
+                    }
+                } else {
+                    float2 kf[EPC / 2];
+                    widen_chunk(w, kf);
+#pragma unroll
+                    for (int k = 0; k < EPC / 2; ++k) d2 = __ffma2_rn(qc[j * (EPC / 2) + k], kf[k], d2);
+                }
             }
             acc[i] = d2.x + d2.y;
+            if constexpr (kMixed) acc[i] *= a.scale_log2 * a.k_scale;
         }
         // reduce over the 4 lanes of a row (lane bits 4 and 3), scattering the
         // NROW rows so that lane c keeps row group g(c)
