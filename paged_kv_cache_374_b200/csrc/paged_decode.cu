@@ -252,28 +252,29 @@ int launch_decode(DecodeArgs args, const void* k_cache, const void* v_cache, int
 }
 
 // fp8 (E4M3) caches.  GQA groups of 2-16: tensor cores, one kv head with its whole
-// query group per unit (one fetch of the codes serves the group), 16-token slots
-// widened into per-warp 16-bit tiles.  MHA (and larger groups): CUDA cores, one
+// query group per unit (one fetch of the codes serves the group), codes widened
+// into per-warp 16-bit tiles.  MHA (and larger groups): CUDA cores, one
 // query head per unit, 32-token slots (8 KiB): with a single head the tensor-core
 // stage carries too little work per byte to keep up.
 template <class Tag>
 int launch_decode_fp8(DecodeArgs args, const void* k_cache, const void* v_cache, int num_kv_heads,
                       cudaStream_t stream) {
-    constexpr int TOK = 16;
+    // 32-token slots of codes (8 KiB) and a 16-token scratch pair (8 KiB): 8 warps keep
+    // 128 KiB of codes in flight per SM
+    constexpr int TOK = 32;
     if (args.group >= 2 && args.group <= PA_GQA_MAX_GROUP) {
         args.unit_heads = num_kv_heads;
         args.heads_per_unit = args.group;
         if (args.group <= 8)
-            return launch_engine<Tag, E4M3Tag, 128, TOK, 12, 2, Fp8TcPolicy<Tag, TOK, 1>>(args, k_cache, v_cache,
-                                                                                            num_kv_heads, stream);
+            return launch_engine<Tag, E4M3Tag, 128, TOK, 8, 2, Fp8TcPolicy<Tag, TOK, 1>>(args, k_cache, v_cache,
+                                                                                           num_kv_heads, stream);
         return launch_engine<Tag, E4M3Tag, 128, TOK, 8, 2, Fp8TcPolicy<Tag, TOK, 2>>(args, k_cache, v_cache,
                                                                                        num_kv_heads, stream);
     }
-    constexpr int TOK32 = 32;
     args.unit_heads = args.num_heads;
     args.heads_per_unit = 1;
-    return launch_engine<Tag, E4M3Tag, 128, TOK32, PA_DECODE_WARPS, PA_DECODE_SLOTS,
-                         MhaPolicy<Tag, E4M3Tag, 128, TOK32>>(args, k_cache, v_cache, num_kv_heads, stream);
+    return launch_engine<Tag, E4M3Tag, 128, TOK, PA_DECODE_WARPS, PA_DECODE_SLOTS, MhaPolicy<Tag, E4M3Tag, 128, TOK>>(
+        args, k_cache, v_cache, num_kv_heads, stream);
 }
 
 }  // namespace
