@@ -54,7 +54,9 @@ def test_cache_write_codes_are_bit_exact():
         assert np.array_equal(kc.cpu().numpy(), kh) and np.array_equal(vc.cpu().numpy(), vh)
 
 
-SHAPES = [(16, 1, F16), (32, 1, BF16), (64, 1, F16), (16, 8, BF16), (32, 4, F16)]
+# groups 1 (CUDA cores), 2-8 and 16 (tensor cores, one or two head tiles), 32 (CUDA cores again)
+SHAPES = [(16, 1, F16), (32, 1, BF16), (64, 1, F16), (16, 8, BF16), (32, 4, F16), (64, 2, BF16), (16, 16, F16),
+          (32, 16, BF16), (16, 32, F16)]
 
 
 @pytest.mark.parametrize("bs,g,dtype", SHAPES)
