@@ -237,6 +237,18 @@ int pa_find_shared_prefixes(const int32_t* block_tables, const int32_t* context_
                             int32_t* group_offsets, int32_t* group_members, int* num_groups, int* max_group_size,
                             int* max_shared_tokens);
 
+/* ------------------------------------------------------------ diagnostics */
+
+/*
+ * pa_selftest_bounded_wait -- no counterpart on the pages: a check of the
+ * library's failure path.  Launches one warp that waits, with the library's
+ * bounded mbarrier wait, on a barrier nothing arrives at.  The wait gives up by
+ * itself (its bound is about 2 s), OR-s PA_DEVERR_TIMEOUT into *err_word and the
+ * kernel returns; the context stays usable.  *outcome (device int32, may be
+ * NULL) becomes 0 when the wait gave up (1 would mean the phase completed).
+ */
+int pa_selftest_bounded_wait(int32_t* err_word, int32_t* outcome, void* stream);
+
 /* ---------------------------------------------------------------- fp8 cache */
 
 /*

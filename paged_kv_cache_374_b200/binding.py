@@ -56,6 +56,7 @@ _sig("pa_decode_shared_prefix", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _
      _i32, _i32, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
 _sig("pa_find_shared_prefixes", _i32, _i32p, _i32p, _i32, _i32, _i32, _i32, _i32p, _i32p, _i32p,
      ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int))
+_sig("pa_selftest_bounded_wait", _i32, _vp, _vp, _vp)
 _sig("pa_allocator_create", _vp, _i32, _i32p)
 _sig("pa_allocator_destroy", None, _vp)
 _sig("pa_num_required_blocks", _i32, _i32, _i32)
@@ -260,6 +261,14 @@ def pa_decode_shared_prefix(q, k_cache, v_cache, block_tables, context_lens, sca
         _stream(stream, q))
     _check(st, "pa_decode_shared_prefix")
     return out
+
+
+def pa_selftest_bounded_wait(err_word, outcome=None, stream=None) -> None:
+    """Run the bounded-wait check (a wait nothing completes must time out and report)."""
+    import torch
+    st = _lib.pa_selftest_bounded_wait(_dev(err_word, "err_word", torch.int32), _dev(outcome, "outcome", torch.int32),
+                                       _stream(stream, err_word))
+    _check(st, "pa_selftest_bounded_wait")
 
 
 def pa_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out,

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIBRARY = os.path.join(PKG, "libpa.so")
 SOURCES = ["allocator.cpp", "reshape_and_cache.cu", "paged_decode.cu", "paged_decode_noalloc.cu", "copy_blocks.cu",
-           "paged_prefill.cu"]
+           "paged_prefill.cu", "selftest.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-Xcompiler", "-fPIC,-O2,-Wall", "-shared", "-cudart", "static"]
 

@@ -142,3 +142,18 @@ def test_empty_batch_and_binding_checks():
                      torch.ones(1, dtype=torch.int32, device="cuda"), 0.1, 4,
                      torch.zeros(1, 4, 96, dtype=torch.float16, device="cuda"))
     assert e.value.status == pa.PA_ERR_UNSUPPORTED
+
+
+def test_bounded_wait_gives_up_and_reports():
+    """A wait on a barrier that nothing completes runs out by itself, reports
+    PA_DEVERR_TIMEOUT, and the context keeps working afterwards."""
+    import time
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    outcome = torch.full((1,), 7, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    pa.pa_selftest_bounded_wait(err, outcome)
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 30
+    assert outcome.item() == 0 and err.item() == pa.PA_DEVERR_TIMEOUT
+    c = PagedCase(np.random.default_rng(80), [100, 300], 4, 4, 128, 16, F16, 0.1)
+    assert_close(run_case(c), c.run(oracle_pkg.get()), "f16", "decode after the self-test")
