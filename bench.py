@@ -40,6 +40,11 @@ PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "paged_decode_llama7b.md")
 DECODE_SOURCES = [os.path.join(ROOT, "paged_kv_cache_374_b200", "csrc", f) for f in
                   ("paged_decode.cu", "decode_engine.cuh", "decode_mha.cuh", "decode_gqa.cuh", "decode_fp8tc.cuh",
                    "pa_device.cuh")]
+GQA_PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "paged_decode_gqa70b.md")
+# ncu summaries that give roofline.traffic, by workload (+fp8 for the e4m3 cache)
+TRAFFIC_SUMMARIES = {"llama7b": PROFILE_SUMMARY, "gqa70b": GQA_PROFILE_SUMMARY,
+                     "llama13b": os.path.join(ROOT, "profiles", "paged_decode_llama13b.md"),
+                     "llama7b+fp8": os.path.join(ROOT, "profiles", "paged_decode_fp8_llama7b.md")}
 SHARED_PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "shared_prefix_beam.md")
 SHARED_SOURCES = DECODE_SOURCES + [os.path.join(ROOT, "paged_kv_cache_374_b200", "csrc", f) for f in
                                    ("paged_prefill.cu", "tcgen05.cuh")]
@@ -111,10 +116,11 @@ def source_digest(paths):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(units_now: int, summary=PROFILE_SUMMARY, sources=DECODE_SOURCES):
+def profiled_traffic(units_now: int, workload: str, summary=PROFILE_SUMMARY, sources=DECODE_SOURCES):
     """DRAM bytes per launch of the decode kernels from a committed ncu summary,
-    scaled to this launch's (unique) tokens; None when the summary is missing or
-    a kernel source has changed since the counters were taken."""
+    scaled to this launch's (unique) tokens; None when the summary is missing, was
+    taken on another workload (bytes per token depend on the head counts), or a
+    kernel source has changed since the counters were taken."""
     try:
         fields = {}
         with open(summary) as f:
@@ -122,7 +128,7 @@ def profiled_traffic(units_now: int, summary=PROFILE_SUMMARY, sources=DECODE_SOU
                 if line.startswith("- ") and ": " in line:
                     k, v = line[2:].split(": ", 1)
                     fields[k.strip()] = v.strip().strip("`")
-        if fields.get("source_sha256_16") != source_digest(sources):
+        if fields.get("workload") != workload or fields.get("source_sha256_16") != source_digest(sources):
             return None
         per_token = float(fields["dram_bytes_per_launch"]) / float(fields["tokens_per_launch"])
         return per_token * units_now
@@ -321,20 +327,21 @@ def run_native(args):
         else:
             pa.pa_reshape_and_cache(k, v, slots, st["k_cache"], st["v_cache"], stream=stream)
 
-    def k2(q, tables, lens, groups=None):
+    def k2(q, tables, lens, groups=None, out=None):
         g = st["groups"]
+        out = st["out"] if out is None else out
         if g is not None:
             start, offs, mem = groups if groups is not None else st["group_dev"]
             pa.pa_decode_shared_prefix(q, st["k_cache"], st["v_cache"], tables, lens, spec.scale, spec.num_kv_heads,
-                                       st["out"], start, offs, mem, g.num_groups, g.max_group_size,
+                                       out, start, offs, mem, g.num_groups, g.max_group_size,
                                        g.max_shared_tokens, workspace=st["workspace"],
                                        partition_tokens=st["partition_tokens"], stream=stream)
         elif fp8:
             pa.pa_decode_fp8(q, st["k_cache"], st["v_cache"], tables, lens, spec.scale, ks, vs, spec.num_kv_heads,
-                             st["out"], workspace=st["workspace"], partition_tokens=st["partition_tokens"],
+                             out, workspace=st["workspace"], partition_tokens=st["partition_tokens"],
                              stream=stream)
         else:
-            pa.pa_decode(q, st["k_cache"], st["v_cache"], tables, lens, spec.scale, spec.num_kv_heads, st["out"],
+            pa.pa_decode(q, st["k_cache"], st["v_cache"], tables, lens, spec.scale, spec.num_kv_heads, out,
                          workspace=st["workspace"], partition_tokens=st["partition_tokens"], stream=stream)
 
     def step():
@@ -350,8 +357,7 @@ def run_native(args):
         step()
     barrier()
 
-    # timed region: K steps, with per-kernel events on the launching stream
-    k1_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # timed region: K steps; the roofline kernel (K2+K3) carries events on the launching stream
     k2_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(gpu_uuid(torch, device)) if not args.no_clocks else None
@@ -360,9 +366,7 @@ def run_native(args):
     barrier()
     start.record(stream)
     for i in range(args.steps):
-        k1_ev[i][0].record(stream)
         k1(st["k"], st["v"], st["slots"])
-        k1_ev[i][1].record(stream)
         k2_ev[i][0].record(stream)
         k2(st["q"], st["tables"], st["lens"])
         k2_ev[i][1].record(stream)
@@ -371,54 +375,101 @@ def run_native(args):
     if sampler:
         sampler.__exit__(None, None, None)
     elapsed_ms = start.elapsed_time(stop)
-    k1_ms = statistics.mean(a.elapsed_time(b) for a, b in k1_ev)
     k2_ms = statistics.mean(a.elapsed_time(b) for a, b in k2_ev)
     (elapsed_ms,) = max_over_ranks([elapsed_ms], dist if world > 1 else None, device)
 
-    # e2e through the binding: per step, H2D of the step's inputs from pinned
-    # host memory, K1, K2(+K3), D2H of the output
-    host = {k: st[k].cpu().pin_memory() for k in ("q", "k", "v", "slots", "tables", "lens")}
-    out_h = torch.empty(st["out"].shape, dtype=st["out"].dtype).pin_memory()
-    dev_in = {k: torch.empty_like(st[k]) for k in host}
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out_h.numel() * out_h.element_size()
+    # K1 alone, for the detail line (outside the timed region)
+    k1_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(200)]
+    for a, b in k1_ev:
+        a.record(stream)
+        k1(st["k"], st["v"], st["slots"])
+        b.record(stream)
+    barrier()
+    k1_ms = statistics.mean(a.elapsed_time(b) for a, b in k1_ev)
 
-    grp_dev = None
-    if st["groups"] is not None:  # the grouping is redone from the host tables every step
-        grp_dev = [torch.empty(st["spec"].num_seqs + 1, dtype=torch.int32, device=device) for _ in range(3)]
-        grp_h = [torch.empty(st["spec"].num_seqs + 1, dtype=torch.int32).pin_memory() for _ in range(3)]
-        h2d += 4 * (2 * st["spec"].num_seqs + 1 + st["groups"].num_groups + 1)
+    # e2e through the binding, two steps in flight: step i+1's inputs go H2D from
+    # pinned host memory on a copy stream while step i computes, and each step's
+    # output goes D2H on a third stream.  Every step still copies all of its own
+    # inputs and reads back its own result inside the timed region.
+    nbuf = 2
+    names = ("q", "k", "v", "slots", "tables", "lens")
+    offs, h2d = {}, 0
+    for n in names:                       # one staging buffer: 256-byte aligned fields
+        offs[n] = h2d
+        h2d += -(-st[n].numel() * st[n].element_size() // 256) * 256
+    host_buf = torch.empty(h2d, dtype=torch.uint8).pin_memory()
+    for n in names:
+        nb = st[n].numel() * st[n].element_size()
+        host_buf[offs[n]:offs[n] + nb].copy_(st[n].cpu().contiguous().view(-1).view(torch.uint8))
+    dev_buf = [torch.empty(h2d, dtype=torch.uint8, device=device) for _ in range(nbuf)]
+    dev_in = [{n: dev_buf[b][offs[n]:offs[n] + st[n].numel() * st[n].element_size()].view(st[n].dtype)
+               .view(st[n].shape) for n in names} for b in range(nbuf)]
+    out_d = [torch.empty_like(st["out"]) for _ in range(nbuf)]
+    out_h = [torch.empty(st["out"].shape, dtype=st["out"].dtype).pin_memory() for _ in range(nbuf)]
+    d2h = out_h[0].numel() * out_h[0].element_size()
+    h2d_stream, d2h_stream = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(nbuf)]     # set b's inputs are on the device
+    ev_used = [torch.cuda.Event() for _ in range(nbuf)]   # K1/K2 of set b are done (inputs read, out_d[b] written)
+    ev_out = [torch.cuda.Event() for _ in range(nbuf)]    # out_d[b] is back on the host
 
-    def e2e_step():
-        for k, v in host.items():
-            dev_in[k].copy_(v, non_blocking=True)
+    grp_dev = grp_h = None
+    if st["groups"] is not None:  # the grouping is redone from the host tables every step: one int32 buffer of
+        n1 = spec.num_seqs + 1    # seq_start | group_offsets | group_members, (num_seqs + 1) entries each
+        grp_dev = [torch.empty(3 * n1, dtype=torch.int32, device=device) for _ in range(nbuf)]
+        grp_h = [torch.zeros(3 * n1, dtype=torch.int32).pin_memory() for _ in range(nbuf)]
+        h2d += 4 * 3 * n1
+
+    def e2e_step(i):
+        b = i % nbuf
         groups = None
         if grp_dev is not None:
             g = pa.pa_find_shared_prefixes(st["tables_h"], st["lens_h"], spec.block_size, st["ptok"])
+            ev_in[b].synchronize()                     # the copy that last read grp_h[b] is done
+            hv = grp_h[b].numpy()
             groups = []
-            for hbuf, dbuf, arr in zip(grp_h, grp_dev, (g.seq_start, g.group_offsets, g.group_members)):
-                n = len(arr)
-                hbuf[:n].copy_(torch.from_numpy(arr))
-                dbuf[:n].copy_(hbuf[:n], non_blocking=True)
-                groups.append(dbuf[:n])
-        k1(dev_in["k"], dev_in["v"], dev_in["slots"])
-        k2(dev_in["q"], dev_in["tables"], dev_in["lens"], groups)
-        out_h.copy_(st["out"], non_blocking=True)
+            for part, arr in enumerate((g.seq_start, g.group_offsets, g.group_members)):
+                hv[part * n1:part * n1 + len(arr)] = arr
+                groups.append(grp_dev[b][part * n1:part * n1 + len(arr)])
+        with torch.cuda.stream(h2d_stream):
+            h2d_stream.wait_event(ev_used[b])          # the step two back has finished with set b
+            dev_buf[b].copy_(host_buf, non_blocking=True)
+            if grp_dev is not None:
+                grp_dev[b].copy_(grp_h[b], non_blocking=True)
+            ev_in[b].record(h2d_stream)
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_out[b])                   # out_d[b] of the step two back is on the host
+        k1(dev_in[b]["k"], dev_in[b]["v"], dev_in[b]["slots"])
+        k2(dev_in[b]["q"], dev_in[b]["tables"], dev_in[b]["lens"], groups, out=out_d[b])
+        ev_used[b].record(stream)
+        d2h_stream.wait_event(ev_used[b])
+        with torch.cuda.stream(d2h_stream):
+            out_h[b].copy_(out_d[b], non_blocking=True)
+            ev_out[b].record(d2h_stream)
 
-    e2e_steps = max(1, min(args.steps, 500))
-    for _ in range(3):
-        e2e_step()
+    e2e_steps = args.steps
+    for i in range(3):
+        e2e_step(i)
     barrier()
+    e2e_sampler = ClockSampler(gpu_uuid(torch, device)) if not args.no_clocks else None
+    if e2e_sampler:
+        e2e_sampler.__enter__()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    h2d_stream.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    stream.wait_event(ev_out[(e2e_steps - 1) % nbuf])  # the last read-back (the D2H stream runs in order)
     e1.record(stream)
     barrier()
+    if e2e_sampler:
+        e2e_sampler.__exit__(None, None, None)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    # the pipelined steps compute what the device-timed ones did (same inputs, same cache slots)
+    e2e_matches = bool(torch.equal(out_h[(e2e_steps - 1) % nbuf], st["out"].cpu()))
     (e2e_ms,) = max_over_ranks([e2e_ms], dist if world > 1 else None, device)
 
     ab = algorithmic_bytes(st)
+    traffic_key = args.workload + ("+fp8" if fp8 else "")
     ms_per_step = elapsed_ms / args.steps
     tokens_per_step = spec.num_seqs
     value = job_throughput(world, tokens_per_step, ms_per_step)
@@ -450,7 +501,7 @@ def run_native(args):
             "kv_gbs": round(achieved, 1), "frac_of_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
             "kv_bytes_per_step": ab["unique"], "logical_kv_bytes_per_step": ab["logical"],
             "k1_us": round(k1_ms * 1e3, 2), "k2k3_us": round(k2_ms * 1e3, 2), "a1_us": round(st["a1_us"], 1),
-            "e2e_ms_per_step": round(e2e_ms, 4),
+            "e2e_ms_per_step": round(e2e_ms, 4), "e2e_output_matches": e2e_matches,
         },
         "roofline": {
             "kernel": ("shared-prefix kernel + paged_decode_kernel + paged_decode_merge_kernel (timed together: one "
@@ -458,12 +509,14 @@ def run_native(args):
                        "paged_decode_kernel + paged_decode_merge_kernel (timed together: one pa_decode call)"),
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
             "unit": "GB/s", "frac": round(achieved / peak, 4),
-            "traffic": (None if fp8 else
-                        profiled_traffic(ab["unique_tokens"], SHARED_PROFILE_SUMMARY, SHARED_SOURCES)
-                        if st["groups"] is not None else profiled_traffic(ab["unique_tokens"])),
+            "traffic": (profiled_traffic(ab["unique_tokens"], args.workload, SHARED_PROFILE_SUMMARY, SHARED_SOURCES)
+                        if st["groups"] is not None else
+                        profiled_traffic(ab["unique_tokens"], traffic_key,
+                                         TRAFFIC_SUMMARIES.get(traffic_key, PROFILE_SUMMARY))),
         },
         "e2e": {"value": round(job_throughput(world, tokens_per_step, e2e_ms), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "clocks": e2e_sampler.summary() if e2e_sampler else None},
         "gpu_launches": args.steps * launches_per_step,
         "clocks": sampler.summary() if sampler else None,
     }

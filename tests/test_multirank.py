@@ -6,6 +6,7 @@ job time is the slowest rank's and the job throughput counts every rank's tokens
 import os
 import socket
 
+import pytest
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
@@ -48,3 +49,18 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks([1.5, 2.5]) == [1.5, 2.5]
     assert bench.job_throughput(1, 64, 0.4) == 64 / 0.0004
+
+
+def test_profiled_traffic_comes_only_from_the_same_workload():
+    """roofline.traffic scales a capture by tokens only when the capture is of the
+    same workload (bytes per token depend on the head counts) and the kernel
+    sources are the ones it was taken on."""
+    import bench
+    per_token_7b = 629657088 / 37801
+    assert bench.profiled_traffic(1000, "llama7b") == pytest.approx(1000 * per_token_7b)
+    assert bench.profiled_traffic(1000, "llama13b") is None
+    assert bench.profiled_traffic(1000, "gqa70b", bench.GQA_PROFILE_SUMMARY) == pytest.approx(
+        1000 * 203340544 / 47015)
+    assert bench.profiled_traffic(1000, "gqa70b") is None           # the 7B capture does not serve gqa70b
+    assert bench.profiled_traffic(1000, "beam", bench.SHARED_PROFILE_SUMMARY, bench.SHARED_SOURCES) is not None
+    assert bench.profiled_traffic(1000, "beam", bench.SHARED_PROFILE_SUMMARY) is None   # other source set
