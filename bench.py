@@ -37,17 +37,12 @@ METRIC = "decode-attention tokens/s and KV-cache HBM GB/s (fraction of ~8 TB/s) 
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "paged_decode_llama7b.md")
-DECODE_SOURCES = [os.path.join(ROOT, "paged_kv_cache_374_b200", "csrc", f) for f in
-                  ("paged_decode.cu", "decode_engine.cuh", "decode_mha.cuh", "decode_gqa.cuh", "decode_fp8tc.cuh",
-                   "pa_device.cuh")]
 GQA_PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "paged_decode_gqa70b.md")
 # ncu summaries that give roofline.traffic, by workload (+fp8 for the e4m3 cache)
 TRAFFIC_SUMMARIES = {"llama7b": PROFILE_SUMMARY, "gqa70b": GQA_PROFILE_SUMMARY,
                      "llama13b": os.path.join(ROOT, "profiles", "paged_decode_llama13b.md"),
                      "llama7b+fp8": os.path.join(ROOT, "profiles", "paged_decode_fp8_llama7b.md")}
 SHARED_PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "shared_prefix_beam.md")
-SHARED_SOURCES = DECODE_SOURCES + [os.path.join(ROOT, "paged_kv_cache_374_b200", "csrc", f) for f in
-                                   ("paged_prefill.cu", "tcgen05.cuh")]
 
 
 def parse():
@@ -116,11 +111,12 @@ def source_digest(paths):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(units_now: int, workload: str, summary=PROFILE_SUMMARY, sources=DECODE_SOURCES):
+def profiled_traffic(units_now: int, workload: str, summary=PROFILE_SUMMARY):
     """DRAM bytes per launch of the decode kernels from a committed ncu summary,
     scaled to this launch's (unique) tokens; None when the summary is missing, was
-    taken on another workload (bytes per token depend on the head counts), or a
-    kernel source has changed since the counters were taken."""
+    taken on another workload (bytes per token depend on the head counts), or one
+    of the sources the profiled kernels are built from (the summary's `sources`)
+    has changed since the counters were taken."""
     try:
         fields = {}
         with open(summary) as f:
@@ -128,6 +124,8 @@ def profiled_traffic(units_now: int, workload: str, summary=PROFILE_SUMMARY, sou
                 if line.startswith("- ") and ": " in line:
                     k, v = line[2:].split(": ", 1)
                     fields[k.strip()] = v.strip().strip("`")
+        sources = [os.path.join(ROOT, "paged_kv_cache_374_b200", "csrc", n.strip())
+                   for n in fields["sources"].split(",")]
         if fields.get("workload") != workload or fields.get("source_sha256_16") != source_digest(sources):
             return None
         per_token = float(fields["dram_bytes_per_launch"]) / float(fields["tokens_per_launch"])
@@ -509,7 +507,7 @@ def run_native(args):
                        "paged_decode_kernel + paged_decode_merge_kernel (timed together: one pa_decode call)"),
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
             "unit": "GB/s", "frac": round(achieved / peak, 4),
-            "traffic": (profiled_traffic(ab["unique_tokens"], args.workload, SHARED_PROFILE_SUMMARY, SHARED_SOURCES)
+            "traffic": (profiled_traffic(ab["unique_tokens"], args.workload, SHARED_PROFILE_SUMMARY)
                         if st["groups"] is not None else
                         profiled_traffic(ab["unique_tokens"], traffic_key,
                                          TRAFFIC_SUMMARIES.get(traffic_key, PROFILE_SUMMARY))),

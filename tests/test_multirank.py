@@ -51,10 +51,10 @@ def test_single_rank_is_identity():
     assert bench.job_throughput(1, 64, 0.4) == 64 / 0.0004
 
 
-def test_profiled_traffic_comes_only_from_the_same_workload():
+def test_profiled_traffic_comes_only_from_the_same_workload(tmp_path):
     """roofline.traffic scales a capture by tokens only when the capture is of the
-    same workload (bytes per token depend on the head counts) and the kernel
-    sources are the ones it was taken on."""
+    same workload (bytes per token depend on the head counts) and the sources its
+    kernels are built from are the ones it was taken on."""
     import bench
     per_token_7b = 629657088 / 37801
     assert bench.profiled_traffic(1000, "llama7b") == pytest.approx(1000 * per_token_7b)
@@ -62,5 +62,10 @@ def test_profiled_traffic_comes_only_from_the_same_workload():
     assert bench.profiled_traffic(1000, "gqa70b", bench.GQA_PROFILE_SUMMARY) == pytest.approx(
         1000 * 203340544 / 47015)
     assert bench.profiled_traffic(1000, "gqa70b") is None           # the 7B capture does not serve gqa70b
-    assert bench.profiled_traffic(1000, "beam", bench.SHARED_PROFILE_SUMMARY, bench.SHARED_SOURCES) is not None
-    assert bench.profiled_traffic(1000, "beam", bench.SHARED_PROFILE_SUMMARY) is None   # other source set
+    assert bench.profiled_traffic(1000, "beam", bench.SHARED_PROFILE_SUMMARY) is not None
+    # a summary whose recorded digest no longer matches its sources gives no traffic
+    stale = tmp_path / "stale.md"
+    text = open(bench.PROFILE_SUMMARY).read()
+    line = next(ln for ln in text.splitlines() if ln.startswith("- source_sha256_16: "))
+    stale.write_text(text.replace(line, "- source_sha256_16: 0000000000000000"))
+    assert bench.profiled_traffic(1000, "llama7b", str(stale)) is None
