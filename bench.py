@@ -41,7 +41,8 @@ GQA_PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "paged_decode_gqa70b.md")
 # ncu summaries that give roofline.traffic, by workload (+fp8 for the e4m3 cache)
 TRAFFIC_SUMMARIES = {"llama7b": PROFILE_SUMMARY, "gqa70b": GQA_PROFILE_SUMMARY,
                      "llama13b": os.path.join(ROOT, "profiles", "paged_decode_llama13b.md"),
-                     "llama7b+fp8": os.path.join(ROOT, "profiles", "paged_decode_fp8_llama7b.md")}
+                     "llama7b+fp8": os.path.join(ROOT, "profiles", "paged_decode_fp8_llama7b.md"),
+                     "gqa70b+fp8": os.path.join(ROOT, "profiles", "paged_decode_fp8_gqa70b.md")}
 SHARED_PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "shared_prefix_beam.md")
 
 

@@ -76,6 +76,72 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
     return y;
 }
 
+// One online-softmax step over a 16-token tile of S^T, shared by the tensor-core
+// policies.  This lane holds tokens g and g+8 x query heads 2t, 2t+1 of each of the
+// NT head tiles (the m16n8 accumulator layout).  The raw dot products are scaled
+// by sc into base-2 units, tokens at or past nv are masked, the per-head running
+// max (and with it the rescale of lsum and of O^T) moves only when some score
+// exceeds it, and P^T is returned as the B fragments of V^T P^T: p = hi + lo in
+// 16-bit pairs of the MMA type P, transposed to (head row, tokens 2t/2t+1).
+template <class P, int NT, int MT>
+__device__ __forceinline__ void gqa_softmax_tile(float (&x)[NT][4], int g, int nv, float sc, float (&m)[NT][2],
+                                                 float (&lsum)[NT][2], float (&o)[NT][MT][4],
+                                                 uint32_t (&bhi)[NT][2], uint32_t (&blo)[NT][2]) {
+    const bool v0 = g < nv, v1 = g + 8 < nv;
+    bool up = false;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x[nt][j] *= sc;
+        if (!v0) x[nt][0] = x[nt][1] = -INFINITY;
+        if (!v1) x[nt][2] = x[nt][3] = -INFINITY;
+        up |= x[nt][0] > m[nt][0] || x[nt][2] > m[nt][0] || x[nt][1] > m[nt][1] || x[nt][3] > m[nt][1];
+    }
+    if (__any_sync(kFullMask, up)) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                float mx = fmaxf(x[nt][j], x[nt][j + 2]);
+                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 16));
+                const float m_new = fmaxf(m[nt][j], mx);
+                const float alpha = fast_exp2(m[nt][j] - m_new);
+                lsum[nt][j] *= alpha;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    o[nt][mt][j] *= alpha;
+                    o[nt][mt][j + 2] *= alpha;
+                }
+                m[nt][j] = m_new;
+            }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        float p[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) p[j] = fast_exp2(x[nt][j] - m[nt][j & 1]);
+        lsum[nt][0] += p[0] + p[2];
+        lsum[nt][1] += p[1] + p[3];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const uint32_t hi = MmaOps<P>::pack(p[2 * half], p[2 * half + 1]);
+            const float2 hv = P::widen2(hi);
+            const uint32_t lo = MmaOps<P>::pack(p[2 * half] - hv.x, p[2 * half + 1] - hv.y);
+            bhi[nt][half] = movmatrix_trans(hi);
+            blo[nt][half] = movmatrix_trans(lo);
+        }
+    }
+}
+
+// Keep-mask of a 16-bit pair holding tokens k and k+1 of a tile with nv valid
+// tokens.  Rows past the sequence end may hold anything (NaN included): their p
+// is 0, but 0 * NaN is NaN inside the MMA, so their V entries are zeroed.
+__device__ __forceinline__ uint32_t gqa_pair_mask(int k, int nv) {
+    return (k < nv ? 0x0000ffffu : 0u) | (k + 1 < nv ? 0xffff0000u : 0u);
+}
+
 template <class Tag, int D, int TOK, int NT>
 struct GqaPolicy {
     static constexpr int KS = D / 16;     // k-steps of q K^T over the head dims
@@ -171,62 +237,11 @@ struct GqaPolicy {
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) Ops::mma(x[nt], af, qb[nt][ks][0], qb[nt][ks][1]);
             }
-            const bool v0 = g < nv, v1 = g + 8 < nv;
             const float sc = a.scale_log2 * a.k_scale;  // k_scale: 1, or the fp8 cache's K scale
-            bool up = false;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) x[nt][j] *= sc;
-                if (!v0) x[nt][0] = x[nt][1] = -INFINITY;
-                if (!v1) x[nt][2] = x[nt][3] = -INFINITY;
-                up |= x[nt][0] > m[nt][0] || x[nt][2] > m[nt][0] || x[nt][1] > m[nt][1] || x[nt][3] > m[nt][1];
-            }
-            // per-head max over the tile's tokens and rescale, only when needed
-            if (__any_sync(kFullMask, up)) {
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        float mx = fmaxf(x[nt][j], x[nt][j + 2]);
-                        mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 4));
-                        mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 8));
-                        mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 16));
-                        const float m_new = fmaxf(m[nt][j], mx);
-                        const float alpha = fast_exp2(m[nt][j] - m_new);
-                        lsum[nt][j] *= alpha;
-#pragma unroll
-                        for (int mt = 0; mt < MT; ++mt) {
-                            o[nt][mt][j] *= alpha;
-                            o[nt][mt][j + 2] *= alpha;
-                        }
-                        m[nt][j] = m_new;
-                    }
-            }
             uint32_t bhi[NT][2], blo[NT][2];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                float p[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) p[j] = fast_exp2(x[nt][j] - m[nt][j & 1]);
-                lsum[nt][0] += p[0] + p[2];
-                lsum[nt][1] += p[1] + p[3];
-                // p = hi + lo in 16-bit pairs (token row, heads 2t/2t+1), then
-                // transposed to (head row, tokens 2t/2t+1): the B fragment of P^T
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const uint32_t hi = Ops::pack(p[2 * half], p[2 * half + 1]);
-                    const float2 hv = Tag::widen2(hi);
-                    const uint32_t lo = Ops::pack(p[2 * half] - hv.x, p[2 * half + 1] - hv.y);
-                    bhi[nt][half] = movmatrix_trans(hi);
-                    blo[nt][half] = movmatrix_trans(lo);
-                }
-            }
-            // Rows past the sequence end may hold anything (NaN included): their
-            // p is 0, but 0 * NaN is NaN inside the MMA, so their V^T entries are
-            // zeroed in the fragment (lane holds tokens 2t, 2t+1 and 2t+8, 2t+9).
-            const uint32_t mask01 = (2 * t < nv ? 0x0000ffffu : 0u) | (2 * t + 1 < nv ? 0xffff0000u : 0u);
-            const uint32_t mask89 = (2 * t + 8 < nv ? 0x0000ffffu : 0u) | (2 * t + 9 < nv ? 0xffff0000u : 0u);
+            gqa_softmax_tile<Tag>(x, g, nv, sc, m, lsum, o, bhi, blo);
+            // V^T entries of tokens past the end are zeroed (lane: tokens 2t, 2t+1 and 2t+8, 2t+9)
+            const uint32_t mask01 = gqa_pair_mask(2 * t, nv), mask89 = gqa_pair_mask(2 * t + 8, nv);
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 uint32_t af[4];

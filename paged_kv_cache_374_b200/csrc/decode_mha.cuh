@@ -33,15 +33,18 @@ struct MhaPolicy {
     static constexpr int DUP = 4 / NROW;   // lanes that end up holding one token's score
     static constexpr int HALF_BYTES = TOK * 128;
 
-    // fp8 codes with fp16 q: q K^T as f32 += f16 * f16 (sm_100 mixed-precision fma) on
-    // the raw q pairs and the exactly widened codes; the scale is applied to the sum
-    static constexpr bool kMixed = CTag::kBytes == 1 && !Tag::kIsBF16;
+    // fp8 codes: q K^T as f32 += f16 * f16 (sm_100 mixed-precision fma) on f16 q pairs and
+    // the exactly widened codes; the scale is applied to the sum.  fp16 q enters as it is;
+    // bf16 q as f16 q * 2^k, with 2^k chosen per unit from its largest |q| (exact for every
+    // element above 2^-31 of that one) and 2^-k applied to the sum with the scale.
+    static constexpr bool kMixed = CTag::kBytes == 1;
 
     int lane, r, c;
     int swz[NCH];       // offset of this lane's chunk j of row r in a tile
     uint4 qn[DL / 8];   // raw q of the next unit
     float2 qc[DL / 2];  // q of the current unit, pre-scaled by scale * log2(e)
-    uint32_t qh[DL / 2];  // kMixed: raw q of the current unit as f16 pairs
+    uint32_t qh[DL / 2];  // kMixed: q of the current unit as f16 pairs (times 2^k for bf16 q)
+    float qinv;           // kMixed: 2^-k
     float m, lsum;
     float2 o[DL / 2];
     bool poisoned;
@@ -68,12 +71,40 @@ struct MhaPolicy {
 
     __device__ __forceinline__ void take_q(const DecodeArgs& a) {
         if constexpr (kMixed) {
+            if constexpr (Tag::kIsBF16) {
+                // lanes with the same c hold the same dims: the max over lane bits 3 and 4 covers the head
+                float mx = 0.f;
 #pragma unroll
-            for (int j = 0; j < DL / 8; ++j) {
-                qh[4 * j] = qn[j].x;
-                qh[4 * j + 1] = qn[j].y;
-                qh[4 * j + 2] = qn[j].z;
-                qh[4 * j + 3] = qn[j].w;
+                for (int j = 0; j < DL / 8; ++j) {
+                    const uint32_t w[4] = {qn[j].x, qn[j].y, qn[j].z, qn[j].w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 v = BF16Tag::widen2(w[k]);
+                        mx = fmaxf(mx, fmaxf(fabsf(v.x), fabsf(v.y)));
+                    }
+                }
+                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 16));
+                float s;
+                f16_entry_scale(mx, s, qinv);
+#pragma unroll
+                for (int j = 0; j < DL / 8; ++j) {
+                    const uint32_t w[4] = {qn[j].x, qn[j].y, qn[j].z, qn[j].w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 v = BF16Tag::widen2(w[k]);
+                        qh[4 * j + k] = pack_f16x2(v.x * s, v.y * s);
+                    }
+                }
+            } else {
+                qinv = 1.f;
+#pragma unroll
+                for (int j = 0; j < DL / 8; ++j) {
+                    qh[4 * j] = qn[j].x;
+                    qh[4 * j + 1] = qn[j].y;
+                    qh[4 * j + 2] = qn[j].z;
+                    qh[4 * j + 3] = qn[j].w;
+                }
             }
             return;
         }
@@ -124,6 +155,8 @@ struct MhaPolicy {
     __device__ __forceinline__ void stage(const DecodeArgs& a, const uint8_t* kt, const uint8_t* vt, int ntok) {
         // partial dot products of rows i*8 + r over this lane's dims
         float acc[NROW];
+        float sum_scale = 1.f;
+        if constexpr (kMixed) sum_scale = a.scale_log2 * a.k_scale * qinv;
 #pragma unroll
         for (int i = 0; i < NROW; ++i) {
             float2 d2 = make_float2(0.f, 0.f);
@@ -145,7 +178,7 @@ struct MhaPolicy {
                 }
             }
             acc[i] = d2.x + d2.y;
-            if constexpr (kMixed) acc[i] *= a.scale_log2 * a.k_scale;
+            if constexpr (kMixed) acc[i] *= sum_scale;
         }
         // reduce over the 4 lanes of a row (lane bits 4 and 3), scattering the
         // NROW rows so that lane c keeps row group g(c)

@@ -76,6 +76,24 @@ struct E4M3Tag {
     }
 };
 
+// Power-of-two scale that enters 16-bit values of a wider range (bf16) into f16
+// arithmetic: given their largest magnitude mx, s = 2^k brings it to [2^14, 2^15)
+// (k clamped so that s and 1/s are normal floats).  x * s is then exact in f16
+// for every |x| >= 2^-31 mx; smaller ones round to f16's subnormal grid.
+__device__ __forceinline__ void f16_entry_scale(float mx, float& s, float& s_inv) {
+    const int ebits = (int)((__float_as_uint(mx) >> 23) & 0xffu);
+    const int k = ebits == 0 ? 0 : max(-114, min(126, 141 - ebits));
+    s = __uint_as_float((uint32_t)(127 + k) << 23);
+    s_inv = __uint_as_float((uint32_t)(127 - k) << 23);
+}
+
+// (lo, hi) -> f16x2, lo in the low half
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
 // ------------------------------------------------------------------- error word
 
 __device__ __forceinline__ void report(int32_t* err_word, int bits) {

@@ -23,6 +23,12 @@
 #ifndef PA_DECODE_SLOTS
 #define PA_DECODE_SLOTS 2        // shared-memory slots per warp
 #endif
+#ifndef PA_FP8TC_WARPS
+#define PA_FP8TC_WARPS 12        // warps per CTA of the fp8 tensor-core engine (groups of up to 8)
+#endif
+#ifndef PA_FP8TC_SLOTS
+#define PA_FP8TC_SLOTS 2         // its 32-token slots per warp
+#endif
 #ifndef PA_DECODE_TOK128
 #define PA_DECODE_TOK128 16      // tokens per slot at head_dim 128
 #endif
@@ -252,22 +258,23 @@ int launch_decode(DecodeArgs args, const void* k_cache, const void* v_cache, int
 }
 
 // fp8 (E4M3) caches.  GQA groups of 2-16: tensor cores, one kv head with its whole
-// query group per unit (one fetch of the codes serves the group), codes widened
-// into per-warp 16-bit tiles.  MHA (and larger groups): CUDA cores, one
-// query head per unit, 32-token slots (8 KiB): with a single head the tensor-core
-// stage carries too little work per byte to keep up.
+// query group per unit (one fetch of the codes serves the group), codes converted
+// from the landed stage straight into MMA fragments.  MHA (and larger groups):
+// CUDA cores, one query head per unit: with a single head the tensor-core stage
+// carries too little work per byte to keep up.
 template <class Tag>
 int launch_decode_fp8(DecodeArgs args, const void* k_cache, const void* v_cache, int num_kv_heads,
                       cudaStream_t stream) {
-    // 32-token slots of codes (8 KiB) and a 16-token scratch pair (8 KiB): 8 warps keep
-    // 128 KiB of codes in flight per SM
+    // 32-token slots of codes (8 KiB for K and V).  Groups of up to 8 run 12 warps (192 KiB
+    // of codes in flight per SM, 166 registers); groups of 9-16 hold twice the accumulators
+    // (255 registers) and run 8 warps.
     constexpr int TOK = 32;
     if (args.group >= 2 && args.group <= PA_GQA_MAX_GROUP) {
         args.unit_heads = num_kv_heads;
         args.heads_per_unit = args.group;
         if (args.group <= 8)
-            return launch_engine<Tag, E4M3Tag, 128, TOK, 8, 2, Fp8TcPolicy<Tag, TOK, 1>>(args, k_cache, v_cache,
-                                                                                           num_kv_heads, stream);
+            return launch_engine<Tag, E4M3Tag, 128, TOK, PA_FP8TC_WARPS, PA_FP8TC_SLOTS, Fp8TcPolicy<Tag, TOK, 1>>(
+                args, k_cache, v_cache, num_kv_heads, stream);
         return launch_engine<Tag, E4M3Tag, 128, TOK, 8, 2, Fp8TcPolicy<Tag, TOK, 2>>(args, k_cache, v_cache,
                                                                                        num_kv_heads, stream);
     }

@@ -56,16 +56,20 @@ def test_profiled_traffic_comes_only_from_the_same_workload(tmp_path):
     same workload (bytes per token depend on the head counts) and the sources its
     kernels are built from are the ones it was taken on."""
     import bench
-    per_token_7b = 629657088 / 37801
-    assert bench.profiled_traffic(1000, "llama7b") == pytest.approx(1000 * per_token_7b)
-    assert bench.profiled_traffic(1000, "llama13b") is None
-    assert bench.profiled_traffic(1000, "gqa70b", bench.GQA_PROFILE_SUMMARY) == pytest.approx(
-        1000 * 203340544 / 47015)
-    assert bench.profiled_traffic(1000, "gqa70b") is None           # the 7B capture does not serve gqa70b
-    assert bench.profiled_traffic(1000, "beam", bench.SHARED_PROFILE_SUMMARY) is not None
-    # a summary whose recorded digest no longer matches its sources gives no traffic
-    stale = tmp_path / "stale.md"
     text = open(bench.PROFILE_SUMMARY).read()
-    line = next(ln for ln in text.splitlines() if ln.startswith("- source_sha256_16: "))
-    stale.write_text(text.replace(line, "- source_sha256_16: 0000000000000000"))
-    assert bench.profiled_traffic(1000, "llama7b", str(stale)) is None
+    fields = dict(ln[2:].split(": ", 1) for ln in text.splitlines() if ln.startswith("- ") and ": " in ln)
+    sources = [os.path.join(bench.ROOT, "paged_kv_cache_374_b200", "csrc", n.strip())
+               for n in fields["sources"].split(",")]
+    old = "- source_sha256_16: " + fields["source_sha256_16"]
+
+    def summary(name, sha):
+        f = tmp_path / name
+        f.write_text(text.replace(old, "- source_sha256_16: " + sha))
+        return str(f)
+
+    current = summary("current.md", bench.source_digest(sources))
+    per_token = int(fields["dram_bytes_per_launch"]) / int(fields["tokens_per_launch"])
+    assert bench.profiled_traffic(1000, fields["workload"], current) == pytest.approx(1000 * per_token)
+    assert bench.profiled_traffic(1000, "gqa70b", current) is None      # another workload's capture
+    assert bench.profiled_traffic(1000, fields["workload"], summary("stale.md", "0" * 16)) is None
+    assert bench.profiled_traffic(1000, fields["workload"], str(tmp_path / "missing.md")) is None
