@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from gpu_cases import Step, assert_close, bits
-from pins import BF16, F16, PagedCase, from_bits
+from pins import BF16, F16, PagedCase, from_bits, to_bits
 import oracle as oracle_pkg
 from paged_kv_cache_374_b200 import binding as pa
 
@@ -108,3 +108,33 @@ def test_llama7b_fp8_full_size():
                        nthreads=8)
     got = out[torch.from_numpy(pairs[:, 0]).long(), torch.from_numpy(pairs[:, 1]).long()]
     assert_close(got, ref, "f16", "llama7b fp8")
+
+
+@pytest.mark.parametrize("g", [1, 8])
+@pytest.mark.parametrize("exp2", [40, -40])
+def test_decode_fp8_bf16_q_outside_f16_range(g, exp2):
+    """bf16 q enters the f16 arithmetic of both fp8 policies as q * 2^k, k chosen per
+    unit: q scaled by 2^40 (past f16's largest finite value) or 2^-40 (below its
+    smallest subnormal), with the softmax scale compensating so that the scores stay
+    in the usual range, must give the oracle's result.  One head also holds elements
+    about 2^30 below its largest: the unit's scale keeps them (the few under 2^-31 of
+    the largest round to f16's subnormal grid, a negligible change of the score)."""
+    rng = np.random.default_rng(53 + g + exp2)
+    hk, d, bs = 2, 128, 16
+    lens = [1, 17, 300, 777]
+    c = PagedCase(rng, lens, hk * g, hk, d, bs, BF16, 1 / math.sqrt(d), extra_blocks=2)
+    q64 = from_bits(c.q, BF16) * 2.0 ** exp2
+    q64[1, 0, 64:] *= 2.0 ** -30                      # one head: dims 64.. far below the head's largest
+    q_bits = to_bits(q64, BF16)
+    assert np.array_equal(from_bits(q_bits, BF16), q64)   # the scaling is exact in bf16
+    scale = c.scale * 2.0 ** -exp2
+    ks, vs = 0.08, 0.05
+    k8 = to_codes(from_bits(c.k_cache, BF16), ks)
+    v8 = to_codes(from_bits(c.v_cache, BF16), vs)
+    ref = oracle_pkg.get().decode_fp8(q_bits, k8, v8, c.tables, c.lens, scale, ks, vs, BF16, nthreads=8)
+    q = torch.from_numpy(q_bits.view(np.int16)).view(torch.bfloat16).cuda()
+    out = torch.empty_like(q)
+    pa.pa_decode_fp8(q, torch.from_numpy(k8).cuda(), torch.from_numpy(v8).cuda(), torch.from_numpy(c.tables).cuda(),
+                     torch.from_numpy(c.lens).cuda(), scale, ks, vs, hk, out)
+    torch.cuda.synchronize()
+    assert_close(out, ref, "bf16", f"fp8 bf16 q x 2^{exp2} g{g}")
