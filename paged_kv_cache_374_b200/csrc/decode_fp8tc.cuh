@@ -8,17 +8,18 @@
 // f16 with fp32 accumulation whatever q's type:
 //   S^T[16 tok x 8 heads] = K[16 tok x 128] . Q^T[128 x 8 heads]
 //   O^T[128 x 8 heads]   += V^T[128 x 16 tok] . P^T[16 tok x 8 heads]
-// A contraction may visit its k index in any order, so both products permute it
-// to suit 16-byte shared loads that hit every bank once:
-//   q K^T: lane (g, t) takes code bytes 32t .. 32t+31 of token rows g and g+8;
+// Each product permutes one index whose order is free, so that its fragments come
+// from 16-byte shared loads that hit every bank once per quarter warp:
+//   q K^T: the reduction index (a contraction may visit it in any order).  Lane
+//          (g, t) takes code bytes 32t .. 32t+31 of token rows g and g+8;
 //          k-step ks covers dims 32t' + 4ks + {0,1} as k = 2t', 2t'+1 and
 //          32t' + 4ks + {2,3} as k = 2t'+8, 2t'+9 (t' = 0..3), and q^T's B
 //          fragment is loaded in the same order.
-//   V^T P^T: the M index (dims) is permuted instead: m-tile mt holds dims
-//          16g + 2mt (row g) and 16g + 2mt + 1 (row g+8), so lane (g, t) reads
-//          16-byte chunk g of token rows 2t, 2t+1, 2t+8, 2t+9 and transposes
-//          bytes in registers (prmt) into the (dim, token pair) fragments; the
-//          output rows are written back to their dims at the end.
+//   V^T P^T: the M index (the output dims, put back in order when written).
+//          m-tile mt holds dims 16g + 2mt (row g) and 16g + 2mt + 1 (row g+8),
+//          so lane (g, t) reads 16-byte chunk g of token rows 2t, 2t+1, 2t+8,
+//          2t+9 and transposes bytes in registers (prmt) into the (dim, token
+//          pair) fragments.
 // q of a bf16 model enters as f16 scaled by a power of two 2^k that brings the
 // group's largest |q| to [2^14, 2^15); the scale is undone on the scores.  This
 // is exact except for elements below 2^-31 of that largest one, which round to
@@ -150,9 +151,12 @@ struct Fp8TcPolicy {
             const uint4 k1b = lds128(kr + (g + 8) * 128 + (((2 * t + 1) ^ g) << 4));
             const uint32_t kw0[8] = {k0a.x, k0a.y, k0a.z, k0a.w, k0b.x, k0b.y, k0b.z, k0b.w};  // token g
             const uint32_t kw1[8] = {k1a.x, k1a.y, k1a.z, k1a.w, k1b.x, k1b.y, k1b.z, k1b.w};  // token g+8
-            float x[NT][4];
+            // two accumulators (even and odd k-steps) halve the chain of dependent MMAs
+            float x[NT][4], y[NT][4];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) x[nt][0] = x[nt][1] = x[nt][2] = x[nt][3] = 0.f;
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) x[nt][j] = y[nt][j] = 0.f;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
                 uint32_t af[4];
@@ -161,8 +165,12 @@ struct Fp8TcPolicy {
                 af[2] = e4m3x2_to_f16x2(kw0[ks] >> 16);      // token g,   dims 32t + 4ks + 2, +3
                 af[3] = e4m3x2_to_f16x2(kw1[ks] >> 16);      // token g+8
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) Ops::mma(x[nt], af, qb[nt][ks][0], qb[nt][ks][1]);
+                for (int nt = 0; nt < NT; ++nt) Ops::mma((ks & 1) ? y[nt] : x[nt], af, qb[nt][ks][0], qb[nt][ks][1]);
             }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) x[nt][j] += y[nt][j];
             uint32_t bhi[NT][2], blo[NT][2];
             gqa_softmax_tile<F16Tag>(x, g, nv, sc, m, lsum, o, bhi, blo);
 
