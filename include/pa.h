@@ -275,10 +275,15 @@ int pa_reshape_and_cache_fp8(const void* k, const void* v, const int64_t* slot_m
 
 /*
  * pa_decode_fp8 -- pa_decode over fp8 caches: the same softmax(scale * q K^T) V
- * with K = code * k_scale and V = code * v_scale, in fp32 (the codes widen
- * exactly; k_scale is folded into q, v_scale into the result).  head_dim 128 only;
- * every other argument, the workspace and the errors as pa_decode.  Query heads
- * are computed on CUDA cores one per unit (a GQA group shares its K/V through L2).
+ * with K = code * k_scale and V = code * v_scale.  The codes widen exactly to f16;
+ * q K^T is accumulated in fp32 from exact f16 x f16 products and scaled by
+ * scale * k_scale afterwards, and v_scale multiplies the result.  fp16 q enters
+ * as it is; bf16 q as q * 2^k in f16, with 2^k chosen per unit from its largest
+ * |q| (exact for every element above 2^-31 of that one; smaller ones round to
+ * f16's subnormal grid) and undone on the scores.  GQA groups of 2-16 share each
+ * K/V fetch and run both products on tensor cores (P^T as a 16-bit hi + lo pair);
+ * MHA and larger groups run on CUDA cores, one query head per unit.  head_dim 128
+ * only; every other argument, the workspace and the errors as pa_decode.
  */
 int pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
                   const int32_t* context_lens, float scale, float k_scale, float v_scale, int num_kv_heads, void* out,
