@@ -5,7 +5,7 @@ import os
 
 import pytest
 
-from oracle.block_pool import BlockPoolModel, ManagerModel, OutOfBlocks, RefcountError
+from oracle.block_pool import BlockPoolModel, ManagerModel, OutOfBlocks, RefcountError, swap_plan
 from pins import GOLDEN
 
 
@@ -83,3 +83,96 @@ def test_copy_on_write_is_all_or_nothing():
     with pytest.raises(OutOfBlocks):
         m.cow_prepare({0: 20, 1: 20, 2: 20, 3: 20})   # needs 3 copies, 2 free
     assert m.pool.num_free() == 2 and m.pool.ref[m.tables[0][1]] == 4
+
+
+# ---------------------------------------------------------------- swap plan
+#
+# Preemption (P3 §三, append_slot's "Preemption required") sends a sequence's KV
+# blocks to host memory and P3 §五 brings them back.  The trace below was worked
+# out by hand from the pool rules (FIFO front allocation, back-of-queue return at
+# count zero, all-or-nothing):
+#
+#   device pool, 6 blocks, free queue 4 1 5 0 3 2; host pool, 4 blocks, queue 2 0 3 1
+#   request A allocates 3 blocks -> row [4, 1, 5], device queue 0 3 2
+#   request B holds A's first block by reference (a shared prefix) -> ref[4] = 2
+#   swap A out: host allocates 2, 0, 3 in row order; device drops one reference
+#     of 4 (2 -> 1, still held by B, stays out of the queue), 1 and 5 (-> 0, to the
+#     back of the queue in row order): pairs (4,2) (1,0) (5,3), row [2, 0, 3],
+#     device queue 0 3 2 1 5, host queue 1
+#   swap A back in: device allocates from the front 0, 3, 2 (never 4, which B still
+#     holds); host frees 2, 0, 3 to its back: pairs (2,0) (0,3) (3,2), row [0, 3, 2],
+#     device queue 1 5, host queue 1 2 0 3
+
+def _swap_trace(plan):
+    """Run the hand-traced swap-out / swap-in through ``plan`` (a swap_plan with the
+    model's signature) and assert every value of the trace; then the two refusals:
+    a row holding a block more often than its count allows, and a target pool
+    too small -- each must leave both pools and the row exactly as they were."""
+    dev = BlockPoolModel(6, initial_order=[4, 1, 5, 0, 3, 2])
+    host = BlockPoolModel(4, initial_order=[2, 0, 3, 1])
+    row = dev.allocate_n(3)
+    assert row == [4, 1, 5]
+    dev.add_ref(4)                                   # request B shares the first block
+    pairs = plan(dev, host, row)
+    assert [tuple(p) for p in pairs] == [(4, 2), (1, 0), (5, 3)]
+    assert row == [2, 0, 3]
+    assert [dev.ref[b] for b in range(6)] == [0, 0, 0, 0, 1, 0]
+    assert list(dev.free_queue) == [0, 3, 2, 1, 5]
+    assert [host.ref[b] for b in range(4)] == [1, 0, 1, 1]
+    assert list(host.free_queue) == [1]
+    assert dev.usage_ratio() == 1 / 6 and host.usage_ratio() == 3 / 4
+    pairs = plan(host, dev, row)
+    assert [tuple(p) for p in pairs] == [(2, 0), (0, 3), (3, 2)]
+    assert row == [0, 3, 2]
+    assert [dev.ref[b] for b in range(6)] == [1, 0, 1, 1, 1, 0]
+    assert list(dev.free_queue) == [1, 5]
+    assert [host.ref[b] for b in range(4)] == [0, 0, 0, 0]
+    assert list(host.free_queue) == [1, 2, 0, 3]
+
+    # refusals change nothing
+    def snapshot():
+        return (list(dev.ref), list(dev.free_queue), dev.allocated, list(host.ref), list(host.free_queue),
+                host.allocated)
+    before, twice = snapshot(), [0, 0, 3]            # block 0 listed twice, held once
+    with pytest.raises(RefcountError):
+        plan(dev, host, twice)
+    assert snapshot() == before and twice == [0, 0, 3]
+    big = BlockPoolModel(6, initial_order=[0, 1, 2, 3, 4, 5])
+    grown = big.allocate_n(5)                        # host pool has 4 free: too few
+    host_before, big_before = snapshot(), (list(big.ref), list(big.free_queue))
+    with pytest.raises(OutOfBlocks):
+        plan(big, host, grown)
+    assert snapshot() == host_before and (list(big.ref), list(big.free_queue)) == big_before
+    assert grown == [0, 1, 2, 3, 4]
+
+
+def test_swap_plan_hand_traced():
+    _swap_trace(swap_plan)
+
+
+# Planted mistakes in the model's swap_plan (its own source with one line changed,
+# compiled on the CPU): each must fail the hand-traced pin above.
+SWAP_MUTANTS = {
+    "row not rewritten": ("table[i] = fresh", "pass"),
+    "source reference not dropped": ("src.free(b)", "pass"),
+    "pair reversed": ("pairs.append((b, fresh))", "pairs.append((fresh, b))"),
+    "held-count check dropped": ("if src.ref[b] < held[b]:", "if False:"),
+    "not all or nothing": ("if dst.num_free() < len(table):", "if False:"),
+    "target taken from the back": ("fresh = dst.allocate()", "fresh = dst.free_queue.pop(); dst.ref[fresh] = 1; "
+                                                              "dst.allocated += 1"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SWAP_MUTANTS))
+def test_swap_plan_pin_catches_planted_mistake(name):
+    import inspect
+    import textwrap
+
+    import oracle.block_pool as bp
+    old, new = SWAP_MUTANTS[name]
+    src = textwrap.dedent(inspect.getsource(bp.swap_plan))
+    assert src.count(old) == 1, f"mutation site for {name!r} not found"
+    scope = dict(vars(bp))
+    exec(compile(src.replace(old, new), "<swap_plan mutant>", "exec"), scope)
+    with pytest.raises((AssertionError, OutOfBlocks, RefcountError, IndexError)):
+        _swap_trace(scope["swap_plan"])
