@@ -8,6 +8,11 @@ Tolerances (stated on the decode output against the fp64 oracle):
         once to bf16.  Rounding the exact result to bf16 alone has a relative L2
         of about 1.5e-3 (half an ulp of 2^-7, uniform), so the 1e-3 bound can only
         apply to the error beyond that unavoidable final rounding.
+  The max |err| bounds apply to the computation before that one final rounding:
+  element i may differ from the unrounded oracle by the bound plus half an ulp of
+  the output type at ref_i.  Rounding alone reaches half an ulp, which is above
+  1e-2 in bf16 from |out| = 4 on (and above 2e-3 in fp16 from 8 on), where a
+  peaked softmax puts outputs with N(0, 1) values.
   cache writes: bit-exact.
 """
 from __future__ import annotations
@@ -32,12 +37,20 @@ def bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
+def half_ulp(ref: np.ndarray, dtype: str) -> np.ndarray:
+    """Half the spacing of the output type's numbers at |ref| (normal range)."""
+    mant = 10 if dtype == wk.F16 else 7
+    e = np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -14)))
+    return 0.5 * np.exp2(e - mant)
+
+
 def errors(got: torch.Tensor, ref: np.ndarray, dtype: str):
+    """(max |err| beyond half an ulp of the output type, relative L2)."""
     g = got.detach().double().cpu().numpy()
     r_target = ref
     if dtype == wk.BF16:
         r_target = torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
-    max_abs = float(np.max(np.abs(g - ref))) if g.size else 0.0
+    max_abs = float(np.max(np.abs(g - ref) - half_ulp(ref, dtype))) if g.size else 0.0
     den = float(np.linalg.norm(r_target))
     rel = float(np.linalg.norm(g - r_target) / den) if den > 0 else float(np.linalg.norm(g - r_target))
     return max_abs, rel
@@ -47,7 +60,8 @@ def assert_close(got: torch.Tensor, ref: np.ndarray, dtype: str, what=""):
     assert not torch.isnan(got).any(), f"{what}: NaN in output"
     max_abs, rel = errors(got, ref, dtype)
     tol_abs, tol_rel = TOL[dtype]
-    assert max_abs <= tol_abs and rel <= tol_rel, f"{what}: max_abs {max_abs:.3g} rel_l2 {rel:.3g}"
+    assert max_abs <= tol_abs and rel <= tol_rel, (
+        f"{what}: max_abs beyond the final rounding {max_abs:.3g} rel_l2 {rel:.3g}")
     return max_abs, rel
 
 

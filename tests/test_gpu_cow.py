@@ -91,3 +91,45 @@ def test_copy_blocks_bad_ids_and_bit_exactness():
         assert oracle_pkg.get().copy_blocks(kh, vh, pairs) == 1
         assert err.item() == pa.PA_DEVERR_TABLE_RANGE
         assert np.array_equal(bits(kc), kh) and np.array_equal(bits(vc), vh)
+
+
+def test_copy_blocks_refuses_overlapping_pairs():
+    """The pairs are copied all at once, so pairs that overlap are skipped with
+    PA_DEVERR_PAIR_CONFLICT instead of being copied in some order: a chain
+    (1->2, 2->3), two pairs into one block (8->9, 10->9), and a destination that is
+    another pair's source (4->12, 12->13).  Pairs that share a source (5->6, 5->7),
+    a pair onto itself and the pairs beside them are copied; an id out of range is
+    skipped with PA_DEVERR_TABLE_RANGE and conflicts with nothing.  The result is
+    the oracle's sequential copy of the non-overlapping pairs alone."""
+    nb, bs, hk, d = 16, 16, 4, 128
+    kc = torch.randn(nb, bs, hk, d, device="cuda").to(torch.float16)
+    vc = torch.randn(nb, bs, hk, d, device="cuda").to(torch.float16)
+    kh, vh = bits(kc), bits(vc)
+    pairs = np.array([[1, 2], [2, 3], [5, 6], [8, 9], [10, 9], [5, 7], [11, 11], [4, 12], [12, 13], [0, 15],
+                      [14, nb + 1]], dtype=np.int32)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_copy_blocks(kc, vc, torch.from_numpy(pairs).cuda(), err_word=err)
+    torch.cuda.synchronize()
+    assert err.item() == pa.PA_DEVERR_PAIR_CONFLICT | pa.PA_DEVERR_TABLE_RANGE
+    oracle_pkg.get().copy_blocks(kh, vh, np.array([[5, 6], [5, 7], [11, 11], [0, 15]], dtype=np.int32))
+    assert np.array_equal(bits(kc), kh) and np.array_equal(bits(vc), vh)
+
+
+@pytest.mark.parametrize("num_pairs,bs,hk,d", [(3, 64, 5, 64), (701, 16, 2, 128)])
+def test_copy_blocks_slices_and_many_pairs(num_pairs, bs, hk, d):
+    """A few large blocks, each spread over several CTAs' slices, and many small
+    ones, several to a slice; in both cases slices start inside a block.
+    Bit-exact against the oracle."""
+    rng = np.random.default_rng(46 + num_pairs)
+    nb = 2 * num_pairs + 5
+    kc = torch.randn(nb, bs, hk, d, device="cuda").to(torch.bfloat16)
+    vc = torch.randn(nb, bs, hk, d, device="cuda").to(torch.bfloat16)
+    kh, vh = bits(kc), bits(vc)
+    perm = rng.permutation(nb).astype(np.int32)
+    pairs = np.stack([perm[:num_pairs], perm[num_pairs:2 * num_pairs]], axis=1).copy()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_copy_blocks(kc, vc, torch.from_numpy(pairs).cuda(), err_word=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    oracle_pkg.get().copy_blocks(kh, vh, pairs)
+    assert np.array_equal(bits(kc), kh) and np.array_equal(bits(vc), vh)

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 from gpu_cases import assert_close, bits
-from pins import BF16, F16, PagedCase, to_bits
+from pins import BF16, F16, PagedCase, from_bits, to_bits
 import oracle as oracle_pkg
 from paged_kv_cache_374_b200 import binding as pa
 
@@ -115,3 +115,149 @@ def test_prefill_bad_entries_give_nan_rows():
     ref = oracle_pkg.get().prefill(q[:40].copy(), c.k_cache, c.v_cache, c.tables[:1].copy(), c.lens[:1].copy(),
                                    qs[:2].copy(), c.scale, F16)
     assert_close(out[:40], ref, "f16", "unaffected sequence")
+
+
+# ------------------------------------------------- large logits: the rescale path
+#
+# The kernel keeps the running max it exponentiates against until a row's tile max
+# grows past it by more than 2^8 (in log2 units), then rescales O and the row sum
+# in tensor memory.  N(0,1) inputs at scale 1/sqrt(d) never get there after the
+# first tile, so these cases make the scores grow along the sequence: keys scaled
+# by (1 + t / 24) at position t, or a large scale.  rescale_events() counts, from
+# fp64 scores on the host, the (row, head) pairs that must take that path, so each
+# case shows it is reached.
+
+LOG2E = 1.4426950408889634
+
+
+def ramp_keys(c, rate=24.0):
+    """Scale every sequence's key at position t by (1 + t / rate)."""
+    for s in range(c.S):
+        k = from_bits(c.seq_k[s], c.dtype)
+        k *= (1.0 + np.arange(k.shape[0]) / rate)[:, None, None]
+        c.seq_k[s] = to_bits(k, c.dtype)
+    c._assemble()
+
+
+def _events(x_row, t_lo, t_hi):
+    """Rescales of one row over tokens [t_lo, t_hi), walked in 64-token tiles."""
+    m, n = None, 0
+    for t0 in range(t_lo, t_hi, 64):
+        mt = float(np.max(x_row[t0:min(t0 + 64, t_hi)]))
+        if m is None:
+            m = mt
+        elif mt > m + 8.0:
+            n, m = n + 1, mt
+    return n
+
+
+def rescale_events(c, q_bits, qs):
+    q = from_bits(q_bits, c.dtype)
+    g = c.H // c.Hk
+    total = 0
+    for s in range(c.S):
+        n, L = int(qs[s + 1] - qs[s]), int(c.lens[s])
+        k = from_bits(c.seq_k[s], c.dtype)
+        for h in range(c.H):
+            x = q[qs[s]:qs[s + 1], h] @ k[:, h // g].T * (c.scale * LOG2E)
+            total += sum(_events(x[i], 0, L - n + i + 1) for i in range(n))
+    return total
+
+
+LARGE = [(128, 16, 1, F16, "ramp"), (128, 32, 4, BF16, "ramp"), (64, 64, 2, BF16, "ramp"),
+         (128, 16, 1, F16, "scale"), (64, 32, 2, BF16, "scale")]
+
+
+@pytest.mark.parametrize("d,bs,g,dtype,kind", LARGE)
+def test_prefill_large_logits_take_the_rescale_path(d, bs, g, dtype, kind):
+    rng = np.random.default_rng(63 + d + bs + g)
+    hk = 2
+    lens = [37, 200, 64, 513, 9]
+    n_new = [37, 70, 1, 200, 9]
+    scale = 2.0 if kind == "scale" else 1 / math.sqrt(d)
+    c = PagedCase(rng, lens, hk * g, hk, d, bs, dtype, scale, extra_blocks=3)
+    if kind == "ramp":
+        ramp_keys(c)
+    qs = np.concatenate([[0], np.cumsum(n_new)]).astype(np.int32)
+    q = to_bits(rng.normal(0, 1, (int(qs[-1]), hk * g, d)), dtype)
+    assert rescale_events(c, q, qs) >= 100
+    ref = oracle_pkg.get().prefill(q, c.k_cache, c.v_cache, c.tables, c.lens, qs, c.scale, dtype, nthreads=8)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = run_prefill(c, q, qs, err=err)
+    assert err.item() == 0
+    assert_close(out, ref, WK[dtype], f"large logits ({kind}) d{d} bs{bs} g{g}")
+
+
+@pytest.mark.parametrize("dtype,kind", [(F16, "ramp"), (BF16, "ramp"), (BF16, "scale")])
+def test_shared_prefix_large_logits_take_the_rescale_path(dtype, kind):
+    """The same kernel in its shared-prefix mode (pa_decode_shared_prefix): each CTA
+    walks one 256-token partition of the shared prefix in four tiles with no mask."""
+    rng = np.random.default_rng(64)
+    d, bs, hk, g, P = 128, 32, 2, 4, 256
+    scale = 2.0 if kind == "scale" else 1 / math.sqrt(d)
+    c = PagedCase(rng, [700, 650, 600, 520, 300, 513], hk * g, hk, d, bs, dtype, scale, extra_blocks=4)
+    if kind == "ramp":
+        ramp_keys(c)
+    members = [0, 1, 2, 3]
+    nb = 512 // bs
+    for s in members[1:]:
+        c.tables[s, :nb] = c.tables[0, :nb]
+        c.seq_k[s][:512] = c.seq_k[0][:512]
+        c.seq_v[s][:512] = c.seq_v[0][:512]
+    c._assemble()
+    grp = pa.pa_find_shared_prefixes(c.tables, c.lens, c.bs, P)
+    assert grp.num_groups == 1 and grp.max_shared_tokens == 512
+    q = from_bits(c.q, dtype)
+    k0 = from_bits(c.seq_k[0], dtype)
+    events = sum(_events(q[s, h] @ k0[:, h // g].T * (c.scale * LOG2E), p * P, (p + 1) * P)
+                 for s in members for h in range(hk * g) for p in range(2))
+    assert events >= 8
+    qd = torch.from_numpy(np.ascontiguousarray(c.q).view(np.int16)).view(TDT[dtype]).cuda()
+    out = torch.empty_like(qd)
+    start, offs, mem = grp.to("cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_decode_shared_prefix(qd, dev(c.k_cache, dtype), dev(c.v_cache, dtype), torch.from_numpy(c.tables).cuda(),
+                               torch.from_numpy(c.lens).cuda(), c.scale, hk, out, start, offs, mem, grp.num_groups,
+                               grp.max_group_size, grp.max_shared_tokens, partition_tokens=P, err_word=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    ref = oracle_pkg.get().decode(c.q, c.k_cache, c.v_cache, c.tables, c.lens, c.scale, dtype, nthreads=8)
+    assert_close(out, ref, WK[dtype], f"shared prefix, large logits ({kind})")
+
+
+# --------------------------------------------------------- the benchmarked size
+
+def test_prefill_at_bench_size_on_sampled_rows():
+    """8 whole 2048-token prompts at the 7B layer shape (32 heads, head_dim 128,
+    block size 16, fp16): the configuration the prefill benchmark times.  Checked
+    on sampled query rows -- the first two and the last of every 128-row tile, plus
+    random ones, every head -- each against the oracle's decode of that row over its
+    visible prefix (a query row at position p attends exactly as a decode over
+    p + 1 tokens does)."""
+    s, chunk, h, d, bs = 8, 2048, 32, 128, 16
+    nblk = chunk // bs
+    nb = s * nblk + 8
+    g = torch.Generator(device="cuda").manual_seed(65)
+    kc = torch.randn(nb, bs, h, d, generator=g, device="cuda").to(torch.float16)
+    vc = torch.randn(nb, bs, h, d, generator=g, device="cuda").to(torch.float16)
+    perm = torch.randperm(nb, generator=torch.Generator().manual_seed(66))[: s * nblk]
+    tables = perm.view(s, nblk).to(torch.int32).numpy().copy()
+    lens = np.full(s, chunk, dtype=np.int32)
+    qs = (np.arange(s + 1) * chunk).astype(np.int32)
+    q = torch.randn(s * chunk, h, d, generator=g, device="cuda").to(torch.float16)
+    out = torch.empty_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_prefill(q, kc, vc, torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda(),
+                  torch.from_numpy(qs).cuda(), 1 / math.sqrt(d), h, out, chunk, err_word=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    rng = np.random.default_rng(67)
+    rows = sorted({0, 1} | {t * 128 + 127 for t in range(chunk // 128)} | set(rng.integers(0, chunk, 6).tolist()))
+    seq_of = np.repeat(np.arange(s), len(rows))
+    pos = np.tile(np.array(rows), s)
+    q_rows = bits(q.view(s, chunk, h, d)[torch.from_numpy(seq_of).long(), torch.from_numpy(pos).long()])
+    ref = oracle_pkg.get().decode(np.ascontiguousarray(q_rows), bits(kc), bits(vc),
+                                  np.ascontiguousarray(tables[seq_of]), (pos + 1).astype(np.int32),
+                                  1 / math.sqrt(d), F16, nthreads=8)
+    got = out.view(s, chunk, h, d)[torch.from_numpy(seq_of).long(), torch.from_numpy(pos).long()]
+    assert_close(got, ref, "f16", "prefill 8 x 2048, sampled rows")

@@ -158,3 +158,35 @@ def test_launch_bounds_too_small_are_reported():
                                    g.num_groups, mg, mt, partition_tokens=64, err_word=err)
         torch.cuda.synchronize()
         assert bool(err.item() & pa.PA_DEVERR_LEN_RANGE) == (mt < 256)
+
+
+@pytest.mark.parametrize("bad", ["member", "end_past_batch", "end_before_start"])
+def test_group_arrays_out_of_range_are_skipped(bad):
+    """group_offsets and group_members come from the caller.  A group whose
+    offsets leave [0, num_seqs] or run backwards, or that lists a member outside
+    the batch, is skipped whole with PA_DEVERR_GROUP_RANGE (no access outside the
+    arrays the caller passed); every sequence outside it still gets the oracle's
+    result."""
+    rng = np.random.default_rng(76)
+    c = PagedCase(rng, [300, 280, 290, 200, 210, 150], 8, 8, 128, 16, F16, 1 / math.sqrt(128))
+    share(c, [0, 1, 2], 256)
+    share(c, [3, 4], 192)
+    start = np.array([256, 256, 256, 192, 192, 0], dtype=np.int32)
+    offs = np.array([0, 3, 5], dtype=np.int32)
+    members = np.array([0, 1, 2, 3, 4], dtype=np.int32)
+    if bad == "member":
+        members[4] = 1 << 20
+    elif bad == "end_past_batch":
+        offs[2] = 6 + 9
+        members = np.concatenate([members, np.zeros(16, dtype=np.int32)])  # the array is long enough; offsets are not
+    else:
+        offs[2] = 2
+    grp = pa.SharedPrefixes(start, offs, members, 2, 3, 256)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, _, _ = run_both(c, 64, err=err, groups=grp)
+    assert err.item() == pa.PA_DEVERR_GROUP_RANGE
+    keep = [0, 1, 2, 5]
+    pairs = np.array([(s, h) for s in keep for h in range(8)], dtype=np.int32)
+    ref = oracle_pkg.get().decode(c.q, c.k_cache, c.v_cache, c.tables, c.lens, c.scale, F16, pairs=pairs)
+    got = out[torch.from_numpy(pairs[:, 0]).long(), torch.from_numpy(pairs[:, 1]).long()]
+    assert_close(got, ref, "f16", f"groups beside a bad one ({bad})")
