@@ -62,6 +62,8 @@ def parse():
                         "pa_decode_shared_prefix; off: plain pa_decode")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--no-detail-workloads", action="store_true",
+                   help="skip the 13B append loop, gqa70b and beam entries of detail.workloads")
     p.add_argument("--row", default="decode", choices=["decode", "copy_blocks", "swap", "prefill"],
                    help="decode: the hot path (default); copy_blocks: copy-on-write block copies alone; "
                         "swap: swap-out / swap-in of blocks to pinned host memory")
@@ -258,12 +260,13 @@ def build_step(name, device, partition_tokens, num_seqs=None, kv_dtype="native",
     return d
 
 
-def algorithmic_bytes(st):
+def algorithmic_bytes(st, lens=None):
     """Bytes K2+K3 must move per step: every sequence's K and V rows once (shared
     prefix blocks once), q in and out back, the table entries read, the lengths,
-    and the partials written by K2 and read by K3."""
-    spec, wl = st["spec"], st["wl"]
-    lens = st["lens_h"].astype(np.int64)
+    and the partials written by K2 and read by K3.  ``lens``: the step's context
+    lengths (default: the step the workload was built for)."""
+    spec = st["spec"]
+    lens = (st["lens_h"] if lens is None else lens).astype(np.int64)
     e = 2                                  # q and out elements
     ec = st["k_cache"].element_size()      # cache elements (1 for fp8 codes)
     hk, d, h, s, bs = spec.num_kv_heads, spec.head_dim, spec.num_heads, spec.num_seqs, spec.block_size
@@ -273,8 +276,7 @@ def algorithmic_bytes(st):
     else:
         unique_tokens = int(np.sum(lens))
     logical_tokens = int(np.sum(lens))
-    from paged_kv_cache_374_b200 import binding as pa
-    ptok = st["partition_tokens"] or pa.pa_decode_partition_tokens(s, h, hk, d, bs, wl.max_blocks_per_seq)
+    ptok = st["ptok"]
     nparts = np.where(lens > ptok, -(-lens // ptok), 0)
     partials = int(np.sum(nparts)) * h * (d + 2) * 4 * 2
     meta = int(np.sum(-(-lens // bs))) * 4 + 4 * s
@@ -301,32 +303,24 @@ def static_config(wl, args, world):
 
 # --------------------------------------------------------------- native arm
 
-def run_native(args):
-    import torch
-    import torch.distributed as dist
-    from paged_kv_cache_374_b200 import binding as pa
+class Ops:
+    """K1 and K2+K3 of one built workload, through the binding, on one stream."""
 
-    rank, world, local = dist_env()
-    if world > 1:
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
-                                timeout=__import__("datetime").timedelta(seconds=120))
-    device = torch.device("cuda", local if world > 1 else 0)
-    torch.cuda.set_device(device)
-    st = build_step(args.workload, device, args.partition_tokens, args.num_seqs, args.kv_dtype,
-                    shared=args.shared_prefix == "auto")
-    fp8 = args.kv_dtype == "fp8"
-    ks = vs = 1.0 / FP8_INV_SCALE
-    spec = st["spec"]
-    stream = torch.cuda.current_stream(device)
+    def __init__(self, st, stream, fp8):
+        from paged_kv_cache_374_b200 import binding as pa
+        self.pa, self.st, self.stream, self.fp8 = pa, st, stream, fp8
+        self.ks = self.vs = 1.0 / FP8_INV_SCALE
 
-    def k1(k, v, slots):
-        if fp8:
-            pa.pa_reshape_and_cache_fp8(k, v, slots, st["k_cache"], st["v_cache"], ks, vs, stream=stream)
+    def k1(self, k, v, slots):
+        st, pa = self.st, self.pa
+        if self.fp8:
+            pa.pa_reshape_and_cache_fp8(k, v, slots, st["k_cache"], st["v_cache"], self.ks, self.vs,
+                                        stream=self.stream)
         else:
-            pa.pa_reshape_and_cache(k, v, slots, st["k_cache"], st["v_cache"], stream=stream)
+            pa.pa_reshape_and_cache(k, v, slots, st["k_cache"], st["v_cache"], stream=self.stream)
 
-    def k2(q, tables, lens, groups=None, out=None):
+    def k2(self, q, tables, lens, groups=None, out=None):
+        st, pa, spec = self.st, self.pa, self.st["spec"]
         g = st["groups"]
         out = st["out"] if out is None else out
         if g is not None:
@@ -334,62 +328,102 @@ def run_native(args):
             pa.pa_decode_shared_prefix(q, st["k_cache"], st["v_cache"], tables, lens, spec.scale, spec.num_kv_heads,
                                        out, start, offs, mem, g.num_groups, g.max_group_size,
                                        g.max_shared_tokens, workspace=st["workspace"],
-                                       partition_tokens=st["partition_tokens"], stream=stream)
-        elif fp8:
-            pa.pa_decode_fp8(q, st["k_cache"], st["v_cache"], tables, lens, spec.scale, ks, vs, spec.num_kv_heads,
-                             out, workspace=st["workspace"], partition_tokens=st["partition_tokens"],
-                             stream=stream)
+                                       partition_tokens=st["partition_tokens"], stream=self.stream)
+        elif self.fp8:
+            pa.pa_decode_fp8(q, st["k_cache"], st["v_cache"], tables, lens, spec.scale, self.ks, self.vs,
+                             spec.num_kv_heads, out, workspace=st["workspace"],
+                             partition_tokens=st["partition_tokens"], stream=self.stream)
         else:
             pa.pa_decode(q, st["k_cache"], st["v_cache"], tables, lens, spec.scale, spec.num_kv_heads, out,
-                         workspace=st["workspace"], partition_tokens=st["partition_tokens"], stream=stream)
+                         workspace=st["workspace"], partition_tokens=st["partition_tokens"], stream=self.stream)
 
-    def step():
-        k1(st["k"], st["v"], st["slots"])
-        k2(st["q"], st["tables"], st["lens"])
+    @property
+    def fused(self):
+        """One pa_decode_step call per step (16-bit cache, no shared-prefix groups)."""
+        return not self.fp8 and self.st["groups"] is None
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(device)
+    def step(self, k, v, slots, q, tables, lens, groups=None, out=None):
+        if self.fused:
+            st = self.st
+            self.pa.pa_decode_step(k, v, slots, q, st["k_cache"], st["v_cache"], tables, lens, st["spec"].scale,
+                                   st["spec"].num_kv_heads, st["out"] if out is None else out,
+                                   workspace=st["workspace"], partition_tokens=st["partition_tokens"],
+                                   stream=self.stream)
+        else:
+            self.k1(k, v, slots)
+            self.k2(q, tables, lens, groups, out)
 
-    for _ in range(max(3, args.warmup)):
-        step()
+    def resident_step(self):
+        st = self.st
+        self.step(st["k"], st["v"], st["slots"], st["q"], st["tables"], st["lens"])
+
+    def launches_per_step(self):
+        st = self.st
+        nparts_max = -(-int(st["wl"].max_blocks_per_seq * st["spec"].block_size) // st["ptok"])
+        return 2 + (1 if nparts_max > 1 else 0) + (1 if st["groups"] is not None else 0)
+
+
+def _events(torch, n):
+    return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+
+
+def time_device_steps(torch, ops, device, steps, warmup, barrier, clocks=True):
+    """W untimed steps, then exactly `steps` steps on resident inputs, bracketed by
+    a barrier and a synchronize on both sides, with clocks sampled meanwhile.  A
+    fused step (one pa_decode_step call) carries no events inside the region: its
+    launches run back to back and the region's events give their mean duration.
+    Otherwise K2+K3 carry their own events on the launching stream."""
+    st, stream = ops.st, ops.stream
+    for _ in range(max(3, warmup)):
+        ops.resident_step()
     barrier()
-
-    # timed region: K steps; the roofline kernel (K2+K3) carries events on the launching stream
-    k2_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    k2_ev = None if ops.fused else _events(torch, steps)
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(gpu_uuid(torch, device)) if not args.no_clocks else None
+    sampler = ClockSampler(gpu_uuid(torch, device)) if clocks else None
     if sampler:
         sampler.__enter__()
     barrier()
     start.record(stream)
-    for i in range(args.steps):
-        k1(st["k"], st["v"], st["slots"])
-        k2_ev[i][0].record(stream)
-        k2(st["q"], st["tables"], st["lens"])
-        k2_ev[i][1].record(stream)
+    for i in range(steps):
+        if k2_ev is None:
+            ops.resident_step()
+        else:
+            ops.k1(st["k"], st["v"], st["slots"])
+            k2_ev[i][0].record(stream)
+            ops.k2(st["q"], st["tables"], st["lens"])
+            k2_ev[i][1].record(stream)
     stop.record(stream)
     barrier()
     if sampler:
         sampler.__exit__(None, None, None)
-    elapsed_ms = start.elapsed_time(stop)
-    k2_ms = statistics.mean(a.elapsed_time(b) for a, b in k2_ev)
-    (elapsed_ms,) = max_over_ranks([elapsed_ms], dist if world > 1 else None, device)
+    elapsed = start.elapsed_time(stop)
+    return {"elapsed_ms": elapsed,
+            "k2_ms": statistics.mean(a.elapsed_time(b) for a, b in k2_ev) if k2_ev else None,
+            "clocks": sampler.summary() if sampler else None}
 
-    # K1 alone, for the detail line (outside the timed region)
-    k1_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(200)]
-    for a, b in k1_ev:
-        a.record(stream)
-        k1(st["k"], st["v"], st["slots"])
-        b.record(stream)
+
+def time_alone(torch, ops, barrier, which, n=200):
+    """K1 alone or K2+K3 alone (outside any timed region), mean event time per call."""
+    st = ops.st
+    ev = _events(torch, n)
+    for a, b in ev:
+        a.record(ops.stream)
+        if which == "k1":
+            ops.k1(st["k"], st["v"], st["slots"])
+        else:
+            ops.k2(st["q"], st["tables"], st["lens"])
+        b.record(ops.stream)
     barrier()
-    k1_ms = statistics.mean(a.elapsed_time(b) for a, b in k1_ev)
+    return statistics.mean(a.elapsed_time(b) for a, b in ev)
 
-    # e2e through the binding, two steps in flight: step i+1's inputs go H2D from
-    # pinned host memory on a copy stream while step i computes, and each step's
-    # output goes D2H on a third stream.  Every step still copies all of its own
-    # inputs and reads back its own result inside the timed region.
+
+def time_e2e_repeated(torch, ops, device, steps, barrier, clocks=True):
+    """e2e through the binding, two steps in flight: step i+1's inputs go H2D from
+    pinned host memory on a copy stream while step i computes, and each step's
+    output goes D2H on a third stream.  Every step still copies all of its own
+    inputs and reads back its own result inside the timed region."""
+    from paged_kv_cache_374_b200 import binding as pa
+    st, stream, spec = ops.st, ops.stream, ops.st["spec"]
     nbuf = 2
     names = ("q", "k", "v", "slots", "tables", "lens")
     offs, h2d = {}, 0
@@ -412,10 +446,10 @@ def run_native(args):
     ev_out = [torch.cuda.Event() for _ in range(nbuf)]    # out_d[b] is back on the host
 
     grp_dev = grp_h = None
+    n1 = spec.num_seqs + 1
     if st["groups"] is not None:  # the grouping is redone from the host tables every step: one int32 buffer of
-        n1 = spec.num_seqs + 1    # seq_start | group_offsets | group_members, (num_seqs + 1) entries each
-        grp_dev = [torch.empty(3 * n1, dtype=torch.int32, device=device) for _ in range(nbuf)]
-        grp_h = [torch.zeros(3 * n1, dtype=torch.int32).pin_memory() for _ in range(nbuf)]
+        grp_dev = [torch.empty(3 * n1, dtype=torch.int32, device=device) for _ in range(nbuf)]  # seq_start |
+        grp_h = [torch.zeros(3 * n1, dtype=torch.int32).pin_memory() for _ in range(nbuf)]     # offsets | members
         h2d += 4 * 3 * n1
 
     def e2e_step(i):
@@ -437,48 +471,320 @@ def run_native(args):
             ev_in[b].record(h2d_stream)
         stream.wait_event(ev_in[b])
         stream.wait_event(ev_out[b])                   # out_d[b] of the step two back is on the host
-        k1(dev_in[b]["k"], dev_in[b]["v"], dev_in[b]["slots"])
-        k2(dev_in[b]["q"], dev_in[b]["tables"], dev_in[b]["lens"], groups, out=out_d[b])
+        ops.step(dev_in[b]["k"], dev_in[b]["v"], dev_in[b]["slots"], dev_in[b]["q"], dev_in[b]["tables"],
+                 dev_in[b]["lens"], groups, out=out_d[b])
         ev_used[b].record(stream)
         d2h_stream.wait_event(ev_used[b])
         with torch.cuda.stream(d2h_stream):
             out_h[b].copy_(out_d[b], non_blocking=True)
             ev_out[b].record(d2h_stream)
 
-    e2e_steps = args.steps
     for i in range(3):
         e2e_step(i)
     barrier()
-    e2e_sampler = ClockSampler(gpu_uuid(torch, device)) if not args.no_clocks else None
-    if e2e_sampler:
-        e2e_sampler.__enter__()
+    sampler = ClockSampler(gpu_uuid(torch, device)) if clocks else None
+    if sampler:
+        sampler.__enter__()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     h2d_stream.wait_event(e0)
-    for i in range(e2e_steps):
+    for i in range(steps):
         e2e_step(i)
-    stream.wait_event(ev_out[(e2e_steps - 1) % nbuf])  # the last read-back (the D2H stream runs in order)
+    stream.wait_event(ev_out[(steps - 1) % nbuf])  # the last read-back (the D2H stream runs in order)
     e1.record(stream)
     barrier()
-    if e2e_sampler:
-        e2e_sampler.__exit__(None, None, None)
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if sampler:
+        sampler.__exit__(None, None, None)
     # the pipelined steps compute what the device-timed ones did (same inputs, same cache slots)
-    e2e_matches = bool(torch.equal(out_h[(e2e_steps - 1) % nbuf], st["out"].cpu()))
-    (e2e_ms,) = max_over_ranks([e2e_ms], dist if world > 1 else None, device)
+    matches = bool(torch.equal(out_h[(steps - 1) % nbuf], st["out"].cpu()))
+    return {"e2e_ms": e0.elapsed_time(e1) / steps, "h2d": h2d, "d2h": d2h, "matches": matches,
+            "clocks": sampler.summary() if sampler else None}
+
+
+def roofline_traffic(st, workload, fp8, ab):
+    key = workload + ("+fp8" if fp8 else "")
+    if st["groups"] is not None:
+        return profiled_traffic(ab["unique_tokens"], workload, SHARED_PROFILE_SUMMARY)
+    return profiled_traffic(ab["unique_tokens"], key, TRAFFIC_SUMMARIES.get(key, PROFILE_SUMMARY))
+
+
+def roofline_leg(ops, ab, t, steps):
+    """(bytes, ms) of the kernel sequence the roofline is taken on: the whole fused
+    step (K1 + K2 + K3: the write's bytes too, and the region's mean per step), or
+    K2+K3 alone with their per-step events."""
+    if ops.fused:
+        return ab["unique"] + ab["k1"], t["elapsed_ms"] / steps
+    return ab["unique"], t["k2_ms"]
+
+
+def roofline_kernel(ops):
+    if ops.fused:
+        return ("reshape_and_cache_kernel + paged_decode_kernel + paged_decode_merge_kernel (one pa_decode_step "
+                "call: K2 a programmatic dependent of K1)")
+    if ops.st["groups"] is not None:
+        return ("shared-prefix kernel + paged_decode_kernel + paged_decode_merge_kernel (timed together: one "
+                "pa_decode_shared_prefix call)")
+    return "paged_decode_kernel + paged_decode_merge_kernel (timed together: one pa_decode call)"
+
+
+def steps_for(torch, ops, target_s, lo=200, hi=40000):
+    """Steps that fill about target_s of device time (from a 20-step probe)."""
+    st, stream = ops.st, ops.stream
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(20):
+        ops.resident_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    per = a.elapsed_time(b) / 20 / 1e3
+    return int(min(hi, max(lo, target_s / max(per, 1e-7))))
+
+
+def measure_repeated(torch, name, device, args, target_s=0.8, shared=True):
+    """One detail entry: the workload's step repeated on resident inputs for about
+    target_s, its K2+K3 against the roofline, and an e2e over as many steps."""
+    st = build_step(name, device, args.partition_tokens, shared=shared)
+    ops = Ops(st, torch.cuda.current_stream(device), False)
+    barrier = lambda: torch.cuda.synchronize(device)
+    for _ in range(5):
+        ops.resident_step()
+    steps = steps_for(torch, ops, target_s)
+    t = time_device_steps(torch, ops, device, steps, 5, barrier)
+    e = time_e2e_repeated(torch, ops, device, steps, barrier)
+    k2k3_ms = time_alone(torch, ops, barrier, "k2k3")
+    ab = algorithmic_bytes(st)
+    peak, _ = measured_hbm_peak()
+    nbytes, ms = roofline_leg(ops, ab, t, steps)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    spec = st["spec"]
+    res = {"workload": f"{spec.name}: {spec.description}", "steps": steps,
+           "tokens_per_s": round(spec.num_seqs / (t["elapsed_ms"] / steps / 1e3), 1),
+           "ms_per_step": round(t["elapsed_ms"] / steps, 5), "k2k3_us_alone": round(k2k3_ms * 1e3, 2),
+           "roofline_kernel": roofline_kernel(ops), "bytes_per_step": nbytes, "kv_gbs": round(gbs, 1),
+           "frac": round(gbs / peak, 4), "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+           "traffic": roofline_traffic(st, name, False, ab), "clocks": t["clocks"],
+           "e2e_tokens_per_s": round(spec.num_seqs / (e["e2e_ms"] / 1e3), 1), "e2e_output_matches": e["matches"],
+           "e2e_clocks": e["clocks"]}
+    if st["groups"] is not None:
+        res["path"] = "pa_decode_shared_prefix: %d group(s), %d shared tokens" % (st["groups"].num_groups,
+                                                                                  st["groups"].max_shared_tokens)
+    del st, ops
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_append_loop(torch, name, device, args, target_s=0.8):
+    """The workload as its configuration states it: `spec.steps` consecutive decode
+    steps, each appending one token per sequence.  Every step runs a1 on the host
+    (pa_append_slots: a new block at each block boundary), K1 into the step's slots
+    and K2+K3 over the grown tables and lengths.
+
+    Device leg: the steps' tables, lengths and slots are resolved by a1 up front and
+    resident in HBM; each pass runs the spec.steps steps in order (K2+K3 timed with
+    events, each step against its own algorithmic bytes); passes repeat for about
+    target_s.  e2e leg: each pass starts from the same allocator state (rebuilt
+    outside the timed region) and every step runs a1 on the host, copies that
+    step's inputs (q, k, v, the grown tables, lengths and slots) H2D from pinned
+    memory, runs K1 + K2+K3 and reads the output back, two steps in flight."""
+    from paged_kv_cache_374_b200 import binding as pa
+    st = build_step(name, device, args.partition_tokens, shared=False)
+    spec, wl = st["spec"], st["wl"]
+    bs, S, nsteps = spec.block_size, spec.num_seqs, spec.steps
+    stream = torch.cuda.current_stream(device)
+    ops = Ops(st, stream, False)
+
+    def fresh_state():
+        """Allocator and host tables/lengths before step 1 (every pass starts here)."""
+        alloc = pa.BlockAllocator(wl.num_blocks, wl.pool_order)
+        tables = np.full((S, wl.max_blocks_per_seq), -1, dtype=np.int32)
+        stored = (wl.context_lens - 1).astype(np.int32)
+        for i in range(S):
+            n = pa.pa_num_required_blocks(int(stored[i]), bs)
+            tables[i, :n] = alloc.alloc_n(n)
+        return alloc, tables, stored.copy()
+
+    alloc, tables, lens = fresh_state()
+    per_step, a1_us = [], []
+    for _ in range(nsteps):
+        t0 = time.perf_counter()
+        slots = alloc.append_slots(tables, lens, bs)
+        a1_us.append((time.perf_counter() - t0) * 1e6)
+        per_step.append((tables.copy(), lens.copy(), slots.copy()))
+    new_blocks = int(np.sum(per_step[-1][0] >= 0) - np.sum(per_step[0][0] >= 0))
+    dev_steps = [tuple(torch.from_numpy(x).to(device) for x in s) for s in per_step]
+    step_bytes = [algorithmic_bytes(st, lens=s[1])["unique"] + (algorithmic_bytes(st)["k1"] if ops.fused else 0)
+                  for s in per_step]
+    del alloc
+
+    def run_pass(ev=None):
+        for i, (tb, ln, sl) in enumerate(dev_steps):
+            if ops.fused:                 # events around the one call of the step
+                if ev is not None:
+                    ev[i][0].record(stream)
+                ops.step(st["k"], st["v"], sl, st["q"], tb, ln)
+            else:                         # events around K2+K3
+                ops.k1(st["k"], st["v"], sl)
+                if ev is not None:
+                    ev[i][0].record(stream)
+                ops.k2(st["q"], tb, ln)
+            if ev is not None:
+                ev[i][1].record(stream)
+
+    for _ in range(3):
+        run_pass()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    run_pass()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    passes = int(min(400, max(3, target_s / max(a.elapsed_time(b) / 1e3, 1e-6))))
+    evs = [_events(torch, nsteps) for _ in range(passes)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(gpu_uuid(torch, device))
+    sampler.__enter__()
+    torch.cuda.synchronize(device)
+    start.record(stream)
+    for p in range(passes):
+        run_pass(evs[p])
+    stop.record(stream)
+    torch.cuda.synchronize(device)
+    sampler.__exit__(None, None, None)
+    total_ms = start.elapsed_time(stop)
+    k2_ms = np.array([[e0.elapsed_time(e1) for e0, e1 in ev] for ev in evs]).mean(axis=0)  # per step
+    peak, _ = measured_hbm_peak()
+    gbs_steps = [by / (ms / 1e3) / 1e9 for by, ms in zip(step_bytes, k2_ms)]
+    gbs = sum(step_bytes) / (float(np.sum(k2_ms)) / 1e3) / 1e9
+    ref_out = st["out"].clone()   # output of the last step of the last pass
+
+    # e2e: a1 on the host, the step's inputs H2D, K1 + K2+K3, the output D2H
+    nbuf = 2
+    sizes = {"q": st["q"], "k": st["k"], "v": st["v"]}
+    mb = wl.max_blocks_per_seq
+    fixed = {n: t.numel() * t.element_size() for n, t in sizes.items()}
+    layout, off = {}, 0
+    for n, nb in list(fixed.items()) + [("tables", S * mb * 4), ("lens", S * 4), ("slots", S * 8)]:
+        layout[n] = (off, nb)
+        off += -(-nb // 256) * 256
+    h2d = off
+    host = [torch.empty(h2d, dtype=torch.uint8).pin_memory() for _ in range(nbuf)]
+    for hb in host:
+        for n, t in sizes.items():
+            o, nb = layout[n]
+            hb[o:o + nb].copy_(t.cpu().contiguous().view(-1).view(torch.uint8))
+    dev_buf = [torch.empty(h2d, dtype=torch.uint8, device=device) for _ in range(nbuf)]
+
+    def view(b, n, dtype, shape):
+        o, nb = layout[n]
+        return dev_buf[b][o:o + nb].view(dtype).view(shape)
+    dev_in = [{"q": view(b, "q", st["q"].dtype, st["q"].shape), "k": view(b, "k", st["k"].dtype, st["k"].shape),
+               "v": view(b, "v", st["v"].dtype, st["v"].shape), "tables": view(b, "tables", torch.int32, (S, mb)),
+               "lens": view(b, "lens", torch.int32, (S,)), "slots": view(b, "slots", torch.int64, (S,))}
+              for b in range(nbuf)]
+    out_d = [torch.empty_like(st["out"]) for _ in range(nbuf)]
+    out_h = [torch.empty(st["out"].shape, dtype=st["out"].dtype).pin_memory() for _ in range(nbuf)]
+    d2h = out_h[0].numel() * out_h[0].element_size()
+    h2d_stream, d2h_stream = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_used = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_out = [torch.cuda.Event() for _ in range(nbuf)]
+
+    def e2e_pass(alloc, tables, lens):
+        for i in range(nsteps):
+            b = i % nbuf
+            slots = alloc.append_slots(tables, lens, bs)       # a1 on the host
+            ev_in[b].synchronize()                            # the copy that last read host[b] is done
+            hv = host[b].numpy()
+            for n, arr in (("tables", tables), ("lens", lens), ("slots", slots)):
+                o, nb = layout[n]
+                hv[o:o + nb] = np.ascontiguousarray(arr).view(np.uint8).reshape(-1)
+            with torch.cuda.stream(h2d_stream):
+                h2d_stream.wait_event(ev_used[b])
+                dev_buf[b].copy_(host[b], non_blocking=True)
+                ev_in[b].record(h2d_stream)
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])
+            ops.step(dev_in[b]["k"], dev_in[b]["v"], dev_in[b]["slots"], dev_in[b]["q"], dev_in[b]["tables"],
+                     dev_in[b]["lens"], out=out_d[b])
+            ev_used[b].record(stream)
+            d2h_stream.wait_event(ev_used[b])
+            with torch.cuda.stream(d2h_stream):
+                out_h[b].copy_(out_d[b], non_blocking=True)
+                ev_out[b].record(d2h_stream)
+
+    e2e_ms, matches = 0.0, True
+    e_sampler = ClockSampler(gpu_uuid(torch, device))
+    e_sampler.__enter__()
+    for p in range(passes + 1):                  # the first pass is a warm-up
+        state = fresh_state()                    # outside the timed region
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        h2d_stream.wait_event(e0)
+        e2e_pass(*state)
+        stream.wait_event(ev_out[(nsteps - 1) % nbuf])
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        if p:
+            e2e_ms += e0.elapsed_time(e1)
+        # every pass re-derives the device leg's tables and slots step for step
+        matches &= bool(np.array_equal(state[1], per_step[-1][0]) and np.array_equal(state[2], per_step[-1][1]))
+    e_sampler.__exit__(None, None, None)
+    matches &= bool(torch.equal(out_h[(nsteps - 1) % nbuf], ref_out.cpu()))
+    res = {"workload": f"{spec.name}: {spec.description}", "steps_per_pass": nsteps, "passes": passes,
+           "new_blocks_per_pass": new_blocks,
+           "tokens_per_s": round(S * nsteps * passes / (total_ms / 1e3), 1),
+           "ms_per_step": round(total_ms / (nsteps * passes), 5),
+           "roofline_kernel": roofline_kernel(ops), "roofline_us_per_step": round(float(np.mean(k2_ms)) * 1e3, 2),
+           "roofline_us_first_last": [round(float(k2_ms[0]) * 1e3, 2), round(float(k2_ms[-1]) * 1e3, 2)],
+           "bytes_per_pass": int(sum(step_bytes)), "kv_gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+           "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+           "kv_gbs_min_max_step": [round(min(gbs_steps), 1), round(max(gbs_steps), 1)],
+           "a1_us_mean": round(float(np.mean(a1_us)), 1), "clocks": sampler.summary(),
+           "e2e_tokens_per_s": round(S * nsteps * passes / (e2e_ms / 1e3), 1),
+           "e2e_h2d_bytes_per_step": h2d, "e2e_d2h_bytes_per_step": d2h, "e2e_output_matches": matches,
+           "e2e_clocks": e_sampler.summary()}
+    del st, ops, dev_steps
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+    st = build_step(args.workload, device, args.partition_tokens, args.num_seqs, args.kv_dtype,
+                    shared=args.shared_prefix == "auto")
+    fp8 = args.kv_dtype == "fp8"
+    spec = st["spec"]
+    stream = torch.cuda.current_stream(device)
+    ops = Ops(st, stream, fp8)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+
+    t = time_device_steps(torch, ops, device, args.steps, args.warmup, barrier, clocks=not args.no_clocks)
+    (elapsed_ms,) = max_over_ranks([t["elapsed_ms"]], dist if world > 1 else None, device)
+    k1_ms = time_alone(torch, ops, barrier, "k1")
+    k2_ms = t["k2_ms"] if t["k2_ms"] is not None else time_alone(torch, ops, barrier, "k2k3")
+    e = time_e2e_repeated(torch, ops, device, args.steps, barrier, clocks=not args.no_clocks)
+    (e2e_ms,) = max_over_ranks([e["e2e_ms"]], dist if world > 1 else None, device)
 
     ab = algorithmic_bytes(st)
-    traffic_key = args.workload + ("+fp8" if fp8 else "")
     ms_per_step = elapsed_ms / args.steps
     tokens_per_step = spec.num_seqs
     value = job_throughput(world, tokens_per_step, ms_per_step)
     peak, peak_kind = measured_hbm_peak()
-    achieved = ab["unique"] / (k2_ms / 1e3) / 1e9
-    nparts_max = -(-int(st["wl"].max_blocks_per_seq * spec.block_size) // (
-        st["partition_tokens"] or pa.pa_decode_partition_tokens(spec.num_seqs, spec.num_heads, spec.num_kv_heads,
-                                                                 spec.head_dim, spec.block_size,
-                                                                 st["wl"].max_blocks_per_seq)))
-    launches_per_step = 2 + (1 if nparts_max > 1 else 0) + (1 if st["groups"] is not None else 0)
+    roof_bytes, roof_ms = roofline_leg(ops, ab, dict(t, elapsed_ms=elapsed_ms), args.steps)
+    achieved = roof_bytes / (roof_ms / 1e3) / 1e9
     result = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -499,26 +805,37 @@ def run_native(args):
         "detail": {
             "kv_gbs": round(achieved, 1), "frac_of_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
             "kv_bytes_per_step": ab["unique"], "logical_kv_bytes_per_step": ab["logical"],
-            "k1_us": round(k1_ms * 1e3, 2), "k2k3_us": round(k2_ms * 1e3, 2), "a1_us": round(st["a1_us"], 1),
-            "e2e_ms_per_step": round(e2e_ms, 4), "e2e_output_matches": e2e_matches,
+            "k1_bytes_per_step": ab["k1"], "roofline_bytes_per_step": roof_bytes,
+            "k1_us_alone": round(k1_ms * 1e3, 2), "k2k3_us" + ("_alone" if ops.fused else ""): round(k2_ms * 1e3, 2),
+            "k2k3_gbs_alone" if ops.fused else "k2k3_gbs": round(ab["unique"] / (k2_ms / 1e3) / 1e9, 1),
+            "a1_us": round(st["a1_us"], 1),
+            "e2e_ms_per_step": round(e2e_ms, 4), "e2e_output_matches": e["matches"],
         },
         "roofline": {
-            "kernel": ("shared-prefix kernel + paged_decode_kernel + paged_decode_merge_kernel (timed together: one "
-                       "pa_decode_shared_prefix call)" if st["groups"] is not None else
-                       "paged_decode_kernel + paged_decode_merge_kernel (timed together: one pa_decode call)"),
-            "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+            "kernel": roofline_kernel(ops),
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+            "peak_kind": (peak_kind + ": a device copy, which reads and writes; this kernel almost only reads, "
+                          "so it can pass 1.0 (frac_of_nominal is against 8 TB/s)"),
             "unit": "GB/s", "frac": round(achieved / peak, 4),
-            "traffic": (profiled_traffic(ab["unique_tokens"], args.workload, SHARED_PROFILE_SUMMARY)
-                        if st["groups"] is not None else
-                        profiled_traffic(ab["unique_tokens"], traffic_key,
-                                         TRAFFIC_SUMMARIES.get(traffic_key, PROFILE_SUMMARY))),
+            "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+            "traffic": roofline_traffic(st, args.workload, fp8, ab),
         },
         "e2e": {"value": round(job_throughput(world, tokens_per_step, e2e_ms), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "clocks": e2e_sampler.summary() if e2e_sampler else None},
-        "gpu_launches": args.steps * launches_per_step,
-        "clocks": sampler.summary() if sampler else None,
+                "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"], "clocks": e["clocks"]},
+        "gpu_launches": args.steps * ops.launches_per_step(),
+        "clocks": t["clocks"],
     }
+    del ops, st
+    torch.cuda.empty_cache()
+    if (world == 1 and not args.no_detail_workloads and not fp8 and args.num_seqs is None
+            and args.workload == "llama7b"):
+        # the other configurations, each with its own clocks: 13B as its 32-step
+        # append loop, GQA long context, and the beam batch's shared prefix
+        result["detail"]["workloads"] = {
+            "llama13b": measure_append_loop(torch, "llama13b", device, args),
+            "gqa70b": measure_repeated(torch, "gqa70b", device, args),
+            "beam": measure_repeated(torch, "beam", device, args, shared=args.shared_prefix == "auto"),
+        }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args.workload, budget_s=12.0)
     if world > 1:

@@ -60,7 +60,9 @@ enum {
     PA_DEVERR_SLOT_RANGE = 1,    /* slot_mapping entry >= num_blocks * block_size (write skipped) */
     PA_DEVERR_TABLE_RANGE = 2,   /* block_tables entry outside [0, num_blocks) (output row is NaN) */
     PA_DEVERR_LEN_RANGE = 4,     /* context_len < 0 or > max_blocks_per_seq * block_size (row NaN) */
-    PA_DEVERR_TIMEOUT = 8        /* an in-kernel wait gave up (the output is not valid) */
+    PA_DEVERR_TIMEOUT = 8,       /* an in-kernel wait gave up (the output is not valid) */
+    PA_DEVERR_GROUP_RANGE = 16,  /* a shared-prefix group's offsets or members out of range (group skipped) */
+    PA_DEVERR_PAIR_CONFLICT = 32 /* a block-copy pair overlaps another pair (pair skipped) */
 };
 
 /* Human-readable name of a pa_status value (static storage). */
@@ -103,8 +105,9 @@ int pa_decode_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, in
 
 /*
  * Bytes of device workspace pa_decode needs for these sizes: 256 bytes of
- * scheduling counters, plus the partial results of split sequences when a
- * sequence can span more than one partition.  partition_tokens: 0 = the default
+ * scheduling counters, plus, when a sequence can span more than one partition,
+ * a merge counter and a merge-queue entry per (sequence, query head) and the
+ * partial results of split sequences.  partition_tokens: 0 = the default
  * above, otherwise a positive multiple of 64, at most 65536.  Returns 0 for
  * invalid sizes.
  */
@@ -134,12 +137,13 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, i
  *   out           [num_seqs][num_heads][head_dim], dtype, device
  *   partition_tokens  0 = default; else a positive multiple of 64
  *   workspace     device scratch of at least pa_decode_workspace_size(...)
- *                 bytes.  Its first 256 bytes are the kernels' work-claim
- *                 counters: zero them once before the first call (cudaMemset);
- *                 every call leaves them zero again, so a workspace can be reused
- *                 call after call on one stream.  Calls that may run at the same
- *                 time need separate workspaces.  After a PA_DEVERR_TIMEOUT,
- *                 zero the counters again.
+ *                 bytes.  It starts with the kernels' counters (work claims and,
+ *                 when contexts are split, the merge queue: 256 bytes plus 8 per
+ *                 (sequence, query head)): zero the whole workspace once before
+ *                 the first call (cudaMemset); every call leaves the counters
+ *                 zero again, so a workspace can be reused call after call on one
+ *                 stream.  Calls that may run at the same time need separate
+ *                 workspaces.  After a PA_DEVERR_TIMEOUT, zero it again.
  *
  * Supported: head_dim in {64, 128}; block_size in {16, 32, 64}; num_heads a
  * multiple of num_kv_heads; any num_seqs >= 0.  Otherwise PA_ERR_UNSUPPORTED or
@@ -150,6 +154,29 @@ int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int
               int num_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
               int dtype, int partition_tokens, void* workspace, size_t workspace_bytes, int32_t* err_word,
               void* stream);
+
+/*
+ * pa_decode_step -- one whole decode step in one call: write each sequence's new
+ * token into its slot, then attend over the caches that now hold it (P2 §2.1,
+ * decode steps 3-5: the current token's K/V join the cache, then attention runs
+ * over all t tokens).  The result is exactly that of
+ *     pa_reshape_and_cache(k, v, slot_mapping, ..., num_tokens = num_seqs, ...)
+ *     pa_decode(q, ...)
+ * in that order on `stream`.  In one call the attention kernel is launched as a
+ * programmatic dependent of the cache write: its launch and its scheduling
+ * prologue (which read only context_lens, block_tables and q) overlap the write,
+ * and every warp waits for the write to complete before its first cache read.
+ *
+ *   k, v, slot_mapping  as pa_reshape_and_cache, one new token per sequence
+ *                       (token i belongs to sequence i; num_tokens = num_seqs)
+ *   everything else     as pa_decode (the caches are written, then read)
+ * Errors: the checks of both calls run first; on an error nothing is launched.
+ */
+int pa_decode_step(const void* k, const void* v, const int64_t* slot_mapping, const void* q, void* k_cache,
+                   void* v_cache, const int32_t* block_tables, const int32_t* context_lens, float scale,
+                   int num_kv_heads, void* out, int num_seqs, int num_heads, int head_dim, int block_size,
+                   int num_blocks, int max_blocks_per_seq, int dtype, int partition_tokens, void* workspace,
+                   size_t workspace_bytes, int32_t* err_word, void* stream);
 
 /*
  * pa_decode_noalloc -- pa_decode for callers that cannot allocate device memory.
@@ -199,7 +226,11 @@ int pa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, c
  *   num_groups     groups of sequences sharing a prefix (host int; 0 = pa_decode)
  *   group_offsets  [num_groups + 1] int32: group g is
  *   group_members  group_members[group_offsets[g] .. group_offsets[g+1]) (sequence
- *                  indices); every member has the same seq_start
+ *                  indices); every member has the same seq_start.  A group whose
+ *                  offsets are not 0 <= offsets[g] <= offsets[g+1] <= num_seqs, or
+ *                  that lists a member outside [0, num_seqs), is skipped and
+ *                  reported as PA_DEVERR_GROUP_RANGE (its members' outputs are
+ *                  then undefined; every other sequence is unaffected)
  *   max_group_size, max_shared_tokens  host ints bounding the group sizes and the
  *                  seq_start values (the launch sizes); a group beyond them is
  *                  reported as PA_DEVERR_LEN_RANGE and its output is undefined
@@ -309,10 +340,11 @@ int pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const
  *   q, out        [T][num_heads][head_dim], T = query_start[num_seqs], dtype, device
  *   query_start   int32 [num_seqs + 1], device; n_s <= context_lens[s]
  *   max_query_len the largest n_s (sizes the grid)
- * Caches, tables, lengths, dtype and supported sizes as pa_decode;
- * max_blocks_per_seq at most 4096.  Tensor cores (mma.sync m16n8k16, fp32
- * accumulation); p enters P.V as two 16-bit terms.  Bad lengths or table entries
- * give NaN rows and PA_DEVERR_* bits.
+ * Caches, tables, lengths, dtype and supported sizes as pa_decode.  Runs on the
+ * 5th-generation tensor cores (tcgen05 MMAs, fp32 accumulators in tensor
+ * memory).  The softmax weights p (at most 2^8 by construction) enter P.V as one
+ * f16 term for f16 inputs, or as two bf16 terms (hi + lo) for bf16 inputs.
+ * Bad lengths or table entries give NaN rows and PA_DEVERR_* bits.
  */
 int pa_prefill(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
                const int32_t* context_lens, const int32_t* query_start, float scale, int num_kv_heads, void* out,
@@ -423,8 +455,13 @@ int pa_cow_prepare(pa_allocator* a, int32_t* block_tables, int max_blocks_per_se
  * v_cache[src_i], all block_size x num_kv_heads x head_dim elements, bit for bit.
  *   copy_pairs  device int32 [2 * num_pairs]: (src, dst) per pair
  *   element_bytes  bytes per cache element (2 for fp16/bf16, 1 for 8-bit caches)
- * Destinations must be distinct and must not be sources of other pairs.  A pair
- * with an id outside [0, num_blocks) is skipped and sets PA_DEVERR_TABLE_RANGE.
+ * The pairs are copied all at once, so they must not overlap: a pair whose
+ * destination is another pair's destination or source, or whose source is
+ * another pair's destination, is skipped and sets PA_DEVERR_PAIR_CONFLICT (a
+ * chained list such as (a, b), (b, c) is refused rather than copied in some
+ * order; pa_cow_prepare never produces one).  Several pairs may share a source.
+ * A pair with an id outside [0, num_blocks) is skipped and sets
+ * PA_DEVERR_TABLE_RANGE.
  */
 int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* copy_pairs, int num_pairs, int num_kv_heads,
                    int head_dim, int block_size, int num_blocks, int element_bytes, int32_t* err_word,

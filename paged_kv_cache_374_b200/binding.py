@@ -18,6 +18,7 @@ LIBRARY = os.path.join(_PKG, "libpa.so")
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_OUT_OF_BLOCKS, PA_ERR_REFCOUNT, PA_ERR_CUDA = range(6)
 PA_F16, PA_BF16 = 0, 1
 PA_DEVERR_SLOT_RANGE, PA_DEVERR_TABLE_RANGE, PA_DEVERR_LEN_RANGE, PA_DEVERR_TIMEOUT = 1, 2, 4, 8
+PA_DEVERR_GROUP_RANGE, PA_DEVERR_PAIR_CONFLICT = 16, 32
 
 if not os.path.exists(LIBRARY):
     raise ImportError(f"{LIBRARY} is missing: build it with `python -m paged_kv_cache_374_b200.build` "
@@ -44,6 +45,8 @@ _sig("pa_decode_partition_tokens", _i32, _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_decode_workspace_size", ctypes.c_size_t, _i32, _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_decode", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
      _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
+_sig("pa_decode_step", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32, _i32, _i32,
+     _i32, _i32, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
 _sig("pa_decode_noalloc", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32, _i32, _i32, _i32, _i32,
      _i32, _i32, _i32, _vp, _vp)
 _sig("pa_reshape_and_cache_fp8", _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_float,
@@ -189,6 +192,38 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_hea
                         s, h, d, bs, nb, mb, dt, int(partition_tokens), ws_ptr, ws_bytes,
                         _dev(err_word, "err_word", torch.int32), _stream(stream, q))
     _check(st, "pa_decode")
+    return out
+
+
+def pa_decode_step(k, v, slot_mapping, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out,
+                   workspace=None, partition_tokens=0, err_word=None, stream=None):
+    """K1 then K2 + K3 in one call: each sequence's new k/v [S, Hk, d] into its slot
+    (slot_mapping int64 [S]), then attention as pa_decode.  Returns ``out``."""
+    import torch
+    s, h, d = q.shape
+    nb, bs, hk, d2 = k_cache.shape
+    if hk != num_kv_heads or d2 != d or v_cache.shape != k_cache.shape or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if k.shape != (s, hk, d) or v.shape != k.shape or slot_mapping.shape != (s,):
+        raise ValueError("k, v must be [S, Hk, d] and slot_mapping [S]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [S, MB] and context_lens [S]")
+    mb = block_tables.shape[1]
+    dt = _dtype_code(q)
+    for t in (k, v, k_cache, v_cache, out):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, the caches and out must share one dtype")
+    need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = _lib.pa_decode_step(_dev(k, "k"), _dev(v, "v"), _dev(slot_mapping, "slot_mapping", torch.int64),
+                             _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                             _dev(block_tables, "block_tables", torch.int32),
+                             _dev(context_lens, "context_lens", torch.int32), float(scale), hk, _dev(out, "out"),
+                             s, h, d, bs, nb, mb, dt, int(partition_tokens), _dev(workspace, "workspace"),
+                             workspace.numel() * workspace.element_size(), _dev(err_word, "err_word", torch.int32),
+                             _stream(stream, q))
+    _check(st, "pa_decode_step")
     return out
 
 

@@ -1,29 +1,79 @@
 // pa_copy_blocks: whole-block copies inside the paged caches (copy-on-write after
-// a beam fork); pa_swap_blocks: the same between two pools (swap-out / swap-in).  One physical block of one cache is block_size * num_kv_heads *
-// head_dim elements, contiguous in the [num_blocks][block_size][num_kv_heads]
-// [head_dim] layout, so a pair is one contiguous run per cache; threads copy
-// 16-byte vectors, grid-stride over (pair, vector), K and V alike.
+// a beam fork); pa_swap_blocks: the same between two pools (swap-out / swap-in).
+// One physical block of one cache is block_size * num_kv_heads * head_dim
+// elements, contiguous in the [num_blocks][block_size][num_kv_heads][head_dim]
+// layout, so a pair is one contiguous run per cache; threads copy 16-byte
+// vectors, K and V alike.
+#include <atomic>
+
 #include "pa_device.cuh"
 #include "pa_host.h"
 
 namespace pa {
 
-__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
-                                                           const int32_t* __restrict__ pairs, int num_pairs,
-                                                           int64_t block_vecs, int num_blocks, int32_t* err_word) {
+// The (pair, 16-byte vector) space of all pairs is cut into one contiguous,
+// equal slice per CTA (every CTA resident at once, no tail wave); a CTA walks its
+// slice pair by pair.  The pairs are copied all at once, so a pair that overlaps
+// another copying pair -- its destination is another's destination or source, or
+// its source is another's destination -- is skipped and reported: a CTA checks
+// each pair its slice touches against the whole list (num_pairs comparisons
+// spread over its threads).  Pairs that copy nothing (ids out of range, source ==
+// destination) conflict with nothing.
+__global__ void __launch_bounds__(256, 4) copy_blocks_kernel(uint4* __restrict__ k_cache,
+                                                              uint4* __restrict__ v_cache,
+                                                              const int32_t* __restrict__ pairs, int num_pairs,
+                                                              int64_t block_vecs, int num_blocks, int32_t* err_word) {
+    constexpr int U = 4;  // 16-byte vectors in flight per thread and cache
     const int64_t total = (int64_t)num_pairs * block_vecs;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
-        const int64_t pi = i / block_vecs;
-        const int64_t c = i - pi * block_vecs;
+    const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+    int64_t lo = (int64_t)blockIdx.x * per;
+    const int64_t hi = lo + per < total ? lo + per : total;
+    while (lo < hi) {
+        const int64_t pi = lo / block_vecs;
+        const int64_t c0 = lo - pi * block_vecs;
+        const int64_t c1 = c0 + (hi - lo) < block_vecs ? c0 + (hi - lo) : block_vecs;
+        lo += c1 - c0;
         const int32_t src = __ldg(pairs + 2 * pi), dst = __ldg(pairs + 2 * pi + 1);
         if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
-            if (c == 0) report(err_word, PA_DEVERR_TABLE_RANGE);
+            if (c0 == 0 && threadIdx.x == 0) report(err_word, PA_DEVERR_TABLE_RANGE);
             continue;
         }
         if (src == dst) continue;
-        k_cache[(int64_t)dst * block_vecs + c] = __ldcs(k_cache + (int64_t)src * block_vecs + c);
-        v_cache[(int64_t)dst * block_vecs + c] = __ldcs(v_cache + (int64_t)src * block_vecs + c);
+        bool conflict = false;
+        for (int j = threadIdx.x; j < num_pairs; j += blockDim.x) {
+            const int32_t sj = __ldg(pairs + 2 * (int64_t)j), dj = __ldg(pairs + 2 * (int64_t)j + 1);
+            if (j == pi || sj == dj || sj < 0 || sj >= num_blocks || dj < 0 || dj >= num_blocks) continue;
+            conflict |= dj == dst || sj == dst || dj == src;
+        }
+        if (__syncthreads_or(conflict)) {
+            if (c0 == 0 && threadIdx.x == 0) report(err_word, PA_DEVERR_PAIR_CONFLICT);
+            continue;
+        }
+        // this slice's part of the pair: n vectors from c0 (a block is far below 2^31 vectors)
+        const int n = (int)(c1 - c0);
+        const uint4* ks = k_cache + (int64_t)src * block_vecs + c0;
+        const uint4* vs = v_cache + (int64_t)src * block_vecs + c0;
+        uint4* kd = k_cache + (int64_t)dst * block_vecs + c0;
+        uint4* vd = v_cache + (int64_t)dst * block_vecs + c0;
+        for (int i = threadIdx.x; i < n; i += 256 * U) {
+            uint4 a[U], b[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int j = i + u * 256;
+                if (j < n) {
+                    a[u] = __ldcs(ks + j);
+                    b[u] = __ldcs(vs + j);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int j = i + u * 256;
+                if (j < n) {
+                    kd[j] = a[u];
+                    vd[j] = b[u];
+                }
+            }
+        }
     }
 }
 
@@ -92,11 +142,21 @@ extern "C" int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* copy_
         return PA_ERR_INVALID_ARG;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t total = (int64_t)num_pairs * (block_bytes / 16);
-    int64_t blocks = (total + 255) / 256;
-    if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+    // every CTA resident at once (as many per SM as fit), each with a slice of at
+    // least 1024 vectors (16 KiB per cache)
+    static std::atomic<int> per_sm{0};
+    if (per_sm.load(std::memory_order_relaxed) == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, copy_blocks_kernel, 256, 0) != cudaSuccess || n < 1)
+            return PA_ERR_CUDA;
+        per_sm.store(n, std::memory_order_relaxed);
+    }
+    const int64_t block_vecs = block_bytes / 16;
+    const int64_t target = (int64_t)sms * per_sm.load(std::memory_order_relaxed);
+    const int64_t slices = ((int64_t)num_pairs * block_vecs + 1023) / 1024;
+    const int64_t blocks = slices < target ? slices : target;
     copy_blocks_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), copy_pairs, num_pairs, block_bytes / 16,
-        num_blocks, err_word);
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), copy_pairs, num_pairs, block_vecs, num_blocks,
+        err_word);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

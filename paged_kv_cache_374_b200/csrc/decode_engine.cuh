@@ -44,7 +44,8 @@ struct DecodeArgs {
     float* ws_m;      // [S*H][Pmax], base-2 units
     float* ws_l;      // [S*H][Pmax]
     float* ws_o;      // [S*H][Pmax][D]
-    int32_t* sched;   // [0] claim counter, [1] finished-warp counter; zero between launches
+    int32_t* sched;   // [0] claim counter, [1] finished-warp counter, [2] merge-queue length,
+                      // [3] engine-done flag, [4] finished merge CTAs; zero between launches
     int32_t* err_word;
     float scale_log2; // scale * log2(e)
     float k_scale;    // fp8 caches: K = code * k_scale (1 for 16-bit caches)
@@ -64,6 +65,19 @@ struct DecodeArgs {
     // seq_start[s] (a multiple of partition_tokens below context_lens[s]) are
     // already in the workspace (a shared prefix); this launch runs the rest.
     const int32_t* seq_start;
+    // Nonzero: launched as a programmatic dependent of the cache write of the same
+    // decode step, which may still be running.  The prologue and the first claims
+    // read only the lengths, tables and q, which that write does not touch; every
+    // warp waits for the write to complete before its first cache load.
+    int wait_prior;
+    // Nonzero (split partitions, no shared prefix): the merge kernel is launched
+    // right after this launch's prologue and merges each (s, h) as soon as its last
+    // partition lands.  merge_cnt[s*H + h] counts the partitions written;
+    // merge_queue lists the (s*H + h) + 1 of completed pairs in completion order.
+    // Both are left zero by the merge kernel.
+    int early_merge;
+    int32_t* merge_cnt;
+    int32_t* merge_queue;
 };
 
 enum UnitKind { kUnitNone = 0, kUnitNormal = 1, kUnitZero = 2, kUnitNaN = 3 };
@@ -350,6 +364,42 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
         ++issued;
     };
 
+    // The merge kernel may launch now: its CTAs take the SMs this grid's CTAs leave
+    // and merge each (s, h) when its partitions are complete.
+    if (a.early_merge) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (a.wait_prior) asm volatile("griddepcontrol.wait;" ::: "memory");  // the step's K/V are in the cache
+
+    // Early merge: the split units this warp finished (lane i holds the i-th, as
+    // s * unit_heads + head slot) are counted in batches, one fence per batch: all
+    // of the warp's partial stores, then one count per query head; the count that
+    // completes a head's partitions queues (s, h) for the merge.  A fence per unit
+    // would stall the warp's stream once per unit.
+    int fin = 0, nfin = 0;  // finished split units not yet counted
+    auto publish = [&]() {
+        __threadfence();
+        __syncwarp();
+        // the (unit, query head) counts spread over the lanes, so that their
+        // round trips overlap: item i is head i % heads_per_unit of unit i / heads_per_unit
+        const int hpu = a.heads_per_unit, items = nfin * hpu;
+        for (int i0 = 0; i0 < items; i0 += 32) {
+            const int i = i0 + lane;
+            const int e = i < items ? i / hpu : 0;
+            const int u = __shfl_sync(kFullMask, fin, e);
+            if (i < items) {
+                const int s = u / a.unit_heads, hs = u - s * a.unit_heads;
+                const int np = (s_len[s] + P - 1) / P;
+                const int sh = s * a.num_heads + hs * hpu + (i - e * hpu);
+                if (atomicAdd(a.merge_cnt + sh, 1) == np - 1) {
+                    const int slot = atomicAdd(a.sched + 2, 1);
+                    asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(a.merge_queue + slot), "r"(sh + 1)
+                                 : "memory");
+                }
+            }
+        }
+        __syncwarp();
+        nfin = 0;
+    };
+
     while (C.kind != kUnitNone && !aborted) {
         if (C.kind != kUnitNormal || C.nst == 0) {
             write_special_rows<Tag, D>(a, C, lane);
@@ -391,6 +441,11 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
             ++consumed;
             if (++cst < C.nst) continue;
             pol.finish(a, C);
+            if (a.early_merge && C.np > 1) {  // counted later, with one fence for many units
+                if (nfin == 32) publish();
+                if (lane == nfin) fin = C.s * a.unit_heads + C.h;
+                ++nfin;
+            }
         }
         // rotate: N becomes current; decode the pending claim as the new N
         const bool issue_was_in_next = in_next;
@@ -412,6 +467,7 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
         cst = 0;
     }
 
+    if (nfin > 0) publish();
     // never leave with copies into shared memory in flight
     for (uint32_t k = consumed; k < issued; ++k)
         if (!__all_sync(kFullMask, mbar_wait(&bars[k % R], (k / R) & 1)) && lane == 0)
@@ -419,6 +475,7 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
     // this warp writes nothing more: the merge kernel may be scheduled
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // the last warp of the launch to finish puts the claim counters back to zero
+    // and, with an early merge, tells the merge kernel that the queue is complete
     if (lane == 0) {
         __threadfence();
         const int total = (int)(gridDim.x * NW);
@@ -426,6 +483,12 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
             atomicExch(a.sched, 0);
             atomicExch(a.sched + 1, 0);
             __threadfence();
+            if (a.early_merge) {
+                // behind the shared-prefix kernel: its counts and queue entries are
+                // complete and visible once that grid is
+                if (a.seq_start) asm volatile("griddepcontrol.wait;" ::: "memory");
+                asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(a.sched + 3), "r"(1) : "memory");
+            }
         }
     }
     // Launched behind the shared-prefix kernel (programmatic dependent launch),

@@ -81,6 +81,27 @@ inline cudaError_t ensure_smem_limit(Kernel kernel, int bytes, std::atomic<uint6
     return e;
 }
 
+// The host-side checks of pa_decode, without its workspace arguments: a pa_status
+// (PA_OK with nothing to launch when num_seqs == 0, else the error pa_decode would
+// return) or -1 when the call may go on to launch.  Launches nothing.
+int check_decode_call(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      const int32_t* context_lens, int num_kv_heads, const void* out, int num_seqs, int num_heads,
+                      int head_dim, int block_size, int num_blocks, int max_blocks_per_seq, int dtype,
+                      int partition_tokens, const int32_t* err_word);
+
+// Bytes at the start of pa_decode's workspace that hold counters (zero before the
+// first call; every call leaves them zero again).
+size_t decode_counter_bytes(int num_seqs, int num_heads, int block_size, int max_blocks_per_seq, int partition_tokens);
+
+// K1's host checks (a pa_status, or -1 when it may launch) and its launch; the
+// launch assumes the checks passed.
+int check_reshape_and_cache(const void* k, const void* v, const int64_t* slot_mapping, const void* k_cache,
+                            const void* v_cache, int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                            int num_blocks, int dtype, const int32_t* err_word);
+int launch_reshape_and_cache(const void* k, const void* v, const int64_t* slot_mapping, void* k_cache,
+                             void* v_cache, int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                             int num_blocks, int32_t* err_word, cudaStream_t stream);
+
 // The prefix half of a two-level decode (paged_prefill.cu): partials of the
 // shared partitions of every group member, written into the decode workspace.
 struct SharedPrefixLaunch {
@@ -99,6 +120,13 @@ struct SharedPrefixLaunch {
     float scale;
     int num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype;
     int partition_tokens, num_partitions, num_groups, max_group_size, max_shared_tokens;
+    int num_seqs;  // bounds the group offsets and member indices
+    // early merge (see DecodeArgs): the prefix kernel counts the partitions it
+    // writes and queues the (s, h) it completes, as the decode engine does
+    int early_merge;
+    int32_t* sched;
+    int32_t* merge_cnt;
+    int32_t* merge_queue;
 };
 int launch_shared_prefix(const SharedPrefixLaunch& l, cudaStream_t stream);
 

@@ -58,19 +58,79 @@ namespace pa {
 // One CTA of 8 warps per (s, h), one pass over the partials: each warp takes
 // every 8th partition (each lane 4 dims, 16-byte loads, 4 partitions in flight)
 // and keeps its own running max, rescaling its sums when the max grows; the 8
-// warp results are combined with the same formula in shared memory.  Launched as
-// a programmatic dependent of K2: its blocks may start while K2's last CTAs
-// finish and wait (griddepcontrol.wait) until K2's writes are complete and visible.
+// warp results are combined with the same formula in shared memory.
+//
+// Launched as a programmatic dependent of K2, in one of two ways:
+//   - early merge (DecodeArgs::early_merge): K2 lets this grid launch right after
+//     its prologue, so its CTAs take the SMs K2's CTAs leave during K2's tail.
+//     CTA b merges the b-th (s, h) whose partitions all landed (K2's merge queue,
+//     in completion order), so merges overlap the partitions still streaming;
+//     Behind the shared-prefix kernel, that kernel counts and queues the prefix
+//     partitions it writes in the same way, and K2 raises its done flag only once
+//     that kernel is complete;
+//   - otherwise (a shared-prefix batch of more than one engine launch) every CTA
+//     waits (griddepcontrol.wait) until K2 and all it waits for are complete, and
+//     CTA b merges (s, h) = b.
 constexpr int kMergeThreads = 256;
 
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Early merge, thread 0: the (s*H + h) queued in slot b, or -1 when the queue ends
+// before slot b (or the wait gives up after about 2 s, reported as a timeout).
+__device__ __forceinline__ int merge_claim(const DecodeArgs& a, int b) {
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0;; ++i) {
+        int e = ld_acquire(a.merge_queue + b);
+        if (e) return e - 1;
+        if (ld_acquire(a.sched + 3)) {  // K2 is done: every entry it queued is visible
+            e = ld_acquire(a.merge_queue + b);
+            return e ? e - 1 : -1;
+        }
+        __nanosleep(256);
+        if ((i & 63u) == 63u && global_ns() - t0 > 2000000000ull) {
+            report(a.err_word, PA_DEVERR_TIMEOUT);
+            return -1;
+        }
+    }
+}
+
+// Early merge, thread 0, after the CTA's merge: the last CTA to get here waits for
+// K2's done flag, puts the queue state back to zero and does not let this grid
+// complete before K2 has.
+__device__ __forceinline__ void merge_retire(const DecodeArgs& a) {
+    __threadfence();
+    if (atomicAdd(a.sched + 4, 1) != (int)gridDim.x - 1) return;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0; !ld_acquire(a.sched + 3); ++i) {
+        __nanosleep(256);
+        if ((i & 63u) == 63u && global_ns() - t0 > 2000000000ull) {
+            report(a.err_word, PA_DEVERR_TIMEOUT);
+            return;
+        }
+    }
+    a.sched[2] = 0;
+    a.sched[3] = 0;
+    a.sched[4] = 0;
+    __threadfence();
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 template <class Tag, int D>
-__global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const DecodeArgs a) {
+__device__ __forceinline__ void merge_pair(const DecodeArgs& a, int64_t sh) {
     constexpr int NWM = kMergeThreads / 32;
     constexpr int BATCH = 4;
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     __shared__ float s_m[NWM], s_l[NWM];
     __shared__ float4 s_acc[NWM][D / 4];
-    const int64_t sh = blockIdx.x;
     const int s = (int)(sh / a.num_heads);
     const int L = a.context_lens[s];
     if (L <= 0 || L > a.max_blocks_per_seq * a.block_size) return;  // rows written by K2
@@ -91,9 +151,11 @@ __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const
         for (int j = 0; j < BATCH; ++j) {  // loads of BATCH partitions first
             const int p = p0 + j * NWM;
             const bool in = p < nparts;
-            mb[j] = in ? pm[p] : -INFINITY;
-            lb[j] = in ? pl[p] : 0.f;
-            ob[j] = (in && active) ? po[(int64_t)p * (D / 4) + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+            // L2 loads: with an early merge the partials were written by CTAs that ran
+            // beside this one
+            mb[j] = in ? __ldcg(pm + p) : -INFINITY;
+            lb[j] = in ? __ldcg(pl + p) : 0.f;
+            ob[j] = (in && active) ? __ldcg(po + (int64_t)p * (D / 4) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int j = 0; j < BATCH; ++j) {
@@ -145,6 +207,27 @@ __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const
     }
 }
 
+template <class Tag, int D>
+__global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const DecodeArgs a) {
+    if (!a.early_merge) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        merge_pair<Tag, D>(a, blockIdx.x);
+        return;
+    }
+    __shared__ int s_sh;
+    if (threadIdx.x == 0) s_sh = merge_claim(a, blockIdx.x);
+    __syncthreads();
+    const int sh = s_sh;
+    if (sh >= 0) {
+        merge_pair<Tag, D>(a, sh);
+        if (threadIdx.x == 0) {  // left zero for the next launch
+            a.merge_cnt[sh] = 0;
+            a.merge_queue[blockIdx.x] = 0;
+        }
+    }
+    if (threadIdx.x == 0) merge_retire(a);
+}
+
 namespace {
 
 constexpr int kDefaultPartition = PA_DECODE_PARTITION;
@@ -157,9 +240,18 @@ int64_t num_partitions(int max_blocks_per_seq, int block_size, int ptok) {
 
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Counters (left zero by every call) then partials:
+//   [0, 256)           scheduling counters (DecodeArgs::sched)
+//   when P > 1: merge_cnt int32 [S*H], merge_queue int32 [S*H], then the
+//   partials m, l fp32 [S*H][P] and o fp32 [S*H][P][D].
+size_t counter_bytes_for(int64_t sh, int64_t P) {
+    if (P <= 1) return kSchedBytes;
+    return kSchedBytes + 2 * up256(sh * 4);
+}
+
 size_t workspace_bytes_for(int64_t sh, int64_t P, int D) {
     if (P <= 1) return kSchedBytes;
-    return kSchedBytes + up256(sh * P * 4) * 2 + up256(sh * P * D * 4);
+    return counter_bytes_for(sh, P) + up256(sh * P * 4) * 2 + up256(sh * P * D * 4);
 }
 
 int sm_count() {
@@ -200,8 +292,9 @@ int launch_engine(DecodeArgs args, const void* k_cache, const void* v_cache, int
             c.ws_l += shoff * args.num_partitions;
             c.ws_o += shoff * args.num_partitions * D;
         }
-        if (c.seq_start && s0 == 0) {
-            // behind the shared-prefix kernel: start on the SMs it leaves free
+        if ((c.seq_start || c.wait_prior) && s0 == 0) {
+            // behind the shared-prefix kernel (start on the SMs it leaves free) or
+            // behind the step's cache write (overlap its launch and prologue)
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3((unsigned)sms);
             cfg.blockDim = dim3(NW * 32);
@@ -294,6 +387,13 @@ extern "C" int pa_decode_partition_tokens(int num_seqs, int num_heads, int num_k
     return pa::kDefaultPartition;
 }
 
+namespace pa {
+size_t decode_counter_bytes(int num_seqs, int num_heads, int block_size, int max_blocks_per_seq, int partition_tokens) {
+    const int ptok = partition_tokens > 0 ? partition_tokens : kDefaultPartition;
+    return counter_bytes_for((int64_t)num_seqs * num_heads, num_partitions(max_blocks_per_seq, block_size, ptok));
+}
+}  // namespace pa
+
 extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                            int block_size, int max_blocks_per_seq, int partition_tokens) {
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
@@ -353,9 +453,13 @@ int prepare_decode(DecodeArgs& args, const void* q, const void* k_cache, const v
     uint8_t* w = static_cast<uint8_t*>(workspace);
     args.sched = reinterpret_cast<int32_t*>(w);
     if (P > 1) {
-        args.ws_m = reinterpret_cast<float*>(w + kSchedBytes);
-        args.ws_l = reinterpret_cast<float*>(w + kSchedBytes + up256(SH * P * 4));
-        args.ws_o = reinterpret_cast<float*>(w + kSchedBytes + 2 * up256(SH * P * 4));
+        const size_t c0 = counter_bytes_for(SH, P);
+        args.merge_cnt = reinterpret_cast<int32_t*>(w + kSchedBytes);
+        args.merge_queue = reinterpret_cast<int32_t*>(w + kSchedBytes + up256(SH * 4));
+        args.ws_m = reinterpret_cast<float*>(w + c0);
+        args.ws_l = reinterpret_cast<float*>(w + c0 + up256(SH * P * 4));
+        args.ws_o = reinterpret_cast<float*>(w + c0 + 2 * up256(SH * P * 4));
+        args.early_merge = 1;  // cleared for the shared-prefix path
     }
     args.err_word = err_word;
     args.scale_log2 = scale * 1.4426950408889634f;
@@ -373,6 +477,20 @@ int prepare_decode(DecodeArgs& args, const void* q, const void* k_cache, const v
 }
 
 }  // namespace
+
+int check_decode_call(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      const int32_t* context_lens, int num_kv_heads, const void* out, int num_seqs, int num_heads,
+                      int head_dim, int block_size, int num_blocks, int max_blocks_per_seq, int dtype,
+                      int partition_tokens, const int32_t* err_word) {
+    // pa_decode's checks with a stand-in workspace that is present, aligned and
+    // large enough: no pointer is dereferenced and nothing is launched.
+    DecodeArgs args;
+    return prepare_decode(args, q, k_cache, v_cache, block_tables, context_lens, 1.f, num_kv_heads,
+                          const_cast<void*>(out), num_seqs, num_heads, head_dim, block_size, num_blocks,
+                          max_blocks_per_seq, dtype, partition_tokens, reinterpret_cast<void*>(uintptr_t{256}),
+                          SIZE_MAX, const_cast<int32_t*>(err_word));
+}
+
 }  // namespace pa
 
 extern "C" int pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
@@ -461,10 +579,46 @@ extern "C" int pa_decode_shared_prefix(const void* q, const void* k_cache, const
         l.num_groups = num_groups;
         l.max_group_size = max_group_size;
         l.max_shared_tokens = max_shared_tokens;
+        l.num_seqs = num_seqs;
+        // both kernels count partitions by (s, h) in one index space only when the
+        // engine runs in a single launch
+        args.early_merge = num_seqs <= kMaxSeqsPerLaunch ? 1 : 0;
+        l.early_merge = args.early_merge;
+        l.sched = args.sched;
+        l.merge_cnt = args.merge_cnt;
+        l.merge_queue = args.merge_queue;
         const int r = launch_shared_prefix(l, st);
         if (r != PA_OK) return r;
         args.seq_start = seq_start;
     }
+    if (head_dim == 128)
+        return dtype == PA_F16 ? launch_decode<F16Tag, 128>(args, k_cache, v_cache, num_kv_heads, st)
+                               : launch_decode<BF16Tag, 128>(args, k_cache, v_cache, num_kv_heads, st);
+    return dtype == PA_F16 ? launch_decode<F16Tag, 64>(args, k_cache, v_cache, num_kv_heads, st)
+                           : launch_decode<BF16Tag, 64>(args, k_cache, v_cache, num_kv_heads, st);
+}
+
+extern "C" int pa_decode_step(const void* k, const void* v, const int64_t* slot_mapping, const void* q,
+                              void* k_cache, void* v_cache, const int32_t* block_tables,
+                              const int32_t* context_lens, float scale, int num_kv_heads, void* out, int num_seqs,
+                              int num_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                              int dtype, int partition_tokens, void* workspace, size_t workspace_bytes,
+                              int32_t* err_word, void* stream) {
+    using namespace pa;
+    // every check of both calls before anything is launched
+    const int rk = check_reshape_and_cache(k, v, slot_mapping, k_cache, v_cache, num_seqs, num_kv_heads, head_dim,
+                                           block_size, num_blocks, dtype, err_word);
+    if (rk > 0) return rk;
+    DecodeArgs args;
+    const int rc = prepare_decode(args, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out,
+                                  num_seqs, num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype,
+                                  partition_tokens, workspace, workspace_bytes, err_word);
+    if (rc >= 0) return rc;  // an error, or an empty batch (num_seqs == 0: nothing to write either)
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int r1 = launch_reshape_and_cache(k, v, slot_mapping, k_cache, v_cache, num_seqs, num_kv_heads, head_dim,
+                                            block_size, num_blocks, err_word, st);
+    if (r1 != PA_OK) return r1;
+    args.wait_prior = 1;
     if (head_dim == 128)
         return dtype == PA_F16 ? launch_decode<F16Tag, 128>(args, k_cache, v_cache, num_kv_heads, st)
                                : launch_decode<BF16Tag, 128>(args, k_cache, v_cache, num_kv_heads, st);

@@ -43,9 +43,12 @@ extern "C" int pa_decode_noalloc(const void* q, const void* k_cache, const void*
                                  int num_kv_heads, void* out, int num_seqs, int num_heads, int head_dim,
                                  int block_size, int num_blocks, int max_blocks_per_seq, int dtype,
                                  int partition_tokens, int32_t* err_word, void* stream) {
-    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
-        max_blocks_per_seq < 0 || partition_tokens < 0)
-        return PA_ERR_INVALID_ARG;
+    // pa_decode's own checks first, so that errors (and the early PA_OK of an empty
+    // batch) are pa_decode's and nothing is queued on the stream for them
+    const int rc = pa::check_decode_call(q, k_cache, v_cache, block_tables, context_lens, num_kv_heads, out,
+                                         num_seqs, num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                                         dtype, partition_tokens, err_word);
+    if (rc >= 0) return rc;
     const size_t need = pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                                  max_blocks_per_seq, partition_tokens);
     if (need == 0) return PA_ERR_INVALID_ARG;
@@ -55,9 +58,11 @@ extern "C" int pa_decode_noalloc(const void* q, const void* k_cache, const void*
     void* scratch = scratch_address(dev);
     if (!scratch) return PA_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // The scratch keeps whatever the previous call left; the work-claim counters
-    // at its start must be zero when the kernels start.
-    if (cudaMemsetAsync(scratch, 0, 256, st) != cudaSuccess) return PA_ERR_CUDA;
+    // The scratch keeps whatever the previous call left; the counters at its start
+    // must be zero when the kernels start.
+    const size_t counters = pa::decode_counter_bytes(num_seqs, num_heads, block_size, max_blocks_per_seq,
+                                                     partition_tokens);
+    if (cudaMemsetAsync(scratch, 0, counters, st) != cudaSuccess) return PA_ERR_CUDA;
     return pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out, num_seqs,
                      num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype, partition_tokens,
                      scratch, (size_t)PA_DECODE_NOALLOC_SCRATCH_BYTES, err_word, stream);

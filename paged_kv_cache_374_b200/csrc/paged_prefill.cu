@@ -19,8 +19,9 @@
 //     softmax of tile j+1 overlaps the tensor core's work on tile j;
 //   - warps 0-3 own one query row per thread (tensor-memory lane = row): read
 //     S_j, apply the causal mask and the online softmax in base 2, write P_j over
-//     S_j as two 16-bit terms (hi + lo, about 16 significant bits, so the result
-//     keeps the decode path's accuracy), and at the end normalise O and store it.
+//     S_j (one f16 term for f16 inputs; for bf16, two terms hi + lo, about 16
+//     significant bits, so the result keeps the decode path's accuracy), and at
+//     the end normalise O and store it.
 // The running max used for the exponentials only moves when a row's max grows
 // by more than 2^8 (then O and the row sum are rescaled in tensor memory); the
 // result is the same softmax, p stays <= 256.  V rows past the sequence end are
@@ -88,9 +89,13 @@ __device__ __forceinline__ float tile_row_max(const float (&x)[kPfTok], int vis)
 }
 
 // p_t = 2^(x_t c - m) for the row's tile (0 past the diagonal when kDiag), written
-// to tensor memory at `taddr` as P_hi (columns 0-31) and P_lo (32-63), two tokens
-// per column; returns the sum of the fp32 p_t.  Packed fp32x2 arithmetic.
-template <class Tag, bool kDiag>
+// to tensor memory at `taddr` two tokens per column: P_hi in columns 0-31 and, when
+// kHiLo, P_lo = p - P_hi in columns 32-63.  Returns the sum of the weights the MMA
+// sees (P_hi + P_lo = p, or the rounded P_hi alone), so that the row's weights
+// always sum to its denominator.  Packed fp32x2 arithmetic.  p <= 256, so an f16
+// P_hi alone is within 2^-11 of p (the f16 path); a bf16 P_hi (2^-8) needs the lo
+// term to keep that accuracy.
+template <class Tag, bool kDiag, bool kHiLo>
 __device__ __forceinline__ float tile_row_p(const float (&x)[kPfTok], int vis, float c, float m, uint32_t taddr) {
     const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m), neg1 = make_float2(-1.f, -1.f);
     float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -106,13 +111,17 @@ __device__ __forceinline__ float tile_row_p(const float (&x)[kPfTok], int vis, f
                 p.x = t <= vis ? p.x : 0.f;
                 p.y = t + 1 <= vis ? p.y : 0.f;
             }
-            acc[k & 3] = __fadd2_rn(acc[k & 3], p);
             ph[k] = MmaOps<Tag>::pack(p.x, p.y);
-            const float2 lo = __ffma2_rn(Tag::widen2(ph[k]), neg1, p);  // p - hi, exact
-            pl[k] = MmaOps<Tag>::pack(lo.x, lo.y);
+            if (kHiLo) {
+                acc[k & 3] = __fadd2_rn(acc[k & 3], p);
+                const float2 lo = __ffma2_rn(Tag::widen2(ph[k]), neg1, p);  // p - hi, exact
+                pl[k] = MmaOps<Tag>::pack(lo.x, lo.y);
+            } else {
+                acc[k & 3] = __fadd2_rn(acc[k & 3], Tag::widen2(ph[k]));  // the rounded weights
+            }
         }
         umma::st16(taddr + 16 * half, ph);
-        umma::st16(taddr + 32 + 16 * half, pl);
+        if (kHiLo) umma::st16(taddr + 32 + 16 * half, pl);
     }
     acc[0] = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
     return acc[0].x + acc[0].y;
@@ -138,7 +147,27 @@ struct PrefillArgs {
     float* ws_l;
     float* ws_o;
     int partition_tokens, num_partitions, max_shared_partitions;
+    int num_seqs;  // shared-prefix mode: group offsets lie in [0, num_seqs], members in [0, num_seqs)
+    // shared-prefix mode with an early merge: count each partial written per (s, h)
+    // and queue the (s, h) whose partitions it completes (the decode engine counts
+    // the rest; the merge kernel reads the queue)
+    int early_merge;
+    int32_t* sched;
+    int32_t* merge_cnt;
+    int32_t* merge_queue;
 };
+
+// One partial of (seq, head) is in the workspace (this thread's stores fenced
+// first); the write that completes the sequence's partitions queues it.
+__device__ __forceinline__ void count_partial(const PrefillArgs& a, int seq, int head) {
+    __threadfence();
+    const int sh = seq * a.num_heads + head;
+    const int np = (a.context_lens[seq] + a.partition_tokens - 1) / a.partition_tokens;
+    if (atomicAdd(a.merge_cnt + sh, 1) == np - 1) {
+        const int slot = atomicAdd(a.sched + 2, 1);
+        asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(a.merge_queue + slot), "r"(sh + 1) : "memory");
+    }
+}
 
 template <int D>
 struct PfLayout {
@@ -172,6 +201,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
                                                                       const __grid_constant__ CUtensorMap vmap) {
     using Lay = PfLayout<D>;
     constexpr bool kBF16 = Tag::kIsBF16;
+    constexpr bool kHiLo = kBF16;  // P as hi + lo 16-bit terms (bf16), or one f16 term
     constexpr uint32_t kIdS = umma::idesc_f16(kBF16, false, kPfRows, kPfTok);
     constexpr uint32_t kIdO = umma::idesc_f16(kBF16, true, kPfRows, D);
     constexpr unsigned FULL = 0xffffffffu;
@@ -222,7 +252,20 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
         p = blockIdx.z - g * a.max_shared_partitions;
         kv_head = blockIdx.y;
         m0 = a.group_offsets[g];
-        const int rows = (a.group_offsets[g + 1] - m0) * a.group;
+        const int m1 = a.group_offsets[g + 1];
+        // the group's offsets and members come from the caller: a group that
+        // points outside the batch is skipped whole (every CTA of it agrees)
+        bool bad_group = m0 < 0 || m1 < m0 || m1 > a.num_seqs;
+        if (!bad_group)
+            for (int i = m0 + tid; i < m1; i += kPfThreads) {
+                const int mem = __ldg(a.group_members + i);
+                bad_group |= mem < 0 || mem >= a.num_seqs;
+            }
+        if (__syncthreads_or(bad_group)) {
+            if (tid == 0 && p == 0 && blockIdx.x == 0 && blockIdx.y == 0) report(a.err_word, PA_DEVERR_GROUP_RANGE);
+            return;
+        }
+        const int rows = (m1 - m0) * a.group;
         q_first = blockIdx.x * kPfRows;
         if (q_first >= rows) return;
         nrows = min(rows - q_first, kPfRows);
@@ -268,6 +311,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
                 const int64_t pi = ((int64_t)seq * a.num_heads + head) * a.num_partitions + p;
                 a.ws_m[pi] = __int_as_float(0x7fc00000);
                 a.ws_l[pi] = __int_as_float(0x7fc00000);
+                if (a.early_merge) count_partial(a, seq, head);  // merged, so the NaN reaches the row
             }
         }
         if (tid == 0) report(a.err_word, PA_DEVERR_TABLE_RANGE);
@@ -418,7 +462,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
                 for (int kk = 0; kk < kPfTok / 16; ++kk) {
                     const uint64_t db = bv + (uint64_t)(kk * (2048 >> 4));  // 16 tokens further
                     umma::mma_ts(tO, tp + kk * 8, db, kIdO, (j > 0 || kk > 0) ? 1u : 0u);  // P_hi V
-                    umma::mma_ts(tO, tp + 32 + kk * 8, db, kIdO, 1u);                      // P_lo V
+                    if (kHiLo) umma::mma_ts(tO, tp + 32 + kk * 8, db, kIdO, 1u);           // P_lo V
                 }
                 umma::commit(&bars[kBarVEmpty + st]);
                 umma::commit(&bars[kBarOFull + st]);
@@ -492,8 +536,8 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
                 }
                 m_used = m_new;
             }
-            l += diag ? tile_row_p<Tag, true>(x, vis, c, m_used, tS + b * 64 + lrow)
-                      : tile_row_p<Tag, false>(x, vis, c, m_used, tS + b * 64 + lrow);
+            l += diag ? tile_row_p<Tag, true, kHiLo>(x, vis, c, m_used, tS + b * 64 + lrow)
+                      : tile_row_p<Tag, false, kHiLo>(x, vis, c, m_used, tS + b * 64 + lrow);
             umma::wait_st();
             umma::fence_before_sync();
             mbar_arrive(&bars[kBarPFull + b]);
@@ -505,8 +549,8 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             umma::fence_after_sync();
             bool write = r < nrows;
             int64_t pi = 0;
+            int seq = 0, head = 0;
             if (write) {
-                int seq, head;
                 shared_row(r, seq, head);
                 const int Ls = a.context_lens[seq];
                 // a member must share the group's prefix length and extend past it
@@ -532,6 +576,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             if (write) {
                 a.ws_m[pi] = m_used;
                 a.ws_l[pi] = l;
+                if (a.early_merge) count_partial(a, seq, head);
             }
         } else if (ok) {
             umma::fence_after_sync();
@@ -632,6 +677,11 @@ int launch_shared_prefix(const SharedPrefixLaunch& l, cudaStream_t stream) {
     args.partition_tokens = l.partition_tokens;
     args.num_partitions = l.num_partitions;
     args.max_shared_partitions = (int)maxpp;
+    args.num_seqs = l.num_seqs;
+    args.early_merge = l.early_merge;
+    args.sched = l.sched;
+    args.merge_cnt = l.merge_cnt;
+    args.merge_queue = l.merge_queue;
     if (l.head_dim == 128)
         return l.dtype == PA_F16 ? launch_shared<F16Tag, 128>(args, l.k_cache, l.v_cache, l.num_kv_heads, l.num_groups,
                                                               l.max_group_size, stream)

@@ -74,10 +74,11 @@ def test_workspace_size_arithmetic():
     from paged_kv_cache_374_b200 import binding as pa
     # one partition: only the 256 bytes of scheduling counters
     assert pa.pa_decode_workspace_size(8, 32, 32, 128, 16, 4, 512) == 256
-    # 4096 tokens at 512 per partition: 8 partitions of (m, l, o[128]) per (s, h), 256-byte aligned pieces
+    # 4096 tokens at 512 per partition: a merge counter and a merge-queue entry per (s, h), then
+    # 8 partitions of (m, l, o[128]) per (s, h), in 256-byte aligned pieces
     n = pa.pa_decode_workspace_size(64, 32, 32, 128, 16, 256, 512)
     sh, p = 64 * 32, 8
     up = lambda x: (x + 255) // 256 * 256
-    assert n == 256 + 2 * up(sh * p * 4) + up(sh * p * 128 * 4)
+    assert n == 256 + 2 * up(sh * 4) + 2 * up(sh * p * 4) + up(sh * p * 128 * 4)
     assert pa.pa_decode_workspace_size(8, 32, 32, 128, 16, 4, 100) == 0   # bad partition size
     assert pa.pa_decode_partition_tokens(64, 32, 32, 128, 16, 256) % 64 == 0

@@ -157,3 +157,63 @@ def test_bounded_wait_gives_up_and_reports():
     assert outcome.item() == 0 and err.item() == pa.PA_DEVERR_TIMEOUT
     c = PagedCase(np.random.default_rng(80), [100, 300], 4, 4, 128, 16, F16, 0.1)
     assert_close(run_case(c), c.run(oracle_pkg.get()), "f16", "decode after the self-test")
+
+
+@pytest.mark.parametrize("mode", ["mha", "gqa", "fp8", "shared_prefix"])
+def test_many_calls_on_one_workspace_leave_the_counters_zero(mode):
+    """Decode calls in a row on one workspace, with split contexts: the merge of
+    each (sequence, head) runs in the engine's tail from a completion queue whose
+    counters live at the start of the workspace.  Every call must leave them zero
+    (the next call starts from them) and give the same output bit for bit, which
+    must match the oracle."""
+    rng = np.random.default_rng(35)
+    lens = [700, 2100, 257, 1024, 33, 1500, 513, 3000]
+    g = 4 if mode == "gqa" else 1
+    hk = 2 if mode == "gqa" else 4
+    c = PagedCase(rng, lens, hk * g, hk, 128, 16, BF16 if mode == "gqa" else F16, 1 / math.sqrt(128))
+    if mode == "shared_prefix":
+        members, nb = [1, 3, 5, 7], 512 // 16
+        for s in members[1:]:
+            c.tables[s, :nb] = c.tables[1, :nb]
+            c.seq_k[s][:512] = c.seq_k[1][:512]
+            c.seq_v[s][:512] = c.seq_v[1][:512]
+        c._assemble()
+    P = 256
+    s_, h_ = c.S, c.H
+    need = pa.pa_decode_workspace_size(s_, h_, hk, 128, 16, c.MB, P)
+    up = lambda x: (x + 255) // 256 * 256
+    counters = 256 + 2 * up(s_ * h_ * 4)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    q = dev(c.q, c.dtype)
+    tb, ln = torch.from_numpy(c.tables).cuda(), torch.from_numpy(c.lens).cuda()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if mode == "fp8":
+        codes = lambda bits: (torch.from_numpy(bits.view(np.int16)).view(torch.float16).float() * 32).clamp(
+            -448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+        kc, vc = codes(c.k_cache).cuda(), codes(c.v_cache).cuda()
+        call = lambda out: pa.pa_decode_fp8(q, kc, vc, tb, ln, c.scale, 1 / 32, 1 / 32, hk, out, workspace=ws,
+                                            partition_tokens=P, err_word=err)
+        ref = oracle_pkg.get().decode_fp8(c.q, kc.cpu().numpy(), vc.cpu().numpy(), c.tables, c.lens, c.scale,
+                                          1 / 32, 1 / 32, F16, nthreads=8)
+    else:
+        kc, vc = dev(c.k_cache, c.dtype), dev(c.v_cache, c.dtype)
+        if mode == "shared_prefix":
+            grp = pa.pa_find_shared_prefixes(c.tables, c.lens, c.bs, P)
+            assert grp.num_groups == 1 and grp.max_shared_tokens == 512
+            start, offs, mem = grp.to("cuda")
+            call = lambda out: pa.pa_decode_shared_prefix(q, kc, vc, tb, ln, c.scale, hk, out, start, offs, mem,
+                                                          grp.num_groups, grp.max_group_size, grp.max_shared_tokens,
+                                                          workspace=ws, partition_tokens=P, err_word=err)
+        else:
+            call = lambda out: pa.pa_decode(q, kc, vc, tb, ln, c.scale, hk, out, workspace=ws, partition_tokens=P,
+                                            err_word=err)
+        ref = c.run(oracle_pkg.get(), nthreads=8)
+    outs = [torch.full_like(q, float("nan")) for _ in range(40)]
+    for out in outs:
+        call(out)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert int(ws[:counters].count_nonzero()) == 0
+    for out in outs[1:]:
+        assert torch.equal(out, outs[0])
+    assert_close(outs[0], ref, WK[c.dtype], mode)
