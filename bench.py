@@ -339,16 +339,22 @@ class Ops:
 
     @property
     def fused(self):
-        """One pa_decode_step call per step (16-bit cache, no shared-prefix groups)."""
-        return not self.fp8 and self.st["groups"] is None
+        """One pa_decode_step(_fp8) call per step (no shared-prefix groups)."""
+        return self.st["groups"] is None
 
     def step(self, k, v, slots, q, tables, lens, groups=None, out=None):
         if self.fused:
             st = self.st
-            self.pa.pa_decode_step(k, v, slots, q, st["k_cache"], st["v_cache"], tables, lens, st["spec"].scale,
-                                   st["spec"].num_kv_heads, st["out"] if out is None else out,
-                                   workspace=st["workspace"], partition_tokens=st["partition_tokens"],
-                                   stream=self.stream)
+            out = st["out"] if out is None else out
+            if self.fp8:
+                self.pa.pa_decode_step_fp8(k, v, slots, q, st["k_cache"], st["v_cache"], tables, lens,
+                                           st["spec"].scale, self.ks, self.vs, st["spec"].num_kv_heads, out,
+                                           workspace=st["workspace"], partition_tokens=st["partition_tokens"],
+                                           stream=self.stream)
+            else:
+                self.pa.pa_decode_step(k, v, slots, q, st["k_cache"], st["v_cache"], tables, lens, st["spec"].scale,
+                                       st["spec"].num_kv_heads, out, workspace=st["workspace"],
+                                       partition_tokens=st["partition_tokens"], stream=self.stream)
         else:
             self.k1(k, v, slots)
             self.k2(q, tables, lens, groups, out)
@@ -519,8 +525,9 @@ def roofline_leg(ops, ab, t, steps):
 
 def roofline_kernel(ops):
     if ops.fused:
-        return ("reshape_and_cache_kernel + paged_decode_kernel + paged_decode_merge_kernel (one pa_decode_step "
-                "call: K2 a programmatic dependent of K1)")
+        call = "pa_decode_step_fp8" if ops.fp8 else "pa_decode_step"
+        return ("reshape_and_cache_kernel + paged_decode_kernel + paged_decode_merge_kernel (one %s call: K2 a "
+                "programmatic dependent of K1)" % call)
     if ops.st["groups"] is not None:
         return ("shared-prefix kernel + paged_decode_kernel + paged_decode_merge_kernel (timed together: one "
                 "pa_decode_shared_prefix call)")

@@ -322,6 +322,21 @@ int pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const
                   int dtype, int partition_tokens, void* workspace, size_t workspace_bytes, int32_t* err_word,
                   void* stream);
 
+/*
+ * pa_decode_step_fp8 -- pa_decode_step over fp8 caches: exactly
+ *     pa_reshape_and_cache_fp8(k, v, slot_mapping, ..., num_tokens = num_seqs, ...)
+ *     pa_decode_fp8(q, ...)
+ * in one call, the attention launched as a programmatic dependent of the cache
+ * write as in pa_decode_step.  Arguments as those two calls; the checks of both
+ * run before anything is launched.
+ */
+int pa_decode_step_fp8(const void* k, const void* v, const int64_t* slot_mapping, const void* q, void* k_cache,
+                       void* v_cache, const int32_t* block_tables, const int32_t* context_lens, float scale,
+                       float k_scale, float v_scale, int num_kv_heads, void* out, int num_seqs, int num_heads,
+                       int head_dim, int block_size, int num_blocks, int max_blocks_per_seq, int dtype,
+                       int partition_tokens, void* workspace, size_t workspace_bytes, int32_t* err_word,
+                       void* stream);
+
 /* ----------------------------------------------------------------- prefill */
 
 /*

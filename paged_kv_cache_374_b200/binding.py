@@ -47,6 +47,8 @@ _sig("pa_decode", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32
      _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
 _sig("pa_decode_step", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32, _i32, _i32,
      _i32, _i32, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
+_sig("pa_decode_step_fp8", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float,
+     ctypes.c_float, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
 _sig("pa_decode_noalloc", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32, _i32, _i32, _i32, _i32,
      _i32, _i32, _i32, _vp, _vp)
 _sig("pa_reshape_and_cache_fp8", _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_float,
@@ -224,6 +226,41 @@ def pa_decode_step(k, v, slot_mapping, q, k_cache, v_cache, block_tables, contex
                              workspace.numel() * workspace.element_size(), _dev(err_word, "err_word", torch.int32),
                              _stream(stream, q))
     _check(st, "pa_decode_step")
+    return out
+
+
+def pa_decode_step_fp8(k, v, slot_mapping, q, k_cache, v_cache, block_tables, context_lens, scale, k_scale,
+                       v_scale, num_kv_heads, out, workspace=None, partition_tokens=0, err_word=None, stream=None):
+    """pa_decode_step over uint8 E4M3 caches: the fp8 cache write then pa_decode_fp8,
+    in one call.  Returns ``out``."""
+    import torch
+    s, h, d = q.shape
+    nb, bs, hk, d2 = k_cache.shape
+    if hk != num_kv_heads or d2 != d or v_cache.shape != k_cache.shape or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if k.shape != (s, hk, d) or v.shape != k.shape or slot_mapping.shape != (s,):
+        raise ValueError("k, v must be [S, Hk, d] and slot_mapping [S]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [S, MB] and context_lens [S]")
+    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+        raise TypeError("fp8 caches are uint8 E4M3 codes")
+    for t in (k, v, out):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v and out must share one dtype")
+    mb = block_tables.shape[1]
+    need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = _lib.pa_decode_step_fp8(_dev(k, "k"), _dev(v, "v"), _dev(slot_mapping, "slot_mapping", torch.int64),
+                                 _dev(q, "q"), _dev(k_cache, "k_cache", torch.uint8),
+                                 _dev(v_cache, "v_cache", torch.uint8),
+                                 _dev(block_tables, "block_tables", torch.int32),
+                                 _dev(context_lens, "context_lens", torch.int32), float(scale), float(k_scale),
+                                 float(v_scale), hk, _dev(out, "out"), s, h, d, bs, nb, mb, _dtype_code(q),
+                                 int(partition_tokens), _dev(workspace, "workspace"),
+                                 workspace.numel() * workspace.element_size(), _dev(err_word, "err_word", torch.int32),
+                                 _stream(stream, q))
+    _check(st, "pa_decode_step_fp8")
     return out
 
 

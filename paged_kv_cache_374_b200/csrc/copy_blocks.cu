@@ -11,67 +11,80 @@
 
 namespace pa {
 
-// The (pair, 16-byte vector) space of all pairs is cut into one contiguous,
-// equal slice per CTA (every CTA resident at once, no tail wave); a CTA walks its
-// slice pair by pair.  The pairs are copied all at once, so a pair that overlaps
-// another copying pair -- its destination is another's destination or source, or
-// its source is another's destination -- is skipped and reported: a CTA checks
-// each pair its slice touches against the whole list (num_pairs comparisons
-// spread over its threads).  Pairs that copy nothing (ids out of range, source ==
-// destination) conflict with nothing.
-__global__ void __launch_bounds__(256, 4) copy_blocks_kernel(uint4* __restrict__ k_cache,
-                                                              uint4* __restrict__ v_cache,
-                                                              const int32_t* __restrict__ pairs, int num_pairs,
-                                                              int64_t block_vecs, int num_blocks, int32_t* err_word) {
-    constexpr int U = 4;  // 16-byte vectors in flight per thread and cache
-    const int64_t total = (int64_t)num_pairs * block_vecs;
-    const int64_t per = (total + gridDim.x - 1) / gridDim.x;
-    int64_t lo = (int64_t)blockIdx.x * per;
-    const int64_t hi = lo + per < total ? lo + per : total;
-    while (lo < hi) {
-        const int64_t pi = lo / block_vecs;
-        const int64_t c0 = lo - pi * block_vecs;
-        const int64_t c1 = c0 + (hi - lo) < block_vecs ? c0 + (hi - lo) : block_vecs;
-        lo += c1 - c0;
-        const int32_t src = __ldg(pairs + 2 * pi), dst = __ldg(pairs + 2 * pi + 1);
+// The pairs' blocks are cut into chunks of kChunk 16-byte vectors, in pair order,
+// and the CTAs walk them grid-stride, so that at any time they copy one window of
+// consecutive chunks (the source blocks are read in the pairs' order).  The pairs
+// are copied all at once, so a pair that overlaps another copying pair -- its
+// destination is another's destination or source, or its source is another's
+// destination -- is skipped and reported: each chunk's CTA checks its pair
+// against the whole list, held in shared memory when it fits (kStagedPairs).
+// Pairs that copy nothing (ids out of range, source == destination) conflict
+// with nothing.
+constexpr int kCopyThreads = 256;
+constexpr int kCopyUnroll = 4;                              // vectors in flight per thread and cache
+constexpr int kChunk = kCopyThreads * kCopyUnroll;          // 16 KiB of each cache
+constexpr int kStagedPairs = 2048;                          // 16 KiB of shared memory
+
+__device__ __forceinline__ bool copies(int32_t s, int32_t d, int num_blocks) {
+    return s >= 0 && s < num_blocks && d >= 0 && d < num_blocks && s != d;
+}
+
+__global__ void __launch_bounds__(kCopyThreads, 4) copy_blocks_kernel(uint4* __restrict__ k_cache,
+                                                                       uint4* __restrict__ v_cache,
+                                                                       const int32_t* __restrict__ pairs,
+                                                                       int num_pairs, int64_t block_vecs,
+                                                                       int num_blocks, int32_t* err_word) {
+    __shared__ int2 s_pairs[kStagedPairs];
+    const bool staged = num_pairs <= kStagedPairs;
+    if (staged)
+        for (int j = threadIdx.x; j < num_pairs; j += kCopyThreads)
+            s_pairs[j] = make_int2(__ldg(pairs + 2 * j), __ldg(pairs + 2 * j + 1));
+    __syncthreads();
+    const int64_t per_pair = (block_vecs + kChunk - 1) / kChunk;
+    const int64_t chunks = (int64_t)num_pairs * per_pair;
+    for (int64_t w = blockIdx.x; w < chunks; w += gridDim.x) {
+        const int pi = (int)(w / per_pair);
+        const int64_t c0 = (w - (int64_t)pi * per_pair) * kChunk;
+        const int n = (int)(block_vecs - c0 < kChunk ? block_vecs - c0 : kChunk);
+        const int2 me = staged ? s_pairs[pi] : make_int2(__ldg(pairs + 2 * (int64_t)pi), __ldg(pairs + 2 * (int64_t)pi + 1));
+        const int32_t src = me.x, dst = me.y;
         if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
             if (c0 == 0 && threadIdx.x == 0) report(err_word, PA_DEVERR_TABLE_RANGE);
             continue;
         }
         if (src == dst) continue;
+        // the CTA's threads split the scan (a per-warp scan, without the barrier,
+        // measured slower: every warp repeats the whole list)
         bool conflict = false;
-        for (int j = threadIdx.x; j < num_pairs; j += blockDim.x) {
-            const int32_t sj = __ldg(pairs + 2 * (int64_t)j), dj = __ldg(pairs + 2 * (int64_t)j + 1);
-            if (j == pi || sj == dj || sj < 0 || sj >= num_blocks || dj < 0 || dj >= num_blocks) continue;
-            conflict |= dj == dst || sj == dst || dj == src;
+        for (int j = threadIdx.x; j < num_pairs; j += kCopyThreads) {
+            const int2 o = staged ? s_pairs[j]
+                                  : make_int2(__ldg(pairs + 2 * (int64_t)j), __ldg(pairs + 2 * (int64_t)j + 1));
+            if (j == pi || !copies(o.x, o.y, num_blocks)) continue;
+            conflict |= o.y == dst || o.x == dst || o.y == src;
         }
         if (__syncthreads_or(conflict)) {
             if (c0 == 0 && threadIdx.x == 0) report(err_word, PA_DEVERR_PAIR_CONFLICT);
             continue;
         }
-        // this slice's part of the pair: n vectors from c0 (a block is far below 2^31 vectors)
-        const int n = (int)(c1 - c0);
         const uint4* ks = k_cache + (int64_t)src * block_vecs + c0;
         const uint4* vs = v_cache + (int64_t)src * block_vecs + c0;
         uint4* kd = k_cache + (int64_t)dst * block_vecs + c0;
         uint4* vd = v_cache + (int64_t)dst * block_vecs + c0;
-        for (int i = threadIdx.x; i < n; i += 256 * U) {
-            uint4 a[U], b[U];
+        uint4 a[kCopyUnroll], b[kCopyUnroll];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int j = i + u * 256;
-                if (j < n) {
-                    a[u] = __ldcs(ks + j);
-                    b[u] = __ldcs(vs + j);
-                }
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int j = threadIdx.x + u * kCopyThreads;
+            if (j < n) {
+                a[u] = __ldcs(ks + j);
+                b[u] = __ldcs(vs + j);
             }
+        }
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int j = i + u * 256;
-                if (j < n) {
-                    kd[j] = a[u];
-                    vd[j] = b[u];
-                }
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int j = threadIdx.x + u * kCopyThreads;
+            if (j < n) {
+                kd[j] = a[u];
+                vd[j] = b[u];
             }
         }
     }
@@ -142,20 +155,20 @@ extern "C" int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* copy_
         return PA_ERR_INVALID_ARG;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // every CTA resident at once (as many per SM as fit), each with a slice of at
-    // least 1024 vectors (16 KiB per cache)
+    // as many CTAs as are resident at once; they stride over the chunks
     static std::atomic<int> per_sm{0};
     if (per_sm.load(std::memory_order_relaxed) == 0) {
         int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, copy_blocks_kernel, 256, 0) != cudaSuccess || n < 1)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, copy_blocks_kernel, kCopyThreads, 0) != cudaSuccess ||
+            n < 1)
             return PA_ERR_CUDA;
         per_sm.store(n, std::memory_order_relaxed);
     }
     const int64_t block_vecs = block_bytes / 16;
     const int64_t target = (int64_t)sms * per_sm.load(std::memory_order_relaxed);
-    const int64_t slices = ((int64_t)num_pairs * block_vecs + 1023) / 1024;
-    const int64_t blocks = slices < target ? slices : target;
-    copy_blocks_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+    const int64_t chunks = (int64_t)num_pairs * ((block_vecs + kChunk - 1) / kChunk);
+    const int64_t blocks = chunks < target ? chunks : target;
+    copy_blocks_kernel<<<(unsigned)blocks, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), copy_pairs, num_pairs, block_vecs, num_blocks,
         err_word);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;

@@ -136,8 +136,84 @@ struct Fp8TcPolicy {
 
     __device__ __forceinline__ void poison() { poisoned = true; }
 
+    // q K^T of one 16-token tile (rows g and g+8 of the codes at kr) into x, two
+    // accumulators (even and odd k-steps) halving the chain of dependent MMAs
+    __device__ __forceinline__ void scores(const uint8_t* kr, float (&x)[NT][4]) const {
+        const uint4 k0a = lds128(kr + g * 128 + (((2 * t) ^ g) << 4));
+        const uint4 k0b = lds128(kr + g * 128 + (((2 * t + 1) ^ g) << 4));
+        const uint4 k1a = lds128(kr + (g + 8) * 128 + (((2 * t) ^ g) << 4));
+        const uint4 k1b = lds128(kr + (g + 8) * 128 + (((2 * t + 1) ^ g) << 4));
+        const uint32_t kw0[8] = {k0a.x, k0a.y, k0a.z, k0a.w, k0b.x, k0b.y, k0b.z, k0b.w};  // token g
+        const uint32_t kw1[8] = {k1a.x, k1a.y, k1a.z, k1a.w, k1b.x, k1b.y, k1b.z, k1b.w};  // token g+8
+        float y[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) x[nt][j] = y[nt][j] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            uint32_t af[4];
+            af[0] = e4m3x2_to_f16x2(kw0[ks] & 0xffffu);
+            af[1] = e4m3x2_to_f16x2(kw1[ks] & 0xffffu);
+            af[2] = e4m3x2_to_f16x2(kw0[ks] >> 16);
+            af[3] = e4m3x2_to_f16x2(kw1[ks] >> 16);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) Ops::mma((ks & 1) ? y[nt] : x[nt], af, qb[nt][ks][0], qb[nt][ks][1]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) x[nt][j] += y[nt][j];
+    }
+
+    // O^T += V^T P^T for one 16-token tile (codes at vr, nv valid tokens)
+    __device__ __forceinline__ void values(const uint8_t* vr, int nv, const uint32_t (&bhi)[NT][2],
+                                           const uint32_t (&blo)[NT][2]) {
+        const uint4 r0 = lds128(vr + (2 * t) * 128 + ((g ^ (2 * t)) << 4));
+        const uint4 r1 = lds128(vr + (2 * t + 1) * 128 + ((g ^ (2 * t + 1)) << 4));
+        const uint4 r8 = lds128(vr + (2 * t + 8) * 128 + ((g ^ (2 * t)) << 4));
+        const uint4 r9 = lds128(vr + (2 * t + 9) * 128 + ((g ^ (2 * t + 1)) << 4));
+        const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
+        const uint32_t w8[4] = {r8.x, r8.y, r8.z, r8.w}, w9[4] = {r9.x, r9.y, r9.z, r9.w};
+        const uint32_t mask01 = gqa_pair_mask(2 * t, nv), mask89 = gqa_pair_mask(2 * t + 8, nv);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+            const uint32_t p01 = byte_perm(w0[mt >> 1], w1[mt >> 1], sel);
+            const uint32_t p89 = byte_perm(w8[mt >> 1], w9[mt >> 1], sel);
+            uint32_t af[4];
+            af[0] = e4m3x2_to_f16x2(p01 & 0xffffu);
+            af[1] = e4m3x2_to_f16x2(p01 >> 16);
+            af[2] = e4m3x2_to_f16x2(p89 & 0xffffu);
+            af[3] = e4m3x2_to_f16x2(p89 >> 16);
+            if (nv < 16) {
+                af[0] &= mask01;
+                af[1] &= mask01;
+                af[2] &= mask89;
+                af[3] &= mask89;
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                Ops::mma(o[nt][mt], af, bhi[nt][0], bhi[nt][1]);
+                Ops::mma(o[nt][mt], af, blo[nt][0], blo[nt][1]);
+            }
+        }
+    }
+
     __device__ __forceinline__ void stage(const DecodeArgs& a, const uint8_t* kt, const uint8_t* vt, int ntok) {
         const float sc = a.scale_log2 * a.k_scale * qinv;
+        if (NTT == 2 && ntok > 16) {
+            // both 16-token tiles of the stage together: two independent score chains,
+            // one softmax step over the 32 tokens, then both P.V products
+            float xa[NT][4], xb[NT][4];
+            scores(kt, xa);
+            scores(kt + 2048, xb);
+            uint32_t bhi[2][NT][2], blo[2][NT][2];
+            gqa_softmax_2tiles<F16Tag>(xa, xb, g, 16, ntok - 16, sc, m, lsum, o, bhi, blo);
+            values(vt, 16, bhi[0], blo[0]);
+            values(vt + 2048, ntok - 16, bhi[1], blo[1]);
+            return;
+        }
 #pragma unroll
         for (int tt = 0; tt < NTT; ++tt) {
             const int nv = ntok - tt * 16;  // valid tokens in this tile (warp-uniform)

@@ -135,6 +135,71 @@ __device__ __forceinline__ void gqa_softmax_tile(float (&x)[NT][4], int g, int n
     }
 }
 
+// The same step over two 16-token tiles at once (tokens g, g+8 of tile A in xa,
+// of tile B in xb; nva, nvb valid tokens): one max update and one rescale for the
+// 32 tokens, then P^T fragments for both tiles.  The result is the online
+// softmax of the two tiles taken in one step (the same softmax up to rounding).
+template <class P, int NT, int MT>
+__device__ __forceinline__ void gqa_softmax_2tiles(float (&xa)[NT][4], float (&xb)[NT][4], int g, int nva, int nvb,
+                                                   float sc, float (&m)[NT][2], float (&lsum)[NT][2],
+                                                   float (&o)[NT][MT][4], uint32_t (&bhi)[2][NT][2],
+                                                   uint32_t (&blo)[2][NT][2]) {
+    bool up = false;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            xa[nt][j] *= sc;
+            xb[nt][j] *= sc;
+        }
+        if (!(g < nva)) xa[nt][0] = xa[nt][1] = -INFINITY;
+        if (!(g + 8 < nva)) xa[nt][2] = xa[nt][3] = -INFINITY;
+        if (!(g < nvb)) xb[nt][0] = xb[nt][1] = -INFINITY;
+        if (!(g + 8 < nvb)) xb[nt][2] = xb[nt][3] = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+            up |= fmaxf(fmaxf(xa[nt][j], xa[nt][j + 2]), fmaxf(xb[nt][j], xb[nt][j + 2])) > m[nt][j];
+    }
+    if (__any_sync(kFullMask, up)) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                float mx = fmaxf(fmaxf(xa[nt][j], xa[nt][j + 2]), fmaxf(xb[nt][j], xb[nt][j + 2]));
+                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 16));
+                const float m_new = fmaxf(m[nt][j], mx);
+                const float alpha = fast_exp2(m[nt][j] - m_new);
+                lsum[nt][j] *= alpha;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    o[nt][mt][j] *= alpha;
+                    o[nt][mt][j + 2] *= alpha;
+                }
+                m[nt][j] = m_new;
+            }
+    }
+#pragma unroll
+    for (int tile = 0; tile < 2; ++tile)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float p[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) p[j] = fast_exp2((tile ? xb : xa)[nt][j] - m[nt][j & 1]);
+            lsum[nt][0] += p[0] + p[2];
+            lsum[nt][1] += p[1] + p[3];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const uint32_t hi = MmaOps<P>::pack(p[2 * half], p[2 * half + 1]);
+                const float2 hv = P::widen2(hi);
+                const uint32_t lo = MmaOps<P>::pack(p[2 * half] - hv.x, p[2 * half + 1] - hv.y);
+                bhi[tile][nt][half] = movmatrix_trans(hi);
+                blo[tile][nt][half] = movmatrix_trans(lo);
+            }
+        }
+}
+
 // Keep-mask of a 16-bit pair holding tokens k and k+1 of a tile with nv valid
 // tokens.  Rows past the sequence end may hold anything (NaN included): their p
 // is 0, but 0 * NaN is NaN inside the MMA, so their V entries are zeroed.

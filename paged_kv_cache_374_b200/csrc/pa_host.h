@@ -89,6 +89,15 @@ int check_decode_call(const void* q, const void* k_cache, const void* v_cache, c
                       int head_dim, int block_size, int num_blocks, int max_blocks_per_seq, int dtype,
                       int partition_tokens, const int32_t* err_word);
 
+// The same for the fp8 cache write (pa_reshape_and_cache_fp8).
+int check_reshape_and_cache_fp8(const void* k, const void* v, const int64_t* slot_mapping, const void* k_cache,
+                                const void* v_cache, int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                                int num_blocks, int dtype, float k_scale, float v_scale, const int32_t* err_word);
+int launch_reshape_and_cache_fp8(const void* k, const void* v, const int64_t* slot_mapping, void* k_cache,
+                                 void* v_cache, int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                                 int num_blocks, int dtype, float k_scale, float v_scale, int32_t* err_word,
+                                 cudaStream_t st);
+
 // Bytes at the start of pa_decode's workspace that hold counters (zero before the
 // first call; every call leaves them zero again).
 size_t decode_counter_bytes(int num_seqs, int num_heads, int block_size, int max_blocks_per_seq, int partition_tokens);

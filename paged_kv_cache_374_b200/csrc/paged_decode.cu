@@ -625,3 +625,32 @@ extern "C" int pa_decode_step(const void* k, const void* v, const int64_t* slot_
     return dtype == PA_F16 ? launch_decode<F16Tag, 64>(args, k_cache, v_cache, num_kv_heads, st)
                            : launch_decode<BF16Tag, 64>(args, k_cache, v_cache, num_kv_heads, st);
 }
+
+extern "C" int pa_decode_step_fp8(const void* k, const void* v, const int64_t* slot_mapping, const void* q,
+                                  void* k_cache, void* v_cache, const int32_t* block_tables,
+                                  const int32_t* context_lens, float scale, float k_scale, float v_scale,
+                                  int num_kv_heads, void* out, int num_seqs, int num_heads, int head_dim,
+                                  int block_size, int num_blocks, int max_blocks_per_seq, int dtype,
+                                  int partition_tokens, void* workspace, size_t workspace_bytes, int32_t* err_word,
+                                  void* stream) {
+    using namespace pa;
+    if (head_dim != 128) return PA_ERR_UNSUPPORTED;
+    const int rk = check_reshape_and_cache_fp8(k, v, slot_mapping, k_cache, v_cache, num_seqs, num_kv_heads,
+                                               head_dim, block_size, num_blocks, dtype, k_scale, v_scale, err_word);
+    if (rk > 0) return rk;
+    DecodeArgs args;
+    const int rc = prepare_decode(args, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out,
+                                  num_seqs, num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype,
+                                  partition_tokens, workspace, workspace_bytes, err_word);
+    if (rc >= 0) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int r1 = launch_reshape_and_cache_fp8(k, v, slot_mapping, k_cache, v_cache, num_seqs, num_kv_heads,
+                                                head_dim, block_size, num_blocks, dtype, k_scale, v_scale, err_word,
+                                                st);
+    if (r1 != PA_OK) return r1;
+    args.k_scale = k_scale;
+    args.v_scale = v_scale;
+    args.wait_prior = 1;
+    return dtype == PA_F16 ? launch_decode_fp8<F16Tag>(args, k_cache, v_cache, num_kv_heads, st)
+                           : launch_decode_fp8<BF16Tag>(args, k_cache, v_cache, num_kv_heads, st);
+}

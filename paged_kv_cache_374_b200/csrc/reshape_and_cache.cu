@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(const uint4*
                                                                      uint4* __restrict__ v_cache, int num_tokens,
                                                                      int row_vecs, int64_t num_slots, float k_scale,
                                                                      float v_scale, int32_t* err_word) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // as the 16-bit kernel
     const int64_t total = (int64_t)num_tokens * row_vecs;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
@@ -87,11 +88,11 @@ __global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(const uint4*
 
 }  // namespace pa
 
-extern "C" int pa_reshape_and_cache_fp8(const void* k, const void* v, const int64_t* slot_mapping, void* k_cache,
-                                        void* v_cache, int num_tokens, int num_kv_heads, int head_dim,
-                                        int block_size, int num_blocks, int dtype, float k_scale, float v_scale,
-                                        int32_t* err_word, void* stream) {
-    using namespace pa;
+namespace pa {
+
+int check_reshape_and_cache_fp8(const void* k, const void* v, const int64_t* slot_mapping, const void* k_cache,
+                                const void* v_cache, int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                                int num_blocks, int dtype, float k_scale, float v_scale, const int32_t* err_word) {
     if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks < 0)
         return PA_ERR_INVALID_ARG;
     if (!(k_scale > 0.f) || !(v_scale > 0.f) || !isfinite(k_scale) || !isfinite(v_scale)) return PA_ERR_INVALID_ARG;
@@ -102,15 +103,20 @@ extern "C" int pa_reshape_and_cache_fp8(const void* k, const void* v, const int6
     if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
         (reinterpret_cast<uintptr_t>(slot_mapping) & 7u) || (err_word && !aligned4(err_word)))
         return PA_ERR_INVALID_ARG;
-    const int64_t row_vecs64 = (int64_t)num_kv_heads * head_dim / 16;
-    if (row_vecs64 > INT32_MAX) return PA_ERR_UNSUPPORTED;
-    const int row_vecs = (int)row_vecs64;
+    if ((int64_t)num_kv_heads * head_dim / 16 > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    return -1;
+}
+
+int launch_reshape_and_cache_fp8(const void* k, const void* v, const int64_t* slot_mapping, void* k_cache,
+                                 void* v_cache, int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                                 int num_blocks, int dtype, float k_scale, float v_scale, int32_t* err_word,
+                                 cudaStream_t st) {
+    const int row_vecs = (int)((int64_t)num_kv_heads * head_dim / 16);
     const int64_t total = (int64_t)num_tokens * row_vecs;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int64_t blocks = (total + 255) / 256;
     if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t num_slots = (int64_t)num_blocks * block_size;
     if (dtype == PA_F16)
         reshape_and_cache_fp8_kernel<F16Tag><<<(unsigned)blocks, 256, 0, st>>>(
@@ -121,6 +127,21 @@ extern "C" int pa_reshape_and_cache_fp8(const void* k, const void* v, const int6
             static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, static_cast<uint4*>(k_cache),
             static_cast<uint4*>(v_cache), num_tokens, row_vecs, num_slots, k_scale, v_scale, err_word);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace pa
+
+extern "C" int pa_reshape_and_cache_fp8(const void* k, const void* v, const int64_t* slot_mapping, void* k_cache,
+                                        void* v_cache, int num_tokens, int num_kv_heads, int head_dim,
+                                        int block_size, int num_blocks, int dtype, float k_scale, float v_scale,
+                                        int32_t* err_word, void* stream) {
+    using namespace pa;
+    const int rc = check_reshape_and_cache_fp8(k, v, slot_mapping, k_cache, v_cache, num_tokens, num_kv_heads,
+                                               head_dim, block_size, num_blocks, dtype, k_scale, v_scale, err_word);
+    if (rc >= 0) return rc;
+    return launch_reshape_and_cache_fp8(k, v, slot_mapping, k_cache, v_cache, num_tokens, num_kv_heads, head_dim,
+                                        block_size, num_blocks, dtype, k_scale, v_scale, err_word,
+                                        static_cast<cudaStream_t>(stream));
 }
 
 namespace pa {

@@ -115,11 +115,13 @@ def test_copy_blocks_refuses_overlapping_pairs():
     assert np.array_equal(bits(kc), kh) and np.array_equal(bits(vc), vh)
 
 
-@pytest.mark.parametrize("num_pairs,bs,hk,d", [(3, 64, 5, 64), (701, 16, 2, 128)])
-def test_copy_blocks_slices_and_many_pairs(num_pairs, bs, hk, d):
-    """A few large blocks, each spread over several CTAs' slices, and many small
-    ones, several to a slice; in both cases slices start inside a block.
-    Bit-exact against the oracle."""
+@pytest.mark.parametrize("num_pairs,bs,hk,d,overlap", [(3, 64, 5, 64, False), (701, 16, 2, 128, False),
+                                                       (2100, 16, 1, 64, False), (2100, 16, 1, 64, True)])
+def test_copy_blocks_chunks_and_many_pairs(num_pairs, bs, hk, d, overlap):
+    """A few large blocks (several 16 KiB chunks each, the last one partial), many
+    small ones (one partial chunk each), and more pairs than the kernel stages in
+    shared memory (2048), with and without two pairs into one block.  Bit-exact
+    against the oracle's copy of the pairs that do not overlap."""
     rng = np.random.default_rng(46 + num_pairs)
     nb = 2 * num_pairs + 5
     kc = torch.randn(nb, bs, hk, d, device="cuda").to(torch.bfloat16)
@@ -127,9 +129,13 @@ def test_copy_blocks_slices_and_many_pairs(num_pairs, bs, hk, d):
     kh, vh = bits(kc), bits(vc)
     perm = rng.permutation(nb).astype(np.int32)
     pairs = np.stack([perm[:num_pairs], perm[num_pairs:2 * num_pairs]], axis=1).copy()
+    keep = np.ones(num_pairs, dtype=bool)
+    if overlap:
+        pairs[2077, 1] = pairs[3, 1]     # two pairs into one block: both refused
+        keep[[3, 2077]] = False
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     pa.pa_copy_blocks(kc, vc, torch.from_numpy(pairs).cuda(), err_word=err)
     torch.cuda.synchronize()
-    assert err.item() == 0
-    oracle_pkg.get().copy_blocks(kh, vh, pairs)
+    assert err.item() == (pa.PA_DEVERR_PAIR_CONFLICT if overlap else 0)
+    oracle_pkg.get().copy_blocks(kh, vh, np.ascontiguousarray(pairs[keep]))
     assert np.array_equal(bits(kc), kh) and np.array_equal(bits(vc), vh)

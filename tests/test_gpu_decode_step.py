@@ -94,3 +94,28 @@ def test_decode_step_checks_both_calls_first():
                           workspace=torch.zeros(16, dtype=torch.uint8, device="cuda"))
     torch.cuda.synchronize()
     assert np.array_equal(bits(t["k_cache"]), before)
+
+
+@pytest.mark.parametrize("name", ["llama7b", "gqa70b"])
+def test_decode_step_fp8_equals_write_then_decode(name):
+    """pa_decode_step_fp8 against pa_reshape_and_cache_fp8 followed by
+    pa_decode_fp8: codes and output bit for bit (MHA and the tensor-core GQA
+    policy)."""
+    step = Step(name, num_seqs=8)
+    t = step.tensors()
+    to_codes = lambda x: (x.float() * 32).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    kc, vc = to_codes(t["k_cache"]), to_codes(t["v_cache"])
+    kc2, vc2 = kc.clone(), vc.clone()
+    tables, lens, slots = device_inputs(step, t)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty_like(t["q"])
+    pa.pa_decode_step_fp8(t["k"], t["v"], slots, t["q"], kc, vc, tables, lens, step.spec.scale, 1 / 32, 1 / 32,
+                          step.spec.num_kv_heads, out, err_word=err)
+    pa.pa_reshape_and_cache_fp8(t["k"], t["v"], slots, kc2, vc2, 1 / 32, 1 / 32)
+    ref = torch.empty_like(out)
+    pa.pa_decode_fp8(t["q"], kc2, vc2, tables, lens, step.spec.scale, 1 / 32, 1 / 32, step.spec.num_kv_heads, ref)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert torch.equal(kc, kc2) and torch.equal(vc, vc2)
+    assert not torch.isnan(out).any()
+    assert torch.equal(out, ref)

@@ -159,7 +159,7 @@ def test_bounded_wait_gives_up_and_reports():
     assert_close(run_case(c), c.run(oracle_pkg.get()), "f16", "decode after the self-test")
 
 
-@pytest.mark.parametrize("mode", ["mha", "gqa", "fp8", "shared_prefix"])
+@pytest.mark.parametrize("mode", ["mha", "gqa", "fp8", "shared_prefix", "two_launches"])
 def test_many_calls_on_one_workspace_leave_the_counters_zero(mode):
     """Decode calls in a row on one workspace, with split contexts: the merge of
     each (sequence, head) runs in the engine's tail from a completion queue whose
@@ -168,8 +168,10 @@ def test_many_calls_on_one_workspace_leave_the_counters_zero(mode):
     must match the oracle."""
     rng = np.random.default_rng(35)
     lens = [700, 2100, 257, 1024, 33, 1500, 513, 3000]
+    if mode == "two_launches":   # more sequences than one engine launch schedules (1024)
+        lens = rng.integers(200, 700, size=1100).tolist()
     g = 4 if mode == "gqa" else 1
-    hk = 2 if mode == "gqa" else 4
+    hk = 2 if mode in ("gqa", "two_launches") else 4
     c = PagedCase(rng, lens, hk * g, hk, 128, 16, BF16 if mode == "gqa" else F16, 1 / math.sqrt(128))
     if mode == "shared_prefix":
         members, nb = [1, 3, 5, 7], 512 // 16
@@ -208,7 +210,7 @@ def test_many_calls_on_one_workspace_leave_the_counters_zero(mode):
             call = lambda out: pa.pa_decode(q, kc, vc, tb, ln, c.scale, hk, out, workspace=ws, partition_tokens=P,
                                             err_word=err)
         ref = c.run(oracle_pkg.get(), nthreads=8)
-    outs = [torch.full_like(q, float("nan")) for _ in range(40)]
+    outs = [torch.full_like(q, float("nan")) for _ in range(8 if mode == "two_launches" else 40)]
     for out in outs:
         call(out)
     torch.cuda.synchronize()
