@@ -310,6 +310,10 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
     uint32_t badmask = 0;  // slots whose stage was dropped for a bad table entry
     bool aborted = false;
     int cst = 0;
+    // Every K/V row is read once per launch: its lines are the first the L2 gives
+    // up, so that the partials (written here, read back by the merge, rewritten at
+    // the next step), q, the tables and the output stay resident.
+    const uint64_t kv_policy = policy_evict_first();
 
     auto issue_stage = [&](const Unit& I, int st) {
         const int slot = issued % R;
@@ -354,8 +358,9 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
                         for (int hh = 0; hh < ROWB / 128; ++hh) {
                             uint8_t* kd = dst + hh * Lay::kHalfBytes + j * br * 128;
                             const int x = hh * (128 / CTag::kBytes);
-                            tma_load_3d(kd, &kmap, x, I.kv_head, row, &bars[slot]);
-                            tma_load_3d(kd + Lay::kTileBytes, &vmap, x, I.kv_head, row, &bars[slot]);
+                            tma_load_3d_hint(kd, &kmap, x, I.kv_head, row, &bars[slot], kv_policy);
+                            tma_load_3d_hint(kd + Lay::kTileBytes, &vmap, x, I.kv_head, row, &bars[slot],
+                                             kv_policy);
                         }
                     }
                 }
