@@ -284,8 +284,17 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
     // ------------------------------------------------------------ warp engine
     Policy pol;
     pol.setup(lane, smem + Lay::kOffScratch + warp * Policy::kScratchBytes);
+    // The first two units of warp w are w and w + (all warps): no claim for them,
+    // so that the launch does not start with every warp's atomics queued on one
+    // counter.  The counter hands out the rest, from unit 2 x (all warps) on.
+    // Behind the shared-prefix kernel the CTAs start over several microseconds,
+    // as that kernel's CTAs leave the SMs: there every unit is claimed, so that
+    // the first CTAs to start take the first units.
     int32_t* claim_ctr = a.sched;
-    auto claim = [&]() -> int { return lane == 0 ? atomicAdd(claim_ctr, 1) : 0; };
+    const bool static_first = a.seq_start == nullptr;
+    const int all_warps = (int)gridDim.x * NW, gw = (int)blockIdx.x * NW + warp;
+    const int claim_base = static_first ? 2 * all_warps : 0;
+    auto claim = [&]() -> int { return lane == 0 ? atomicAdd(claim_ctr, 1) + claim_base : 0; };
     auto load_tab = [&](const Unit& U, int chunk) -> int {
         const int idx = chunk * 32 + lane;
         return (U.kind == kUnitNormal && idx < U.nblk)
@@ -294,12 +303,12 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
     };
 
     // current unit C (being consumed), next unit N, and a pending raw claim
-    Unit C = decode_unit(__shfl_sync(kFullMask, claim(), 0), a, s_cum, s_key, s_len, TOK);
-    Unit N = decode_unit(__shfl_sync(kFullMask, claim(), 0), a, s_cum, s_key, s_len, TOK);
+    Unit C = decode_unit(static_first ? gw : __shfl_sync(kFullMask, claim(), 0), a, s_cum, s_key, s_len, TOK);
+    Unit N = decode_unit(static_first ? gw + all_warps : __shfl_sync(kFullMask, claim(), 0), a, s_cum, s_key,
+                         s_len, TOK);
     int pend = claim();
-    pol.fetch_q(a, C);
-    pol.take_q(a);
-    pol.fetch_q(a, N);
+    pol.fetch_q(a, C);  // taken once C's first copies are issued (q_first below)
+    bool q_first = true;
     pol.reset();
     int ntab0 = load_tab(N, 0), ntab1 = load_tab(N, 1);
     // issue cursor: in C (in_next = false) or N; its rolling table chunk pair
@@ -407,6 +416,10 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
 
     while (C.kind != kUnitNone && !aborted) {
         if (C.kind != kUnitNormal || C.nst == 0) {
+            if (q_first) {
+                pol.fetch_q(a, N);
+                q_first = false;
+            }
             write_special_rows<Tag, D>(a, C, lane);
         } else {
             // keep R stages in flight: C's remaining stages, then N's
@@ -425,6 +438,11 @@ __global__ void __launch_bounds__(NW * 32, 1) paged_decode_kernel(const DecodeAr
                 }
                 if (ist < N.nst) issue_stage(N, ist++);
                 else break;
+            }
+            if (q_first) {  // the first unit's q, loaded while its first copies were issued
+                pol.take_q(a);
+                pol.fetch_q(a, N);
+                q_first = false;
             }
             // consume one stage of C
             const int slot = consumed % R;

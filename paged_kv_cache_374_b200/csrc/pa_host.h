@@ -9,6 +9,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <utility>
 
 #include "../../include/pa.h"
 
@@ -69,6 +70,25 @@ inline bool encode_cache_map_swizzled(CUtensorMap* map, const void* base, int he
 }
 
 // Raise a kernel's dynamic shared-memory limit once per device.
+// Launch `kernel` as a programmatic dependent of the kernel before it in `stream`:
+// it may be scheduled before that kernel completes, so it must wait for it
+// (griddepcontrol.wait) before it touches memory that kernel may have written.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                   cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <typename Kernel>
 inline cudaError_t ensure_smem_limit(Kernel kernel, int bytes, std::atomic<uint64_t>& done_mask) {
     int dev = 0;

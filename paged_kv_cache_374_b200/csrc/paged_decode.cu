@@ -209,6 +209,9 @@ __device__ __forceinline__ void merge_pair(const DecodeArgs& a, int64_t sh) {
 
 template <class Tag, int D>
 __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const DecodeArgs a) {
+    // The next step's cache write, launched as a programmatic dependent, may be
+    // scheduled now: it waits for this grid to complete before it does anything.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!a.early_merge) {
         asm volatile("griddepcontrol.wait;" ::: "memory");
         merge_pair<Tag, D>(a, blockIdx.x);

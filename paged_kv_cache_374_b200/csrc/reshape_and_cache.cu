@@ -20,8 +20,12 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(const uint4* __r
                                                                  uint4* __restrict__ v_cache, int num_tokens,
                                                                  int row_vecs, int64_t num_slots,
                                                                  int32_t* err_word) {
-    // An attention launch that follows as a programmatic dependent (pa_decode_step)
-    // may start its prologue now; it waits for this grid before it reads the cache.
+    // Launched as a programmatic dependent of the kernel before it in the stream,
+    // which may have produced k and v: wait for that grid to complete before
+    // reading anything.  Then an attention launch that follows as a programmatic
+    // dependent (pa_decode_step) may start its prologue; it waits for this grid
+    // before it reads the cache.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t total = (int64_t)num_tokens * row_vecs;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -52,7 +56,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(const uint4*
                                                                      uint4* __restrict__ v_cache, int num_tokens,
                                                                      int row_vecs, int64_t num_slots, float k_scale,
                                                                      float v_scale, int32_t* err_word) {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // as the 16-bit kernel
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // as the 16-bit kernel
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t total = (int64_t)num_tokens * row_vecs;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
@@ -118,15 +123,12 @@ int launch_reshape_and_cache_fp8(const void* k, const void* v, const int64_t* sl
     int64_t blocks = (total + 255) / 256;
     if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
     const int64_t num_slots = (int64_t)num_blocks * block_size;
-    if (dtype == PA_F16)
-        reshape_and_cache_fp8_kernel<F16Tag><<<(unsigned)blocks, 256, 0, st>>>(
-            static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, static_cast<uint4*>(k_cache),
-            static_cast<uint4*>(v_cache), num_tokens, row_vecs, num_slots, k_scale, v_scale, err_word);
-    else
-        reshape_and_cache_fp8_kernel<BF16Tag><<<(unsigned)blocks, 256, 0, st>>>(
-            static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, static_cast<uint4*>(k_cache),
-            static_cast<uint4*>(v_cache), num_tokens, row_vecs, num_slots, k_scale, v_scale, err_word);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    auto kernel = dtype == PA_F16 ? reshape_and_cache_fp8_kernel<F16Tag> : reshape_and_cache_fp8_kernel<BF16Tag>;
+    const cudaError_t e = launch_dependent(
+        kernel, dim3((unsigned)blocks), dim3(256), 0, st, static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+        slot_mapping, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), num_tokens, row_vecs, num_slots,
+        k_scale, v_scale, err_word);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace pa
@@ -173,10 +175,11 @@ int launch_reshape_and_cache(const void* k, const void* v, const int64_t* slot_m
     int64_t blocks = (total + threads - 1) / threads;
     const int64_t cap = (int64_t)sms * 8;
     if (blocks > cap) blocks = cap;
-    reshape_and_cache_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
-        static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, static_cast<uint4*>(k_cache),
-        static_cast<uint4*>(v_cache), num_tokens, row_vecs, (int64_t)num_blocks * block_size, err_word);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const cudaError_t e = launch_dependent(
+        reshape_and_cache_kernel, dim3((unsigned)blocks), dim3(threads), 0, stream, static_cast<const uint4*>(k),
+        static_cast<const uint4*>(v), slot_mapping, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+        num_tokens, row_vecs, (int64_t)num_blocks * block_size, err_word);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace pa
