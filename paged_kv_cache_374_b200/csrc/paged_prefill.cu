@@ -7,27 +7,32 @@
 // at position L - n + i and attends to tokens 0 .. L - n + i through the table.
 //
 // A real dense contraction, run on the 5th-generation tensor cores (tcgen05, fp32
-// accumulators in tensor memory).  One CTA = 128 query rows of one head (the MMA's
-// M), two CTAs per SM:
-//   - warp 4 streams the kv head's K and V in 64-token tiles through two-stage
-//     TMA rings (the 128-byte-swizzled tensor maps of the decode path; a tile's
-//     table entries are read as it is issued, after one up-front range check);
-//   - warp 5 owns the tensor memory and issues every MMA from one thread:
-//       S_j = Q K_j^T   (A = Q, B = K, both K-major in shared memory; M 128 x N 64)
-//       O  += P_j V_j   (A = P_j in tensor memory, B = V_j MN-major; M 128 x N d)
-//     in the order S_0, S_1, PV_0, S_2, PV_1, ... with S double-buffered, so the
-//     softmax of tile j+1 overlaps the tensor core's work on tile j;
-//   - warps 0-3 own one query row per thread (tensor-memory lane = row): read
-//     S_j, apply the causal mask and the online softmax in base 2, write P_j over
-//     S_j (one f16 term for f16 inputs; for bf16, two terms hi + lo, about 16
-//     significant bits, so the result keeps the decode path's accuracy), and at
-//     the end normalise O and store it.
-// The running max used for the exponentials only moves when a row's max grows
-// by more than 2^8 (then O and the row sum are rescaled in tensor memory); the
-// result is the same softmax, p stays <= 256.  V rows past the sequence end are
-// zeroed in shared memory before PV (0 * NaN is NaN in an MMA).  Every wait is
-// bounded; a timeout reports PA_DEVERR_TIMEOUT and the CTA drains its copies and
-// MMAs before freeing tensor memory.
+// accumulators in tensor memory).  One CTA per SM runs two query tiles A and B of
+// 128 rows each (the MMAs' M) against the same K/V tiles of 128 tokens:
+//   - warp 8 streams the kv head's K and V tiles through two-stage TMA rings (the
+//     128-byte-swizzled tensor maps of the decode path; a tile's table entries
+//     are read as it is issued, after one up-front range check); both query tiles
+//     read every K and V tile the ring holds;
+//   - warp 9 owns the tensor memory (O_A, O_B, and one S/P buffer per query tile)
+//     and issues every MMA from one thread:
+//       S_X = Q_X K_j^T  (A = Q_X, B = K_j, both K-major in shared memory; M 128 x N 128)
+//       O_X += P_X V_j   (A = P_X in tensor memory, B = V_j MN-major; M 128 x N d)
+//     in the order S_A0, S_B0, PV_A0, S_A1, PV_B0, S_B1, PV_A1, ...: while one
+//     tile's softmax runs, the tensor core works on the other tile's MMAs;
+//   - warps 0-3 (tile A) and 4-7 (tile B) own one query row per thread
+//     (tensor-memory lane = row): read S_X, apply the causal mask and the online
+//     softmax in base 2, write P_X over S_X (one f16 term for f16 inputs; for
+//     bf16, two terms hi + lo, about 16 significant bits, so the result keeps the
+//     decode path's accuracy), and at the end normalise O_X and store it.
+// S_X(j+1) is issued after PV_X(j) and the tensor core runs one thread's MMAs in
+// order, so the arrival that says S_X(j+1) landed also says PV_X(j) has: the
+// softmax may rescale O_X then without another wait.  The running max used for
+// the exponentials only moves when a row's max grows by more than 2^8 (then O_X
+// and the row sum are rescaled in tensor memory); the result is the same
+// softmax, p stays <= 256.  V rows past the sequence end are zeroed in shared
+// memory before PV (0 * NaN is NaN in an MMA).  Every wait is bounded; a timeout
+// reports PA_DEVERR_TIMEOUT and the CTA drains its copies and MMAs before freeing
+// tensor memory.
 #include <cmath>
 
 #include "decode_gqa.cuh"
@@ -36,10 +41,12 @@
 
 namespace pa {
 
-constexpr int kPfRows = 128;         // query rows per CTA
-constexpr int kPfTok = 64;           // tokens per K/V tile
-constexpr int kPfThreads = 192;      // softmax warps 0-3, load warp 4, MMA warp 5
-constexpr uint32_t kPfTmemCols = 256;  // O at column 0, S/P buffers at 128 and 192
+constexpr int kPfRows = 128;          // query rows of one tile (the MMAs' M)
+constexpr int kPfCtaRows = 2 * kPfRows; // tiles A and B
+constexpr int kPfTok = 128;           // tokens per K/V tile (the S MMAs' N)
+constexpr int kPfLoadWarp = 8, kPfMmaWarp = 9;
+constexpr int kPfThreads = 320;       // softmax warps 0-3 (A) and 4-7 (B), load warp, MMA warp
+constexpr uint32_t kPfTmemCols = 512;   // O_X at column X d, S/P of tile X at 256 + 128 X
 constexpr float kPfRescaleLog2 = 8.f;
 
 #ifndef PA_PF_SPIN
@@ -72,14 +79,19 @@ __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity) {
 #endif
 }
 
-// The largest visible raw score of a row's tile (8 independent max chains).
+// A row's tile is read from tensor memory 64 tokens at a time (two passes: the
+// max, then the weights), so that no thread holds more than 64 scores.
+constexpr int kPfHalf = 64;
+
+// The largest visible raw score of 64 tokens of a row (8 independent max chains);
+// tokens past `vis` are left out when kDiag.
 template <bool kDiag>
-__device__ __forceinline__ float tile_row_max(const float (&x)[kPfTok], int vis) {
+__device__ __forceinline__ float half_row_max(const float (&x)[kPfHalf], int vis) {
     float m[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) m[i] = (!kDiag || i <= vis) ? x[i] : -INFINITY;
 #pragma unroll
-    for (int t = 8; t < kPfTok; ++t)
+    for (int t = 8; t < kPfHalf; ++t)
         if (!kDiag || t <= vis) m[t & 7] = fmaxf(m[t & 7], x[t]);
 #pragma unroll
     for (int w = 4; w > 0; w >>= 1)
@@ -88,23 +100,24 @@ __device__ __forceinline__ float tile_row_max(const float (&x)[kPfTok], int vis)
     return m[0];
 }
 
-// p_t = 2^(x_t c - m) for the row's tile (0 past the diagonal when kDiag), written
-// to tensor memory at `taddr` two tokens per column: P_hi in columns 0-31 and, when
-// kHiLo, P_lo = p - P_hi in columns 32-63.  Returns the sum of the weights the MMA
-// sees (P_hi + P_lo = p, or the rounded P_hi alone), so that the row's weights
-// always sum to its denominator.  Packed fp32x2 arithmetic.  p <= 256, so an f16
-// P_hi alone is within 2^-11 of p (the f16 path); a bf16 P_hi (2^-8) needs the lo
-// term to keep that accuracy.
+// p_t = 2^(x_t c - m) for 64 tokens of a row (0 past `vis` when kDiag), written to
+// tensor memory two tokens per column: P_hi at tHi (32 columns) and, when kHiLo,
+// P_lo = p - P_hi at tLo.  Returns the sum of the weights the MMA sees (P_hi + P_lo
+// = p, or the rounded P_hi alone), so that the row's weights always sum to its
+// denominator.  Packed fp32x2 arithmetic.  p <= 256, so an f16 P_hi alone is
+// within 2^-11 of p (the f16 path); a bf16 P_hi (2^-8) needs the lo term to keep
+// that accuracy.
 template <class Tag, bool kDiag, bool kHiLo>
-__device__ __forceinline__ float tile_row_p(const float (&x)[kPfTok], int vis, float c, float m, uint32_t taddr) {
+__device__ __forceinline__ float half_row_p(const float (&x)[kPfHalf], int vis, float c, float m, uint32_t tHi,
+                                            uint32_t tLo) {
     const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m), neg1 = make_float2(-1.f, -1.f);
     float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {  // 32 tokens -> 16 hi and 16 lo columns
+    for (int part = 0; part < 2; ++part) {  // 32 tokens -> 16 hi and 16 lo columns
         uint32_t ph[16], pl[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            const int t = 32 * half + 2 * k;
+            const int t = 32 * part + 2 * k;
             const float2 e = __ffma2_rn(make_float2(x[t], x[t + 1]), c2, nm2);
             float2 p = make_float2(fast_exp2(e.x), fast_exp2(e.y));
             if (kDiag) {
@@ -120,11 +133,24 @@ __device__ __forceinline__ float tile_row_p(const float (&x)[kPfTok], int vis, f
                 acc[k & 3] = __fadd2_rn(acc[k & 3], Tag::widen2(ph[k]));  // the rounded weights
             }
         }
-        umma::st16(taddr + 16 * half, ph);
-        if (kHiLo) umma::st16(taddr + 32 + 16 * half, pl);
+        umma::st16(tHi + 16 * part, ph);
+        if (kHiLo) umma::st16(tLo + 16 * part, pl);
     }
     acc[0] = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
     return acc[0].x + acc[0].y;
+}
+
+// 64 scores of a row from tensor memory (two 32-column loads, one wait).
+__device__ __forceinline__ void load_half(uint32_t taddr, float (&x)[kPfHalf]) {
+    uint32_t a[32], b[32];
+    umma::ld32(taddr, a);
+    umma::ld32(taddr + 32, b);
+    umma::wait_ld();
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+        x[t] = __uint_as_float(a[t]);
+        x[32 + t] = __uint_as_float(b[t]);
+    }
 }
 
 struct PrefillArgs {
@@ -171,32 +197,34 @@ __device__ __forceinline__ void count_partial(const PrefillArgs& a, int seq, int
 
 template <int D>
 struct PfLayout {
-    static constexpr int kQHalf = kPfRows * 128;  // 64 dims of every query row
-    static constexpr int kTHalf = kPfTok * 128;   // 64 dims of every token of a tile
+    static constexpr int kQHalf = kPfRows * 128;  // 64 dims of every row of a query tile
+    static constexpr int kQTile = (D / 64) * kQHalf;
+    static constexpr int kTHalf = kPfTok * 128;   // 64 dims of every token of a K/V tile
     static constexpr int kTile = (D / 64) * kTHalf;
-    static constexpr int kOffK = (D / 64) * kQHalf;
+    static constexpr int kOffK = 2 * kQTile;      // Q tiles A and B first
     static constexpr int kOffV = kOffK + 2 * kTile;
     static constexpr int kOffBars = kOffV + 2 * kTile;
     static constexpr int kNumBars = 16;
     static constexpr int kBytes = kOffBars + kNumBars * 8 + 16;
-    static constexpr int kAlloc = kBytes + 1024;
+    // each CTA takes all 512 tensor-memory columns, so at most one may be resident
+    // per SM: at least 116 KiB of shared memory (the head_dim 64 layout needs less)
+    static constexpr int kAlloc = kBytes + 1024 > 116 * 1024 ? kBytes + 1024 : 116 * 1024;
 };
 
 // mbarrier slots
 enum : int {
-    kBarKFull = 0,    // [2] TMA landed a K tile
-    kBarKEmpty = 2,   // [2] the S MMAs reading a K stage are done
-    kBarVFull = 4,    // [2]
-    kBarVEmpty = 6,   // [2] the PV MMAs reading a V stage are done
-    kBarSFull = 8,    // [2] S_j is in its buffer
-    kBarPFull = 10,   // [2] the 128 row threads wrote P_j
-    kBarOFull = 12,   // [2] PV_j has landed in O (alternating by tile parity)
-    kBarOLast = 14,   // the last PV has landed
-    kBarDrain = 15,   // every MMA issued has completed
+    kBarKFull = 0,   // [2] TMA landed a K tile
+    kBarKEmpty = 2,  // [2] the S MMAs reading a K stage are done
+    kBarVFull = 4,   // [2]
+    kBarVEmpty = 6,  // [2] the PV MMAs reading a V stage are done
+    kBarSFull = 8,   // [A, B] S_X(j) is in tile X's buffer (and PV_X(j-1) in O_X)
+    kBarPFull = 10,  // [A, B] tile X's 128 row threads wrote P_X(j)
+    kBarOLast = 12,  // [A, B] tile X's last PV has landed
+    kBarDrain = 14,  // every MMA issued has completed
 };
 
 template <class Tag, int D, bool kShared>
-__global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const PrefillArgs a,
+__global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const PrefillArgs a,
                                                                       const __grid_constant__ CUtensorMap kmap,
                                                                       const __grid_constant__ CUtensorMap vmap) {
     using Lay = PfLayout<D>;
@@ -215,9 +243,9 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
     const int bs = a.block_size;
 
     // The job of this CTA: nrows query rows (row r at position base_pos + r sees
-    // tokens 0 .. base_pos + r), K/V tiles tile0 .. tile0 + ntiles - 1 of the table
-    // row `tab`, of a sequence of L tokens.
-    int nrows, L, base_pos, tile0, ntiles, kv_head;
+    // tokens 0 .. base_pos + r) over the tokens [tok0, tok_end) of the table row
+    // `tab`, of a sequence of L tokens; rows 0-127 are tile A, 128-255 tile B.
+    int nrows, L, base_pos, tok0, tok_end, kv_head;
     const int32_t* tab;
     // prefill: rows q_first .. of sequence s, head h
     int s = 0, h = 0, q0 = 0, q_first = 0;
@@ -229,10 +257,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
         const int qt = gridDim.x - 1 - blockIdx.x;  // tiles with the most context first
         q0 = a.query_start[s];
         const int n = a.query_start[s + 1] - q0;
-        if (qt * kPfRows >= n) return;
+        if (qt * kPfCtaRows >= n) return;
         L = a.context_lens[s];
-        q_first = qt * kPfRows;
-        nrows = min(n - q_first, kPfRows);
+        q_first = qt * kPfCtaRows;
+        nrows = min(n - q_first, kPfCtaRows);
         if (L < 0 || L > a.max_blocks_per_seq * bs || n > L) {
             for (int i = tid; i < nrows * D; i += kPfThreads)
                 a.out[((int64_t)(q0 + q_first + i / D) * a.num_heads + h) * D + i % D] =
@@ -241,8 +269,8 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             return;
         }
         base_pos = L - n + q_first;
-        tile0 = 0;
-        ntiles = (base_pos + nrows - 1) / kPfTok + 1;
+        tok0 = 0;
+        tok_end = L;
         kv_head = h / a.group;
         tab = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
     } else {
@@ -266,9 +294,9 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             return;
         }
         const int rows = (m1 - m0) * a.group;
-        q_first = blockIdx.x * kPfRows;
+        q_first = blockIdx.x * kPfCtaRows;
         if (q_first >= rows) return;
-        nrows = min(rows - q_first, kPfRows);
+        nrows = min(rows - q_first, kPfCtaRows);
         const int lead = a.group_members[m0];
         L = a.seq_start[lead];  // tokens shared by the group
         const int P = a.partition_tokens;
@@ -278,22 +306,31 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
         }
         // the launch bounds (max_group_size, max_shared_tokens) must cover every group
         if (tid == 0 && ((p == a.max_shared_partitions - 1 && L > a.max_shared_partitions * P) ||
-                         (blockIdx.x == gridDim.x - 1 && rows > (int)gridDim.x * kPfRows)))
+                         (blockIdx.x == gridDim.x - 1 && rows > (int)gridDim.x * kPfCtaRows)))
             report(a.err_word, PA_DEVERR_LEN_RANGE);
         if ((p + 1) * P > L) return;  // past this group's prefix
-        base_pos = 1 << 29;  // no causal mask: every row sees the whole prefix
-        tile0 = p * (P / kPfTok);
-        ntiles = P / kPfTok;
+        base_pos = 1 << 29;  // no causal mask: every row sees the whole partition
+        tok0 = p * P;
+        tok_end = (p + 1) * P;
         tab = a.block_tables + (int64_t)lead * a.max_blocks_per_seq;
     }
+    // K/V tiles of each query tile: up to the one holding the last token its last row sees
+    auto tiles_of = [&](int x) {
+        const int nx = min(max(nrows - x * kPfRows, 0), kPfRows);
+        const int last = min(base_pos + x * kPfRows + nx - 1, tok_end - 1);
+        return nx > 0 ? (last - tok0) / kPfTok + 1 : 0;
+    };
+    const int nt_a = tiles_of(0), nt_b = tiles_of(1);
+    auto ntx = [&](int x) { return x ? nt_b : nt_a; };
+    const int ntiles = max(nt_a, nt_b);
     // (member sequence, query head) of CTA row r in shared-prefix mode
     auto shared_row = [&](int r, int& seq, int& head) {
         const int gr = q_first + r;
         seq = a.group_members[m0 + gr / a.group];
         head = kv_head * a.group + gr % a.group;
     };
-    const int e0 = tile0 * kPfTok / bs;
-    const int nent = (min((tile0 + ntiles) * kPfTok, L) + bs - 1) / bs;  // table entries the tiles read
+    const int e0 = tok0 / bs;
+    const int nent = (min(tok0 + ntiles * kPfTok, L) + bs - 1) / bs;  // table entries the tiles read
     bool bad = false;
     for (int i = e0 + tid; i < nent; i += kPfThreads) {
         const int id = __ldg(tab + i);
@@ -318,9 +355,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
         return;
     }
 
-    // Q rows -> K-major swizzled tile; rows past the chunk are zero.  A negative
-    // scale is moved into the sign of q (exact), so the softmax sees scale >= 0.
-    if (tid < kPfRows) {
+    // Q rows -> K-major swizzled tiles A and B; rows past the chunk are zero.  A
+    // negative scale is moved into the sign of q (exact), so the softmax sees
+    // scale >= 0.
+    if (tid < kPfCtaRows) {
         const bool live = tid < nrows;
         const uint32_t flip = a.scale_log2 < 0.f ? 0x80008000u : 0u;
         int64_t qrow;  // row of q in [rows][num_heads * D] units of D
@@ -332,6 +370,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             qrow = (int64_t)seq * a.num_heads + head;
         }
         const uint4* src = reinterpret_cast<const uint4*>(a.q + qrow * D);
+        uint8_t* qt = smem + (tid / kPfRows) * Lay::kQTile + (tid % kPfRows) * 128;
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) {
             uint4 v = live ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
@@ -339,34 +378,35 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             v.y ^= flip;
             v.z ^= flip;
             v.w ^= flip;
-            *reinterpret_cast<uint4*>(smem + (c >> 3) * Lay::kQHalf + tid * 128 + (((c & 7) ^ (tid & 7)) << 4)) = v;
+            *reinterpret_cast<uint4*>(qt + (c >> 3) * Lay::kQHalf + (((c & 7) ^ (tid & 7)) << 4)) = v;
         }
         fence_proxy_async_shared();
     }
     if (tid == 0) {
-        for (int i = 0; i < Lay::kNumBars; ++i) mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? kPfRows : 1);
+        for (int i = 0; i < Lay::kNumBars; ++i)
+            mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? kPfRows : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) umma::alloc(tslot, kPfTmemCols);
+    if (warp == kPfMmaWarp) umma::alloc(tslot, kPfTmemCols);
     umma::fence_before_sync();
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tmem = *tslot;
-    const uint32_t tO = tmem, tS = tmem + 128;  // S/P buffer b at tS + 64 b
+    const uint32_t tS = tmem + 256;  // S/P of tile X at tS + 128 X; O_X at tmem + X d
 
-    if (warp == 4) {
+    if (warp == kPfLoadWarp) {
         // ---------------------------------------------------------------- loads
-        // Lane i < 64 / box_rows owns box i of every tile: it reads that box's table
-        // entry (all lanes at once, ahead of the wait for the free stage) and issues
-        // the box's copies; lane 0 posts the byte count first.
+        // Lane i < 128 / box_rows owns box i of every tile: it reads that box's
+        // table entry (all lanes at once, ahead of the wait for the free stage)
+        // and issues the box's copies; lane 0 posts the byte count first.
         const int br = a.box_rows;
         const int nbox = kPfTok / br;
         const uint32_t box_bytes = (uint32_t)(D / 64) * br * 128;
         bool ok = true;
         int issued_k = 0, issued_v = 0;
-        auto row_of = [&](int tile) {  // this lane's cache row for `tile`, or -1
-            const int tj = tile * kPfTok + lane * br;
+        auto row_of = [&](int j) {  // this lane's cache row for tile j, or -1
+            const int tj = tok0 + j * kPfTok + lane * br;
             return (lane < nbox && tj < L) ? __ldg(tab + tj / bs) * bs + tj % bs : -1;
         };
         auto load = [&](const CUtensorMap* map, uint8_t* dst0, uint64_t* bar, int row) {
@@ -379,14 +419,14 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
                     tma_load_3d(dst0 + hh * Lay::kTHalf + lane * br * 128, map, hh * 64, kv_head, row, bar);
             }
         };
-        int row = row_of(tile0);
+        int row = row_of(0);
         for (int j = 0; j < ntiles; ++j) {
             const int st = j & 1;
             if (j >= 2) ok = __all_sync(FULL, pf_wait(&bars[kBarKEmpty + st], ((j >> 1) + 1) & 1) && !*abort_flag);
             if (!ok) break;
             load(&kmap, smem + Lay::kOffK + st * Lay::kTile, &bars[kBarKFull + st], row);
             issued_k = j + 1;
-            const int next = j + 1 < ntiles ? row_of(tile0 + j + 1) : -1;  // in flight during the wait below
+            const int next = j + 1 < ntiles ? row_of(j + 1) : -1;  // in flight during the wait below
             if (j >= 2) ok = __all_sync(FULL, pf_wait(&bars[kBarVEmpty + st], ((j >> 1) + 1) & 1) && !*abort_flag);
             if (!ok) break;
             load(&vmap, smem + Lay::kOffV + st * Lay::kTile, &bars[kBarVFull + st], row);
@@ -403,82 +443,102 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
             for (int j = max(0, issued_v - 2); j < issued_v; ++j) pf_wait(&bars[kBarVFull + (j & 1)], (j >> 1) & 1);
         }
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == kPfMmaWarp) {
         // ----------------------------------------------------------------- MMAs
-        // Operand descriptors, built once: an MMA's descriptor is its stage's plus
-        // the byte offset / 16 in the start-address field (no carry: shared
-        // addresses stay below 2^18).
-        const uint64_t dq = umma::desc_sw128(smem_u32(smem), 16, 1024);
+        // Operand descriptors, built once: an MMA's descriptor is its tile's or
+        // stage's plus the byte offset / 16 in the start-address field (no carry:
+        // shared addresses stay below 2^18).
+        const uint64_t dq0 = umma::desc_sw128(smem_u32(smem), 16, 1024);
         const uint64_t dk0 = umma::desc_sw128(smem_u32(smem + Lay::kOffK), 16, 1024);
         const uint64_t dv0 = umma::desc_sw128(smem_u32(smem + Lay::kOffV), Lay::kTHalf, 1024);
-        constexpr uint64_t kStageStep = Lay::kTile >> 4;  // the second stage of a ring
-        auto issue_s = [&](int j) {  // lane 0: S_j = Q K_j^T into buffer j & 1
+        constexpr uint64_t kQTileStep = Lay::kQTile >> 4;  // tile B's Q
+        constexpr uint64_t kStageStep = Lay::kTile >> 4;   // the second stage of a ring
+        auto issue_s = [&](int x, int j) {  // lane 0: S_X(j) = Q_X K_j^T
+            const uint64_t dq = dq0 + x * kQTileStep;
             const uint64_t bk = dk0 + (j & 1) * kStageStep;
-            const uint32_t d = tS + (j & 1) * 64;
+            const uint32_t d = tS + x * 128;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 constexpr int kQStep = Lay::kQHalf >> 4, kTStep = Lay::kTHalf >> 4;
                 umma::mma_ss(d, dq + (uint64_t)((kk >> 2) * kQStep + (kk & 3) * 2),
                              bk + (uint64_t)((kk >> 2) * kTStep + (kk & 3) * 2), kIdS, kk > 0 ? 1u : 0u);
             }
-            umma::commit(&bars[kBarSFull + (j & 1)]);
-            umma::commit(&bars[kBarKEmpty + (j & 1)]);
+            umma::commit(&bars[kBarSFull + x]);
+        };
+        auto issue_pv = [&](int x, int j) {  // lane 0: O_X += P_X V_j
+            const uint64_t bv = dv0 + (j & 1) * kStageStep;
+            const uint32_t tp = tS + x * 128, to = tmem + x * D;
+#pragma unroll
+            for (int kk = 0; kk < kPfTok / 16; ++kk) {
+                const uint64_t db = bv + (uint64_t)(kk * (2048 >> 4));  // 16 tokens further
+                // tokens 16 kk .. of half kk / 4: P_hi 8 columns in, P_lo 32 further
+                const uint32_t ta = tp + (kk >> 2) * kPfHalf + (kk & 3) * 8;
+                umma::mma_ts(to, ta, db, kIdO, (j > 0 || kk > 0) ? 1u : 0u);  // P_hi V
+                if (kHiLo) umma::mma_ts(to, ta + kPfHalf / 2, db, kIdO, 1u);  // P_lo V
+            }
         };
         auto wait = [&](int bar, uint32_t parity) {  // whole warp
             const bool ok = pf_wait(&bars[bar], parity) && !*abort_flag;
             return __all_sync(FULL, ok);
         };
-        bool ok = true;
-        for (int j = 0; j < 2 && j < ntiles && ok; ++j) {
-            ok = wait(kBarKFull + j, 0);
-            if (ok) {
-                umma::fence_after_sync();
-                if (lane == 0) issue_s(j);
-                __syncwarp();
+        bool ok = ntiles > 0 && wait(kBarKFull, 0);
+        if (ok) {
+            umma::fence_after_sync();
+            if (lane == 0) {
+                for (int x = 0; x < 2; ++x)
+                    if (ntx(x) > 0) issue_s(x, 0);
+                umma::commit(&bars[kBarKEmpty]);
             }
+            __syncwarp();
         }
         for (int j = 0; j < ntiles && ok; ++j) {
             const int st = j & 1;
-            ok = wait(kBarVFull + st, (j >> 1) & 1);
-            if (!ok) break;
-            const int t0 = (tile0 + j) * kPfTok;
-            if (t0 + kPfTok > L) {  // zero the V rows past the sequence end
-                uint8_t* vt = smem + Lay::kOffV + st * Lay::kTile;
-                const int r0 = L - t0;
+            bool v_ready = false;
+            for (int x = 0; x < 2 && ok; ++x) {
+                if (j >= ntx(x)) continue;
+                if (!v_ready) {
+                    ok = wait(kBarVFull + st, (j >> 1) & 1);
+                    if (!ok) break;
+                    const int t0 = tok0 + j * kPfTok;
+                    if (t0 + kPfTok > L) {  // zero the V rows past the sequence end
+                        uint8_t* vt = smem + Lay::kOffV + st * Lay::kTile;
+                        const int r0 = L - t0;
 #pragma unroll
-                for (int hh = 0; hh < D / 64; ++hh)
-                    for (int i = r0 * 8 + lane; i < kPfTok * 8; i += 32)
-                        *reinterpret_cast<uint4*>(vt + hh * Lay::kTHalf + i * 16) = make_uint4(0u, 0u, 0u, 0u);
-                fence_proxy_async_shared();
-                __syncwarp();
-            }
-            ok = wait(kBarPFull + st, (j >> 1) & 1);
-            if (!ok) break;
-            umma::fence_after_sync();
-            if (lane == 0) {
-                const uint64_t bv = dv0 + st * kStageStep;
-                const uint32_t tp = tS + st * 64;
-#pragma unroll
-                for (int kk = 0; kk < kPfTok / 16; ++kk) {
-                    const uint64_t db = bv + (uint64_t)(kk * (2048 >> 4));  // 16 tokens further
-                    umma::mma_ts(tO, tp + kk * 8, db, kIdO, (j > 0 || kk > 0) ? 1u : 0u);  // P_hi V
-                    if (kHiLo) umma::mma_ts(tO, tp + 32 + kk * 8, db, kIdO, 1u);           // P_lo V
+                        for (int hh = 0; hh < D / 64; ++hh)
+                            for (int i = r0 * 8 + lane; i < kPfTok * 8; i += 32)
+                                *reinterpret_cast<uint4*>(vt + hh * Lay::kTHalf + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+                        fence_proxy_async_shared();
+                        __syncwarp();
+                    }
+                    v_ready = true;
                 }
-                umma::commit(&bars[kBarVEmpty + st]);
-                umma::commit(&bars[kBarOFull + st]);
-                if (j == ntiles - 1) umma::commit(&bars[kBarOLast]);
-            }
-            __syncwarp();
-            if (j + 2 < ntiles) {
-                ok = wait(kBarKFull + st, ((j + 2) >> 1) & 1);
+                ok = wait(kBarPFull + x, j & 1);
                 if (!ok) break;
                 umma::fence_after_sync();
-                if (lane == 0) issue_s(j + 2);
+                // the last reader of V_j (tile B, or tile A when B has no tile j)
+                // releases the stage; likewise for K_{j+1} below
+                const bool v_last = x == 1 || j >= nt_b;
+                if (lane == 0) {
+                    issue_pv(x, j);
+                    if (v_last) umma::commit(&bars[kBarVEmpty + st]);
+                    if (j == ntx(x) - 1) umma::commit(&bars[kBarOLast + x]);
+                }
                 __syncwarp();
+                if (j + 1 < ntx(x)) {
+                    ok = wait(kBarKFull + ((j + 1) & 1), ((j + 1) >> 1) & 1);
+                    if (!ok) break;
+                    umma::fence_after_sync();
+                    const bool k_last = x == 1 || j + 1 >= nt_b;
+                    if (lane == 0) {
+                        issue_s(x, j + 1);
+                        if (k_last) umma::commit(&bars[kBarKEmpty + ((j + 1) & 1)]);
+                    }
+                    __syncwarp();
+                }
             }
         }
         if (lane == 0) {
-            if (!ok) {
+            if (!ok && ntiles > 0) {
                 report(a.err_word, PA_DEVERR_TIMEOUT);
                 *abort_flag = 1;
             }
@@ -487,63 +547,69 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------ softmax, one row per thread
-        const int r = tid;
+        // ---------------------------------------------- softmax, one row per thread
+        const int x = warp >> 2;             // query tile
+        const int r = x * kPfRows + (tid & (kPfRows - 1));  // CTA row
+        const int nt = ntx(x);
         const int pos = base_pos + min(r, nrows - 1);
-        const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+        const int last = min(pos, tok_end - 1);  // last visible token of this row
+        const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tSx = tS + x * 128 + lrow, tOx = tmem + x * D + lrow;
         const float c = fabsf(a.scale_log2);
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < ntiles; ++j) {
-            const int b = j & 1;
-            ok = __all_sync(FULL, pf_wait(&bars[kBarSFull + b], (j >> 1) & 1) && !*abort_flag);
+        for (int j = 0; j < nt; ++j) {
+            ok = __all_sync(FULL, pf_wait(&bars[kBarSFull + x], j & 1) && !*abort_flag);
             if (!ok) break;
             umma::fence_after_sync();
-            uint32_t sv[2][32];
-            umma::ld32(tS + b * 64 + lrow, sv[0]);
-            umma::ld32(tS + b * 64 + 32 + lrow, sv[1]);
-            umma::wait_ld();
-            const int t0 = (tile0 + j) * kPfTok;
-            // every row of the CTA sees the whole tile unless it reaches the diagonal
-            const bool diag = t0 + kPfTok - 1 > base_pos;
-            const int vis = diag ? pos - t0 : kPfTok - 1;  // last visible token of the tile, this row
-            float x[kPfTok];  // raw scores
+            const int vis = last - (tok0 + j * kPfTok);  // last visible token of the tile, this row
+            // one branch per warp: the masked path's tensor-memory stores are
+            // warp-aligned instructions, so no lane may take the other path
+            const bool diag = __any_sync(FULL, vis < kPfTok - 1);
+            float xs[kPfHalf];  // raw scores of one half of the tile
+            float mt = -INFINITY;
 #pragma unroll
-            for (int t = 0; t < kPfTok; ++t) x[t] = __uint_as_float(sv[t >> 5][t & 31]);
-            float mt = diag ? tile_row_max<true>(x, vis) : tile_row_max<false>(x, vis);
+            for (int hf = 0; hf < 2; ++hf) {
+                load_half(tSx + hf * kPfHalf, xs);
+                mt = fmaxf(mt, diag ? half_row_max<true>(xs, vis - hf * kPfHalf)
+                                    : half_row_max<false>(xs, vis - hf * kPfHalf));
+            }
             mt = mt == -INFINITY ? -INFINITY : mt * c;  // the tile max in log2 units
             const bool need = mt > m_used + kPfRescaleLog2;  // always on the first tile
             if (__any_sync(FULL, need)) {
                 const float m_new = need ? mt : m_used;
-                if (j > 0) {
+                if (j > 0) {  // PV_X(j-1) has landed in O_X (before S_X(j), see above)
                     const float alpha = fast_exp2(m_used - m_new);
-                    // PV_{j-1} must have landed in O before it is rescaled
-                    ok = __all_sync(FULL, pf_wait(&bars[kBarOFull + ((j - 1) & 1)], ((j - 1) >> 1) & 1) &&
-                                              !*abort_flag);
-                    if (!ok) break;
-                    umma::fence_after_sync();
 #pragma unroll 1
                     for (int cc = 0; cc < D / 32; ++cc) {
                         uint32_t o[32];
-                        umma::ld32(tO + lrow + cc * 32, o);
+                        umma::ld32(tOx + cc * 32, o);
                         umma::wait_ld();
 #pragma unroll
                         for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                        umma::st32(tO + lrow + cc * 32, o);
+                        umma::st32(tOx + cc * 32, o);
                     }
                     umma::wait_st();
                     l *= alpha;
                 }
                 m_used = m_new;
             }
-            l += diag ? tile_row_p<Tag, true, kHiLo>(x, vis, c, m_used, tS + b * 64 + lrow)
-                      : tile_row_p<Tag, false, kHiLo>(x, vis, c, m_used, tS + b * 64 + lrow);
+            // the weights of half hf go to its own 64 columns (P_hi of its token t in
+            // column 64 hf + t / 2, P_lo 32 columns further), which hold only scores
+            // this thread has already read
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                load_half(tSx + hf * kPfHalf, xs);
+                const uint32_t tHi = tSx + hf * kPfHalf, tLo = tHi + kPfHalf / 2;
+                l += diag ? half_row_p<Tag, true, kHiLo>(xs, vis - hf * kPfHalf, c, m_used, tHi, tLo)
+                          : half_row_p<Tag, false, kHiLo>(xs, vis - hf * kPfHalf, c, m_used, tHi, tLo);
+            }
             umma::wait_st();
             umma::fence_before_sync();
-            mbar_arrive(&bars[kBarPFull + b]);
+            mbar_arrive(&bars[kBarPFull + x]);
         }
-        if (ok) ok = __all_sync(FULL, pf_wait(&bars[kBarOLast], 0) && !*abort_flag);
-        if (ok && kShared) {
+        if (ok && nt > 0) ok = __all_sync(FULL, pf_wait(&bars[kBarOLast + x], 0) && !*abort_flag);
+        if (ok && nt > 0 && kShared) {
             // partial of this partition for the row's (sequence, head): running max
             // (base-2 units, scores scaled by scale * log2 e), sum, unnormalised o
             umma::fence_after_sync();
@@ -564,7 +630,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t o[32];
-                umma::ld32(tO + lrow + cc * 32, o);
+                umma::ld32(tOx + cc * 32, o);
                 umma::wait_ld();
                 if (write) {
 #pragma unroll
@@ -578,14 +644,15 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
                 a.ws_l[pi] = l;
                 if (a.early_merge) count_partial(a, seq, head);
             }
-        } else if (ok) {
+        } else if (ok && nt > 0) {
             umma::fence_after_sync();
             const float inv = 1.f / l;
-            uint4* dst = reinterpret_cast<uint4*>(a.out + ((int64_t)(q0 + q_first + min(r, nrows - 1)) * a.num_heads + h) * D);
+            uint4* dst = reinterpret_cast<uint4*>(
+                a.out + ((int64_t)(q0 + q_first + min(r, nrows - 1)) * a.num_heads + h) * D);
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t o[32];
-                umma::ld32(tO + lrow + cc * 32, o);
+                umma::ld32(tOx + cc * 32, o);
                 umma::wait_ld();
                 if (r < nrows) {
 #pragma unroll
@@ -597,14 +664,14 @@ __global__ void __launch_bounds__(kPfThreads, 2) paged_prefill_kernel(const Pref
                     }
                 }
             }
-        } else if (lane == 0) {
+        } else if (!ok && lane == 0) {
             report(a.err_word, PA_DEVERR_TIMEOUT);
             *abort_flag = 1;
         }
     }
     umma::fence_before_sync();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kPfMmaWarp) {
         umma::fence_after_sync();
         umma::dealloc(tmem, kPfTmemCols);
     }
@@ -625,7 +692,8 @@ int launch_prefill(PrefillArgs args, const void* k_cache, const void* v_cache, i
     if (!encode_cache_map_swizzled(&kmap, k_cache, D, num_kv_heads, total_tokens, args.box_rows) ||
         !encode_cache_map_swizzled(&vmap, v_cache, D, num_kv_heads, total_tokens, args.box_rows))
         return PA_ERR_CUDA;
-    dim3 grid((unsigned)((max_query_len + kPfRows - 1) / kPfRows), (unsigned)args.num_heads, (unsigned)num_seqs);
+    dim3 grid((unsigned)((max_query_len + kPfCtaRows - 1) / kPfCtaRows), (unsigned)args.num_heads,
+              (unsigned)num_seqs);
     kernel<<<grid, kPfThreads, Lay::kAlloc, stream>>>(args, kmap, vmap);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -644,7 +712,7 @@ int launch_shared(PrefillArgs args, const void* k_cache, const void* v_cache, in
         !encode_cache_map_swizzled(&vmap, v_cache, D, num_kv_heads, total_tokens, args.box_rows))
         return PA_ERR_CUDA;
     const int64_t rows = (int64_t)max_group_size * args.group;
-    dim3 grid((unsigned)((rows + kPfRows - 1) / kPfRows), (unsigned)num_kv_heads,
+    dim3 grid((unsigned)((rows + kPfCtaRows - 1) / kPfCtaRows), (unsigned)num_kv_heads,
               (unsigned)(num_groups * args.max_shared_partitions));
     kernel<<<grid, kPfThreads, Lay::kAlloc, stream>>>(args, kmap, vmap);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
@@ -653,7 +721,7 @@ int launch_shared(PrefillArgs args, const void* k_cache, const void* v_cache, in
 }  // namespace
 
 int launch_shared_prefix(const SharedPrefixLaunch& l, cudaStream_t stream) {
-    if (l.partition_tokens % kPfTok != 0 || l.max_shared_tokens % l.partition_tokens != 0) return PA_ERR_INVALID_ARG;
+    if (l.partition_tokens % 64 != 0 || l.max_shared_tokens % l.partition_tokens != 0) return PA_ERR_INVALID_ARG;
     const int64_t maxpp = l.max_shared_tokens / l.partition_tokens;
     if (maxpp == 0 || l.num_groups == 0) return PA_OK;
     if (maxpp * l.num_groups > 65535 || l.num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
