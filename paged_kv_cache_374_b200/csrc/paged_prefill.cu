@@ -53,6 +53,7 @@ constexpr float kPfRescaleLog2 = 8.f;
 #define PA_PF_SPIN 1
 #endif
 
+
 // Bounded wait on an mbarrier phase: the suspending try_wait of the library, or
 // (PA_PF_SPIN) a poll of test_wait bounded by 2 s of the global timer.
 __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity) {
@@ -218,7 +219,7 @@ enum : int {
     kBarVFull = 4,   // [2]
     kBarVEmpty = 6,  // [2] the PV MMAs reading a V stage are done
     kBarSFull = 8,   // [A, B] S_X(j) is in tile X's buffer (and PV_X(j-1) in O_X)
-    kBarPFull = 10,  // [A, B] tile X's 128 row threads wrote P_X(j)
+    kBarPFull = 10,  // [A, B] tile X's 4 row warps wrote P_X(j)
     kBarOLast = 12,  // [A, B] tile X's last PV has landed
     kBarDrain = 14,  // every MMA issued has completed
 };
@@ -384,7 +385,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
     }
     if (tid == 0) {
         for (int i = 0; i < Lay::kNumBars; ++i)
-            mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? kPfRows : 1);
+            mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? kPfRows / 32 : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -581,13 +582,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
                 if (j > 0) {  // PV_X(j-1) has landed in O_X (before S_X(j), see above)
                     const float alpha = fast_exp2(m_used - m_new);
 #pragma unroll 1
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t o[32];
-                        umma::ld32(tOx + cc * 32, o);
+                    for (int cc = 0; cc < D / 8; ++cc) {  // 8 columns at a time: few registers beside the scores
+                        uint32_t o[8];
+                        umma::ld8(tOx + cc * 8, o);
                         umma::wait_ld();
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                        umma::st32(tOx + cc * 32, o);
+                        for (int k = 0; k < 8; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                        umma::st8(tOx + cc * 8, o);
                     }
                     umma::wait_st();
                     l *= alpha;
@@ -606,7 +607,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
             }
             umma::wait_st();
             umma::fence_before_sync();
-            mbar_arrive(&bars[kBarPFull + x]);
+            __syncwarp();  // every lane's P is stored: one arrival per warp
+            if (lane == 0) mbar_arrive(&bars[kBarPFull + x]);
         }
         if (ok && nt > 0) ok = __all_sync(FULL, pf_wait(&bars[kBarOLast + x], 0) && !*abort_flag);
         if (ok && nt > 0 && kShared) {
