@@ -597,10 +597,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
             }
             // the weights of half hf go to its own 64 columns (P_hi of its token t in
             // column 64 hf + t / 2, P_lo 32 columns further), which hold only scores
-            // this thread has already read
+            // this thread has already read.  The second half's scores are still in
+            // registers from the max pass: it goes first, then the first is read again.
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                load_half(tSx + hf * kPfHalf, xs);
+            for (int hf = 1; hf >= 0; --hf) {
+                if (hf == 0) load_half(tSx, xs);
                 const uint32_t tHi = tSx + hf * kPfHalf, tLo = tHi + kPfHalf / 2;
                 l += diag ? half_row_p<Tag, true, kHiLo>(xs, vis - hf * kPfHalf, c, m_used, tHi, tLo)
                           : half_row_p<Tag, false, kHiLo>(xs, vis - hf * kPfHalf, c, m_used, tHi, tLo);
