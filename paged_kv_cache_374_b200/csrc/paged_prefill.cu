@@ -568,12 +568,25 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
             // warp-aligned instructions, so no lane may take the other path
             const bool diag = __any_sync(FULL, vis < kPfTok - 1);
             float xs[kPfHalf];  // raw scores of one half of the tile
-            float mt = -INFINITY;
+            float mt;
+            {
+                // the whole row in one round trip; the second half stays in xs
+                float x0[kPfHalf];
+                uint32_t a[32], b[32], c0[32], c1[32];
+                umma::ld32(tSx, a);
+                umma::ld32(tSx + 32, b);
+                umma::ld32(tSx + 64, c0);
+                umma::ld32(tSx + 96, c1);
+                umma::wait_ld();
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                load_half(tSx + hf * kPfHalf, xs);
-                mt = fmaxf(mt, diag ? half_row_max<true>(xs, vis - hf * kPfHalf)
-                                    : half_row_max<false>(xs, vis - hf * kPfHalf));
+                for (int t = 0; t < 32; ++t) {
+                    x0[t] = __uint_as_float(a[t]);
+                    x0[32 + t] = __uint_as_float(b[t]);
+                    xs[t] = __uint_as_float(c0[t]);
+                    xs[32 + t] = __uint_as_float(c1[t]);
+                }
+                mt = fmaxf(diag ? half_row_max<true>(x0, vis) : half_row_max<false>(x0, vis),
+                           diag ? half_row_max<true>(xs, vis - kPfHalf) : half_row_max<false>(xs, vis - kPfHalf));
             }
             mt = mt == -INFINITY ? -INFINITY : mt * c;  // the tile max in log2 units
             const bool need = mt > m_used + kPfRescaleLog2;  // always on the first tile
