@@ -330,6 +330,61 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
         seq = a.group_members[m0 + gr / a.group];
         head = kv_head * a.group + gr % a.group;
     };
+    // K/V copies of tile j (the load warp): lane i < 128 / box_rows owns box i of
+    // every tile and reads that box's table entry; lane 0 posts the byte count first.
+    // An entry out of range is never copied (the range check below then skips the CTA).
+    const int br = a.box_rows;
+    const int nbox = kPfTok / br;
+    const uint32_t box_bytes = (uint32_t)(D / 64) * br * 128;
+    auto row_of = [&](int j) {  // this lane's cache row for tile j, or -1
+        const int tj = tok0 + j * kPfTok + lane * br;
+        if (lane >= nbox || tj >= L) return -1;
+        const int id = __ldg(tab + tj / bs);
+        return (id >= 0 && id < a.num_blocks) ? id * bs + tj % bs : -1;
+    };
+    auto load = [&](const CUtensorMap* map, uint8_t* dst0, uint64_t* bar, int row) {
+        const uint32_t n = __popc(__ballot_sync(FULL, row >= 0));
+        if (lane == 0) mbar_arrive_expect_tx(bar, n * box_bytes);
+        __syncwarp();
+        if (row >= 0) {
+#pragma unroll
+            for (int hh = 0; hh < D / 64; ++hh)
+                tma_load_3d(dst0 + hh * Lay::kTHalf + lane * br * 128, map, hh * 64, kv_head, row, bar);
+        }
+    };
+    // Start-up, overlapped: the load warp sets up the barriers and issues the first
+    // two K/V tiles, the row threads fetch their q rows, and the table range check
+    // runs meanwhile.
+    const int early = ntiles < 2 ? ntiles : 2;  // tiles the load warp issues before the check
+    if (warp == kPfLoadWarp) {
+        if (lane == 0) {
+            for (int i = 0; i < Lay::kNumBars; ++i)
+                mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? kPfRows / 32 : 1);
+            *abort_flag = 0;
+            fence_mbar_init();
+        }
+        __syncwarp();
+        for (int j = 0; j < early; ++j) {
+            const int row = row_of(j);
+            load(&kmap, smem + Lay::kOffK + j * Lay::kTile, &bars[kBarKFull + j], row);
+            load(&vmap, smem + Lay::kOffV + j * Lay::kTile, &bars[kBarVFull + j], row);
+        }
+    }
+    uint4 qv[D / 8];  // this row thread's q row, in flight during the check
+    const bool q_live = tid < nrows;
+    if (tid < kPfCtaRows) {
+        int64_t qrow;  // row of q in [rows][num_heads * D] units of D
+        if constexpr (!kShared) {
+            qrow = (int64_t)(q0 + q_first + (q_live ? tid : 0)) * a.num_heads + h;
+        } else {
+            int seq, head;
+            shared_row(q_live ? tid : 0, seq, head);
+            qrow = (int64_t)seq * a.num_heads + head;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + qrow * D);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) qv[c] = q_live ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
     const int e0 = tok0 / bs;
     const int nent = (min(tok0 + ntiles * kPfTok, L) + bs - 1) / bs;  // table entries the tiles read
     bool bad = false;
@@ -338,6 +393,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
         bad |= id < 0 || id >= a.num_blocks;
     }
     if (__syncthreads_or(bad)) {
+        if (warp == kPfLoadWarp && lane == 0)  // the early copies land before the CTA exits
+            for (int j = 0; j < early; ++j) {
+                pf_wait(&bars[kBarKFull + j], 0);
+                pf_wait(&bars[kBarVFull + j], 0);
+            }
         if constexpr (!kShared) {
             for (int i = tid; i < nrows * D; i += kPfThreads)
                 a.out[((int64_t)(q0 + q_first + i / D) * a.num_heads + h) * D + i % D] =
@@ -360,21 +420,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
     // negative scale is moved into the sign of q (exact), so the softmax sees
     // scale >= 0.
     if (tid < kPfCtaRows) {
-        const bool live = tid < nrows;
         const uint32_t flip = a.scale_log2 < 0.f ? 0x80008000u : 0u;
-        int64_t qrow;  // row of q in [rows][num_heads * D] units of D
-        if constexpr (!kShared) {
-            qrow = (int64_t)(q0 + q_first + (live ? tid : 0)) * a.num_heads + h;
-        } else {
-            int seq, head;
-            shared_row(live ? tid : 0, seq, head);
-            qrow = (int64_t)seq * a.num_heads + head;
-        }
-        const uint4* src = reinterpret_cast<const uint4*>(a.q + qrow * D);
         uint8_t* qt = smem + (tid / kPfRows) * Lay::kQTile + (tid % kPfRows) * 128;
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) {
-            uint4 v = live ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            uint4 v = qv[c];
             v.x ^= flip;
             v.y ^= flip;
             v.z ^= flip;
@@ -382,12 +432,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
             *reinterpret_cast<uint4*>(qt + (c >> 3) * Lay::kQHalf + (((c & 7) ^ (tid & 7)) << 4)) = v;
         }
         fence_proxy_async_shared();
-    }
-    if (tid == 0) {
-        for (int i = 0; i < Lay::kNumBars; ++i)
-            mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? kPfRows / 32 : 1);
-        *abort_flag = 0;
-        fence_mbar_init();
     }
     if (warp == kPfMmaWarp) umma::alloc(tslot, kPfTmemCols);
     umma::fence_before_sync();
@@ -398,30 +442,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
 
     if (warp == kPfLoadWarp) {
         // ---------------------------------------------------------------- loads
-        // Lane i < 128 / box_rows owns box i of every tile: it reads that box's
-        // table entry (all lanes at once, ahead of the wait for the free stage)
-        // and issues the box's copies; lane 0 posts the byte count first.
-        const int br = a.box_rows;
-        const int nbox = kPfTok / br;
-        const uint32_t box_bytes = (uint32_t)(D / 64) * br * 128;
+        // Tiles `early` .. on (the first ones went out during the start-up); a tile's
+        // table entries are read ahead of the wait for its free stage.
         bool ok = true;
-        int issued_k = 0, issued_v = 0;
-        auto row_of = [&](int j) {  // this lane's cache row for tile j, or -1
-            const int tj = tok0 + j * kPfTok + lane * br;
-            return (lane < nbox && tj < L) ? __ldg(tab + tj / bs) * bs + tj % bs : -1;
-        };
-        auto load = [&](const CUtensorMap* map, uint8_t* dst0, uint64_t* bar, int row) {
-            const uint32_t n = __popc(__ballot_sync(FULL, row >= 0));
-            if (lane == 0) mbar_arrive_expect_tx(bar, n * box_bytes);
-            __syncwarp();
-            if (row >= 0) {
-#pragma unroll
-                for (int hh = 0; hh < D / 64; ++hh)
-                    tma_load_3d(dst0 + hh * Lay::kTHalf + lane * br * 128, map, hh * 64, kv_head, row, bar);
-            }
-        };
-        int row = row_of(0);
-        for (int j = 0; j < ntiles; ++j) {
+        int issued_k = early, issued_v = early;
+        int row = early < ntiles ? row_of(early) : -1;
+        for (int j = early; j < ntiles; ++j) {
             const int st = j & 1;
             if (j >= 2) ok = __all_sync(FULL, pf_wait(&bars[kBarKEmpty + st], ((j >> 1) + 1) & 1) && !*abort_flag);
             if (!ok) break;
