@@ -101,20 +101,25 @@ def test_prefill_flow_then_decode():
     assert_close(out1, ref1, "f16", "decode after prefill")
 
 
-def test_prefill_bad_entries_give_nan_rows():
-    rng = np.random.default_rng(62)
-    c = PagedCase(rng, [100, 100], 4, 4, 128, 16, F16, 0.1)
-    qs = np.array([0, 40, 80], dtype=np.int32)
-    q = to_bits(rng.normal(0, 1, (80, 4, 128)), F16)
+@pytest.mark.parametrize("bad_block,bad_id", [(2, "past"), (10, "negative"), (20, "past")])
+def test_prefill_bad_entries_give_nan_rows(bad_block, bad_id):
+    """A bad table entry in the first K/V tile (its copy goes out before the range
+    check, so the box is skipped and the CTA waits for its other copies), in the
+    second, or in a later one: NaN rows for that sequence only, the error bit, and
+    the other sequence unchanged."""
+    rng = np.random.default_rng(62 + bad_block)
+    c = PagedCase(rng, [400, 400], 4, 4, 128, 16, F16, 0.1)
+    qs = np.array([0, 300, 600], dtype=np.int32)
+    q = to_bits(rng.normal(0, 1, (600, 4, 128)), F16)
     tables = c.tables.copy()
-    tables[1, 2] = c.NB + 7
+    tables[1, bad_block] = c.NB + 7 if bad_id == "past" else -3
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = run_prefill(c, q, qs, err=err, tables=tables)
     assert err.item() & pa.PA_DEVERR_TABLE_RANGE
-    assert torch.isnan(out[40:]).all()
-    ref = oracle_pkg.get().prefill(q[:40].copy(), c.k_cache, c.v_cache, c.tables[:1].copy(), c.lens[:1].copy(),
-                                   qs[:2].copy(), c.scale, F16)
-    assert_close(out[:40], ref, "f16", "unaffected sequence")
+    assert torch.isnan(out[300:]).all()
+    ref = oracle_pkg.get().prefill(q[:300].copy(), c.k_cache, c.v_cache, c.tables[:1].copy(), c.lens[:1].copy(),
+                                   qs[:2].copy(), c.scale, F16, nthreads=8)
+    assert_close(out[:300], ref, "f16", "unaffected sequence")
 
 
 # ------------------------------------------------- large logits: the rescale path
