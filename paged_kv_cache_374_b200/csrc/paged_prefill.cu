@@ -222,12 +222,14 @@ enum : int {
     kBarPFull = 10,  // [A, B] tile X's 4 row warps wrote P_X(j)
     kBarOLast = 12,  // [A, B] tile X's last PV has landed
     kBarDrain = 14,  // every MMA issued has completed
+    kBarQ = 15,      // (prefill) the query tiles copied by TMA have landed
 };
 
 template <class Tag, int D, bool kShared>
 __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const PrefillArgs a,
                                                                       const __grid_constant__ CUtensorMap kmap,
-                                                                      const __grid_constant__ CUtensorMap vmap) {
+                                                                      const __grid_constant__ CUtensorMap vmap,
+                                                                      const __grid_constant__ CUtensorMap qmap) {
     using Lay = PfLayout<D>;
     constexpr bool kBF16 = Tag::kIsBF16;
     constexpr bool kHiLo = kBF16;  // P as hi + lo 16-bit terms (bf16), or one f16 term
@@ -240,6 +242,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBars);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + Lay::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+    volatile int* bad_flag = reinterpret_cast<volatile int*>(tslot + 2);  // a table entry out of range
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bs = a.block_size;
 
@@ -252,9 +255,18 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
     int s = 0, h = 0, q0 = 0, q_first = 0;
     // shared prefix: rows q_first .. of the group's (member, query head) list, partition p
     int m0 = 0, p = 0;
+    // prefill: the load warp's table entries for its boxes of tiles 0 and 1, read
+    // before the lengths arrive (entries past the sequence are ignored later)
+    int pre0 = -1, pre1 = -1;
     if constexpr (!kShared) {
         s = blockIdx.z;
         h = blockIdx.y;
+        if (warp == kPfLoadWarp && lane < kPfTok / a.box_rows) {
+            const int32_t* row = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
+            const int e0 = lane * a.box_rows / bs, e1 = (kPfTok + lane * a.box_rows) / bs;
+            if (e0 < a.max_blocks_per_seq) pre0 = __ldg(row + e0);
+            if (e1 < a.max_blocks_per_seq) pre1 = __ldg(row + e1);
+        }
         const int qt = gridDim.x - 1 - blockIdx.x;  // tiles with the most context first
         q0 = a.query_start[s];
         const int n = a.query_start[s + 1] - q0;
@@ -332,15 +344,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
     };
     // K/V copies of tile j (the load warp): lane i < 128 / box_rows owns box i of
     // every tile and reads that box's table entry; lane 0 posts the byte count first.
-    // An entry out of range is never copied (the range check below then skips the CTA).
+    // An entry out of range is never copied and marks the CTA bad.
     const int br = a.box_rows;
     const int nbox = kPfTok / br;
     const uint32_t box_bytes = (uint32_t)(D / 64) * br * 128;
     auto row_of = [&](int j) {  // this lane's cache row for tile j, or -1
         const int tj = tok0 + j * kPfTok + lane * br;
         if (lane >= nbox || tj >= L) return -1;
-        const int id = __ldg(tab + tj / bs);
-        return (id >= 0 && id < a.num_blocks) ? id * bs + tj % bs : -1;
+        const int id = (!kShared && j < 2) ? (j == 0 ? pre0 : pre1) : __ldg(tab + tj / bs);
+        const bool in_range = id >= 0 && id < a.num_blocks;
+        if (!in_range) *bad_flag = 1;
+        return in_range ? id * bs + tj % bs : -1;
     };
     auto load = [&](const CUtensorMap* map, uint8_t* dst0, uint64_t* bar, int row) {
         const uint32_t n = __popc(__ballot_sync(FULL, row >= 0));
@@ -353,15 +367,29 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
         }
     };
     // Start-up, overlapped: the load warp sets up the barriers and issues the first
-    // two K/V tiles, the row threads fetch their q rows, and the table range check
-    // runs meanwhile.
-    const int early = ntiles < 2 ? ntiles : 2;  // tiles the load warp issues before the check
+    // two K/V tiles and (prefill) the full query tiles by TMA; the row threads fetch
+    // the other q rows.  Shared-prefix mode checks the table range before it goes
+    // on; prefill checks each entry as the load warp reads it and turns the CTA's
+    // rows into NaN at the end if one was out of range.
+    const int early = ntiles < 2 ? ntiles : 2;  // tiles the load warp issues first
+    // prefill query tiles of 128 rows come by TMA (rows of a chunk are contiguous in q)
+    auto q_by_tma = [&](int x) { return !kShared && nrows >= (x + 1) * kPfRows; };
     if (warp == kPfLoadWarp) {
         if (lane == 0) {
             for (int i = 0; i < Lay::kNumBars; ++i)
                 mbar_init(&bars[i], (i == kBarPFull || i == kBarPFull + 1) ? kPfRows / 32 : 1);
             *abort_flag = 0;
+            *bad_flag = 0;
             fence_mbar_init();
+            if (!kShared) {
+                mbar_arrive_expect_tx(&bars[kBarQ], (uint32_t)((q_by_tma(0) + q_by_tma(1)) * Lay::kQTile));
+                for (int x = 0; x < 2; ++x)
+                    if (q_by_tma(x))
+#pragma unroll
+                        for (int hh = 0; hh < D / 64; ++hh)
+                            tma_load_3d(smem + x * Lay::kQTile + hh * Lay::kQHalf, &qmap, hh * 64, h,
+                                        q0 + q_first + x * kPfRows, &bars[kBarQ]);
+            }
         }
         __syncwarp();
         for (int j = 0; j < early; ++j) {
@@ -370,9 +398,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
             load(&vmap, smem + Lay::kOffV + j * Lay::kTile, &bars[kBarVFull + j], row);
         }
     }
-    uint4 qv[D / 8];  // this row thread's q row, in flight during the check
+    const bool q_rows = tid < kPfCtaRows && !q_by_tma(tid / kPfRows);  // this thread stores its q row
+    uint4 qv[D / 8];
     const bool q_live = tid < nrows;
-    if (tid < kPfCtaRows) {
+    if (q_rows) {
         int64_t qrow;  // row of q in [rows][num_heads * D] units of D
         if constexpr (!kShared) {
             qrow = (int64_t)(q0 + q_first + (q_live ? tid : 0)) * a.num_heads + h;
@@ -385,24 +414,20 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) qv[c] = q_live ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
     }
-    const int e0 = tok0 / bs;
-    const int nent = (min(tok0 + ntiles * kPfTok, L) + bs - 1) / bs;  // table entries the tiles read
-    bool bad = false;
-    for (int i = e0 + tid; i < nent; i += kPfThreads) {
-        const int id = __ldg(tab + i);
-        bad |= id < 0 || id >= a.num_blocks;
-    }
-    if (__syncthreads_or(bad)) {
-        if (warp == kPfLoadWarp && lane == 0)  // the early copies land before the CTA exits
-            for (int j = 0; j < early; ++j) {
-                pf_wait(&bars[kBarKFull + j], 0);
-                pf_wait(&bars[kBarVFull + j], 0);
-            }
-        if constexpr (!kShared) {
-            for (int i = tid; i < nrows * D; i += kPfThreads)
-                a.out[((int64_t)(q0 + q_first + i / D) * a.num_heads + h) * D + i % D] =
-                    Tag::round1(__int_as_float(0x7fc00000));
-        } else {
+    if constexpr (kShared) {
+        const int e0 = tok0 / bs;
+        const int nent = (min(tok0 + ntiles * kPfTok, L) + bs - 1) / bs;  // table entries the tiles read
+        bool bad = false;
+        for (int i = e0 + tid; i < nent; i += kPfThreads) {
+            const int id = __ldg(tab + i);
+            bad |= id < 0 || id >= a.num_blocks;
+        }
+        if (__syncthreads_or(bad)) {
+            if (warp == kPfLoadWarp && lane == 0)  // the early copies land before the CTA exits
+                for (int j = 0; j < early; ++j) {
+                    pf_wait(&bars[kBarKFull + j], 0);
+                    pf_wait(&bars[kBarVFull + j], 0);
+                }
             for (int r = tid; r < nrows; r += kPfThreads) {
                 int seq, head;
                 shared_row(r, seq, head);
@@ -411,16 +436,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
                 a.ws_l[pi] = __int_as_float(0x7fc00000);
                 if (a.early_merge) count_partial(a, seq, head);  // merged, so the NaN reaches the row
             }
+            if (tid == 0) report(a.err_word, PA_DEVERR_TABLE_RANGE);
+            return;
         }
-        if (tid == 0) report(a.err_word, PA_DEVERR_TABLE_RANGE);
-        return;
     }
 
-    // Q rows -> K-major swizzled tiles A and B; rows past the chunk are zero.  A
-    // negative scale is moved into the sign of q (exact), so the softmax sees
-    // scale >= 0.
-    if (tid < kPfCtaRows) {
-        const uint32_t flip = a.scale_log2 < 0.f ? 0x80008000u : 0u;
+    // q rows -> K-major swizzled tiles A and B (the 128-byte swizzle TMA applies);
+    // rows past the chunk are zero.  A negative scale is moved into the sign of q
+    // (exact), so the softmax sees scale >= 0: the row threads flip their own rows
+    // here, and the rows TMA brings once they have landed (below).
+    const uint32_t flip = a.scale_log2 < 0.f ? 0x80008000u : 0u;
+    if (q_rows) {
         uint8_t* qt = smem + (tid / kPfRows) * Lay::kQTile + (tid % kPfRows) * 128;
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) {
@@ -437,6 +463,28 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
     umma::fence_before_sync();
     __syncthreads();
     umma::fence_after_sync();
+    if (!kShared && flip) {  // the rows TMA brought (the barriers are initialised now)
+        if (tid < kPfCtaRows && !q_rows) {
+            if (pf_wait(&bars[kBarQ], 0)) {
+                uint4* qt = reinterpret_cast<uint4*>(smem + (tid / kPfRows) * Lay::kQTile + (tid % kPfRows) * 128);
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) {  // every 16-byte chunk of the row, wherever the swizzle put it
+                    uint4* w = qt + (c >> 3) * (Lay::kQHalf / 16) + (c & 7);
+                    uint4 v = *w;
+                    v.x ^= flip;
+                    v.y ^= flip;
+                    v.z ^= flip;
+                    v.w ^= flip;
+                    *w = v;
+                }
+                fence_proxy_async_shared();
+            } else {
+                report(a.err_word, PA_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+        }
+        __syncthreads();
+    }
     const uint32_t tmem = *tslot;
     const uint32_t tS = tmem + 256;  // S/P of tile X at tS + 128 X; O_X at tmem + X d
 
@@ -466,6 +514,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
                 *abort_flag = 1;
             }
             // every copy still in flight lands before the CTA may exit
+            if (!kShared) pf_wait(&bars[kBarQ], 0);
             for (int j = max(0, issued_k - 2); j < issued_k; ++j) pf_wait(&bars[kBarKFull + (j & 1)], (j >> 1) & 1);
             for (int j = max(0, issued_v - 2); j < issued_v; ++j) pf_wait(&bars[kBarVFull + (j & 1)], (j >> 1) & 1);
         }
@@ -508,7 +557,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
             const bool ok = pf_wait(&bars[bar], parity) && !*abort_flag;
             return __all_sync(FULL, ok);
         };
-        bool ok = ntiles > 0 && wait(kBarKFull, 0);
+        bool ok = ntiles > 0 && wait(kBarKFull, 0) && (kShared || wait(kBarQ, 0));
         if (ok) {
             umma::fence_after_sync();
             if (lane == 0) {
@@ -717,6 +766,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
         umma::fence_after_sync();
         umma::dealloc(tmem, kPfTmemCols);
     }
+    if (!kShared && *bad_flag) {  // a table entry was out of range: the CTA's rows are NaN
+        for (int i = tid; i < nrows * D; i += kPfThreads)
+            a.out[((int64_t)(q0 + q_first + i / D) * a.num_heads + h) * D + i % D] =
+                Tag::round1(__int_as_float(0x7fc00000));
+        if (tid == 0) report(a.err_word, PA_DEVERR_TABLE_RANGE);
+    }
 }
 
 namespace {
@@ -734,9 +789,15 @@ int launch_prefill(PrefillArgs args, const void* k_cache, const void* v_cache, i
     if (!encode_cache_map_swizzled(&kmap, k_cache, D, num_kv_heads, total_tokens, args.box_rows) ||
         !encode_cache_map_swizzled(&vmap, v_cache, D, num_kv_heads, total_tokens, args.box_rows))
         return PA_ERR_CUDA;
+    // q as [rows][num_heads][D]; the extent covers every row a full query tile may
+    // start at (num_seqs * max_query_len bounds the packed rows), and only tiles
+    // of 128 rows inside one sequence's chunk are copied
+    CUtensorMap qmap;
+    if (!encode_cache_map_swizzled(&qmap, args.q, D, args.num_heads, (int64_t)num_seqs * max_query_len, kPfRows))
+        return PA_ERR_CUDA;
     dim3 grid((unsigned)((max_query_len + kPfCtaRows - 1) / kPfCtaRows), (unsigned)args.num_heads,
               (unsigned)num_seqs);
-    kernel<<<grid, kPfThreads, Lay::kAlloc, stream>>>(args, kmap, vmap);
+    kernel<<<grid, kPfThreads, Lay::kAlloc, stream>>>(args, kmap, vmap, qmap);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -756,7 +817,7 @@ int launch_shared(PrefillArgs args, const void* k_cache, const void* v_cache, in
     const int64_t rows = (int64_t)max_group_size * args.group;
     dim3 grid((unsigned)((rows + kPfCtaRows - 1) / kPfCtaRows), (unsigned)num_kv_heads,
               (unsigned)(num_groups * args.max_shared_partitions));
-    kernel<<<grid, kPfThreads, Lay::kAlloc, stream>>>(args, kmap, vmap);
+    kernel<<<grid, kPfThreads, Lay::kAlloc, stream>>>(args, kmap, vmap, kmap);  // (no q map in this mode)
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

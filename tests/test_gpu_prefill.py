@@ -49,6 +49,22 @@ def test_prefill_matches_oracle(d, bs, g, dtype):
     assert_close(out, ref, WK[dtype], f"prefill d{d} bs{bs} g{g}")
 
 
+@pytest.mark.parametrize("dtype", [F16, BF16])
+def test_prefill_negative_scale(dtype):
+    """A negative scale: the kernel takes the tile max over -x.  Covers query tiles
+    of 128 rows (copied by TMA) and partial ones (stored by the row threads)."""
+    rng = np.random.default_rng(68)
+    d, bs, hk, g = 128, 16, 2, 2
+    lens = [256, 600, 129]
+    n_new = [256, 300, 129]    # two full tiles; a full and a ragged CTA; a tile and one row
+    c = PagedCase(rng, lens, hk * g, hk, d, bs, dtype, -0.7 / math.sqrt(d), extra_blocks=3)
+    qs = np.concatenate([[0], np.cumsum(n_new)]).astype(np.int32)
+    q = to_bits(rng.normal(0, 1, (int(qs[-1]), hk * g, d)), dtype)
+    ref = oracle_pkg.get().prefill(q, c.k_cache, c.v_cache, c.tables, c.lens, qs, c.scale, dtype, nthreads=8)
+    out = run_prefill(c, q, qs)
+    assert_close(out, ref, WK[dtype], "prefill, negative scale")
+
+
 def test_prefill_flow_then_decode():
     """Allocate and write a chunk through the library (pa_prefill_slots, K1), attend
     with pa_prefill, then take one decode step; the oracle replays every step."""

@@ -69,6 +69,17 @@ def test_shared_prefix_matches_oracle(d, bs, g, dtype):
     assert_close(ref_gpu, ref, WK[dtype], "pa_decode")
 
 
+def test_shared_prefix_negative_scale():
+    """A negative scale through the prefix kernel (its tile max is taken over -x)."""
+    rng = np.random.default_rng(79)
+    c = PagedCase(rng, [300, 200, 193, 257, 70], 4, 2, 128, 16, F16, -1 / math.sqrt(128), extra_blocks=4)
+    share(c, [0, 1, 2, 3], 192)
+    out, _, grp = run_both(c, 64)
+    assert grp.num_groups == 1
+    ref = oracle_pkg.get().decode(c.q, c.k_cache, c.v_cache, c.tables, c.lens, c.scale, F16, nthreads=8)
+    assert_close(out, ref, "f16", "shared prefix, negative scale")
+
+
 def test_no_groups_is_pa_decode():
     rng = np.random.default_rng(71)
     c = PagedCase(rng, [100, 300, 64], 4, 4, 128, 16, F16, 0.1)
