@@ -138,18 +138,40 @@ def profiled_traffic(units_now: int, workload: str, summary=PROFILE_SUMMARY):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    """SM clock and clock-event reasons during a timed region.  Read through NVML by
+    a thread every 0.2 ms from entry to exit (the timed regions here are a few
+    milliseconds long, so this puts dozens of samples under load); where NVML is not
+    usable, nvidia-smi every 200 ms around the region instead.  Only reads: no
+    setting of the GPU is changed."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits reported by name
+    NVML_BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown"}
 
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
         self.lines = []
         self.proc = None
+        self.nvml = None
+        self.samples = []  # (sm MHz, reason bits) from NVML
+        self.max_mhz = None
+        self.stop = threading.Event()
 
     def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id) if self.gpu_id.startswith("GPU-")
+                 else pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu_id)))
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.nvml = (pynvml, h)
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
@@ -161,11 +183,28 @@ class ClockSampler:
             self.proc = None
         return self
 
+    def _poll(self):
+        pynvml, h = self.nvml
+        while not self.stop.is_set():
+            try:
+                self.samples.append((float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)),
+                                     int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))))
+            except Exception:
+                return
+            time.sleep(0.0002)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
     def __exit__(self, *exc):
+        if self.nvml:
+            self.stop.set()
+            self.thread.join(timeout=5)
+            try:
+                self.nvml[0].nvmlShutdown()
+            except Exception:
+                pass
         if self.proc:
             time.sleep(0.25)
             self.proc.terminate()
@@ -176,6 +215,11 @@ class ClockSampler:
         return False
 
     def summary(self):
+        if self.samples:
+            sm = [c for c, _ in self.samples]
+            reasons = sorted({name for _, bits in self.samples for b, name in self.NVML_BITS.items() if bits & b})
+            return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                    "samples": len(sm), "source": "nvml, during the timed region"}
         rows = []
         for ln in self.lines:
             parts = [x.strip() for x in ln.split(",")]
@@ -192,7 +236,7 @@ class ClockSampler:
         sm = [r[0] for r in rows]
         loaded = [x for x in sm if x >= 0.5 * max(sm)] or sm
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "source": "nvidia-smi, around the timed region"}
 
 
 def gpu_uuid(torch, device):

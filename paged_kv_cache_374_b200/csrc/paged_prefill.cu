@@ -790,10 +790,12 @@ int launch_prefill(PrefillArgs args, const void* k_cache, const void* v_cache, i
         !encode_cache_map_swizzled(&vmap, v_cache, D, num_kv_heads, total_tokens, args.box_rows))
         return PA_ERR_CUDA;
     // q as [rows][num_heads][D]; the extent covers every row a full query tile may
-    // start at (num_seqs * max_query_len bounds the packed rows), and only tiles
-    // of 128 rows inside one sequence's chunk are copied
+    // start at (num_seqs * max_query_len bounds the packed rows, which int32
+    // query_start keeps below 2^31), and only tiles of 128 rows inside one
+    // sequence's chunk are copied
     CUtensorMap qmap;
-    if (!encode_cache_map_swizzled(&qmap, args.q, D, args.num_heads, (int64_t)num_seqs * max_query_len, kPfRows))
+    const int64_t q_rows = (int64_t)num_seqs * max_query_len;
+    if (!encode_cache_map_swizzled(&qmap, args.q, D, args.num_heads, q_rows < INT32_MAX ? q_rows : INT32_MAX, kPfRows))
         return PA_ERR_CUDA;
     dim3 grid((unsigned)((max_query_len + kPfCtaRows - 1) / kPfCtaRows), (unsigned)args.num_heads,
               (unsigned)num_seqs);
