@@ -48,6 +48,7 @@ constexpr int kPfLoadWarp = 8, kPfMmaWarp = 9;
 constexpr int kPfThreads = 320;       // softmax warps 0-3 (A) and 4-7 (B), load warp, MMA warp
 constexpr uint32_t kPfTmemCols = 512;   // O_X at column X d, S/P of tile X at 256 + 128 X
 constexpr float kPfRescaleLog2 = 8.f;
+constexpr int kPfWindow = 16;         // (sequence, head) pairs ordered together (launch order)
 
 #ifndef PA_PF_SPIN
 #define PA_PF_SPIN 1
@@ -259,15 +260,25 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
     // before the lengths arrive (entries past the sequence are ignored later)
     int pre0 = -1, pre1 = -1;
     if constexpr (!kShared) {
-        s = blockIdx.z;
-        h = blockIdx.y;
+        // CTA b (in launch order) -> (sequence, head, row tile): the (s, h) pairs go
+        // in windows of kPfWindow; inside a window every pair's heaviest row tile
+        // comes first, then every pair's next one, so that the launch ends on the
+        // lightest CTAs while a window's K/V (at most kPfWindow heads' worth) is in L2
+        const int64_t gx = gridDim.x, npairs = (int64_t)gridDim.y * gridDim.z;
+        const int64_t b = blockIdx.x + gx * (blockIdx.y + (int64_t)gridDim.y * blockIdx.z);
+        const int64_t w0 = b / (kPfWindow * gx) * kPfWindow;  // first pair of the window
+        const int64_t wn = min((int64_t)kPfWindow, npairs - w0);  // pairs in the window
+        const int64_t ib = b - w0 * gx;
+        const int64_t pair_id = w0 + ib % wn;
+        s = (int)(pair_id / gridDim.y);
+        h = (int)(pair_id % gridDim.y);
         if (warp == kPfLoadWarp && lane < kPfTok / a.box_rows) {
             const int32_t* row = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
             const int e0 = lane * a.box_rows / bs, e1 = (kPfTok + lane * a.box_rows) / bs;
             if (e0 < a.max_blocks_per_seq) pre0 = __ldg(row + e0);
             if (e1 < a.max_blocks_per_seq) pre1 = __ldg(row + e1);
         }
-        const int qt = gridDim.x - 1 - blockIdx.x;  // tiles with the most context first
+        const int qt = (int)(gx - 1 - ib / wn);  // the most context first
         q0 = a.query_start[s];
         const int n = a.query_start[s + 1] - q0;
         if (qt * kPfCtaRows >= n) return;
