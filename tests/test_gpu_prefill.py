@@ -65,6 +65,23 @@ def test_prefill_negative_scale(dtype):
     assert_close(out, ref, WK[dtype], "prefill, negative scale")
 
 
+def test_prefill_empty_chunks():
+    """Sequences with no new rows (query_start[s] == query_start[s+1]) launch CTAs that
+    find no rows and leave; the others match the oracle."""
+    rng = np.random.default_rng(69)
+    d, bs, hk, g = 128, 16, 2, 2
+    lens = [100, 300, 50, 257]
+    n_new = [0, 300, 0, 1]     # the grid is sized by the 300-row chunk
+    c = PagedCase(rng, lens, hk * g, hk, d, bs, F16, 1 / math.sqrt(d), extra_blocks=3)
+    qs = np.concatenate([[0], np.cumsum(n_new)]).astype(np.int32)
+    q = to_bits(rng.normal(0, 1, (int(qs[-1]), hk * g, d)), F16)
+    ref = oracle_pkg.get().prefill(q, c.k_cache, c.v_cache, c.tables, c.lens, qs, c.scale, F16, nthreads=8)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = run_prefill(c, q, qs, err=err)
+    assert err.item() == 0
+    assert_close(out, ref, "f16", "prefill with empty chunks")
+
+
 def test_prefill_flow_then_decode():
     """Allocate and write a chunk through the library (pa_prefill_slots, K1), attend
     with pa_prefill, then take one decode step; the oracle replays every step."""
