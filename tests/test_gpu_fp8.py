@@ -72,7 +72,7 @@ def test_decode_fp8_matches_oracle(bs, g, dtype):
     ref = oracle_pkg.get().decode_fp8(c.q, k8, v8, c.tables, c.lens, c.scale, ks, vs, dtype, nthreads=8)
     q = torch.from_numpy(c.q.view(np.int16)).view(TDT[dtype]).cuda()
     tb, ln = torch.from_numpy(c.tables).cuda(), torch.from_numpy(c.lens).cuda()
-    for pt in (0, 64):
+    for pt in (0, 64, 320, 512):
         out = torch.empty_like(q)
         pa.pa_decode_fp8(q, torch.from_numpy(k8).cuda(), torch.from_numpy(v8).cuda(), tb, ln, c.scale, ks, vs, hk,
                          out, partition_tokens=pt)
