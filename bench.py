@@ -383,14 +383,23 @@ class Ops:
 
     @property
     def fused(self):
-        """One pa_decode_step(_fp8) call per step (no shared-prefix groups)."""
-        return self.st["groups"] is None
+        """One call per step: pa_decode_step(_fp8), or pa_decode_step_shared_prefix
+        with shared-prefix groups."""
+        return True
 
     def step(self, k, v, slots, q, tables, lens, groups=None, out=None):
         if self.fused:
             st = self.st
             out = st["out"] if out is None else out
-            if self.fp8:
+            g = st["groups"]
+            if g is not None:
+                start, offs, mem = groups if groups is not None else st["group_dev"]
+                self.pa.pa_decode_step_shared_prefix(k, v, slots, q, st["k_cache"], st["v_cache"], tables, lens,
+                                                     st["spec"].scale, st["spec"].num_kv_heads, out, start, offs, mem,
+                                                     g.num_groups, g.max_group_size, g.max_shared_tokens,
+                                                     workspace=st["workspace"],
+                                                     partition_tokens=st["partition_tokens"], stream=self.stream)
+            elif self.fp8:
                 self.pa.pa_decode_step_fp8(k, v, slots, q, st["k_cache"], st["v_cache"], tables, lens,
                                            st["spec"].scale, self.ks, self.vs, st["spec"].num_kv_heads, out,
                                            workspace=st["workspace"], partition_tokens=st["partition_tokens"],
@@ -568,13 +577,13 @@ def roofline_leg(ops, ab, t, steps):
 
 
 def roofline_kernel(ops):
+    if ops.fused and ops.st["groups"] is not None:
+        return ("reshape_and_cache_kernel + shared-prefix kernel + paged_decode_kernel + paged_decode_merge_kernel "
+                "(one pa_decode_step_shared_prefix call: the prefix kernel a programmatic dependent of K1)")
     if ops.fused:
         call = "pa_decode_step_fp8" if ops.fp8 else "pa_decode_step"
         return ("reshape_and_cache_kernel + paged_decode_kernel + paged_decode_merge_kernel (one %s call: K2 a "
                 "programmatic dependent of K1)" % call)
-    if ops.st["groups"] is not None:
-        return ("shared-prefix kernel + paged_decode_kernel + paged_decode_merge_kernel (timed together: one "
-                "pa_decode_shared_prefix call)")
     return "paged_decode_kernel + paged_decode_merge_kernel (timed together: one pa_decode call)"
 
 

@@ -250,6 +250,29 @@ int pa_decode_shared_prefix(const void* q, const void* k_cache, const void* v_ca
                             void* stream);
 
 /*
+ * pa_decode_step_shared_prefix -- one decode step over shared prefixes: exactly
+ *     pa_reshape_and_cache(k, v, slot_mapping, ..., num_tokens = num_seqs, ...)
+ *     pa_decode_shared_prefix(q, ...)
+ * in one call (P2 §2.1: the step's new K/V enter their slots, then the step's
+ * query attends over the whole context; P3 §四: the beams share the prompt).
+ * The shared-prefix kernel is launched as a programmatic dependent of the cache
+ * write and lets the decode engine launch only after that write has completed:
+ * the write's launch and the prefix kernel's start overlap.  Arguments, layouts,
+ * ownership and errors as those two calls; the checks of both run before anything
+ * is launched.  The write must not touch a shared block (a block the write
+ * appends to is private to its sequence, as after copy-on-write), since the
+ * prefix kernel may read shared blocks before the write has completed.
+ */
+int pa_decode_step_shared_prefix(const void* k, const void* v, const int64_t* slot_mapping, const void* q,
+                                 void* k_cache, void* v_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, float scale, int num_kv_heads, void* out, int num_seqs,
+                                 int num_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                                 int dtype, const int32_t* seq_start, int num_groups, const int32_t* group_offsets,
+                                 const int32_t* group_members, int max_group_size, int max_shared_tokens,
+                                 int partition_tokens, void* workspace, size_t workspace_bytes, int32_t* err_word,
+                                 void* stream);
+
+/*
  * pa_find_shared_prefixes -- host-side grouping for pa_decode_shared_prefix.
  * Sequences whose first partition (partition_tokens tokens) maps to the same
  * physical blocks form a group; the group shares the longest run of whole

@@ -59,6 +59,8 @@ _sig("pa_prefill", _i32, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp
      _i32, _i32, _vp, _vp)
 _sig("pa_decode_shared_prefix", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32, _i32, _i32, _i32, _i32,
      _i32, _i32, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
+_sig("pa_decode_step_shared_prefix", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32,
+     _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
 _sig("pa_find_shared_prefixes", _i32, _i32p, _i32p, _i32, _i32, _i32, _i32, _i32p, _i32p, _i32p,
      ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int))
 _sig("pa_selftest_bounded_wait", _i32, _vp, _vp, _vp)
@@ -335,6 +337,43 @@ def pa_decode_shared_prefix(q, k_cache, v_cache, block_tables, context_lens, sca
     return out
 
 
+def pa_decode_step_shared_prefix(k, v, slot_mapping, q, k_cache, v_cache, block_tables, context_lens, scale,
+                                 num_kv_heads, out, seq_start, group_offsets, group_members, num_groups,
+                                 max_group_size, max_shared_tokens, workspace=None, partition_tokens=0, err_word=None,
+                                 stream=None):
+    """K1 then pa_decode_shared_prefix in one call: each sequence's new k/v [S, Hk, d]
+    into its slot (slot_mapping int64 [S]), then attention with the groups' shared
+    prefixes attended once per group.  Returns ``out``."""
+    import torch
+    s, h, d = q.shape
+    nb, bs, hk, d2 = k_cache.shape
+    if hk != num_kv_heads or d2 != d or v_cache.shape != k_cache.shape or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if k.shape != (s, hk, d) or v.shape != k.shape or slot_mapping.shape != (s,):
+        raise ValueError("k, v must be [S, Hk, d] and slot_mapping [S]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [S, MB] and context_lens [S]")
+    mb = block_tables.shape[1]
+    dt = _dtype_code(q)
+    for t in (k, v, k_cache, v_cache, out):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, the caches and out must share one dtype")
+    need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _lib.pa_decode_step_shared_prefix(
+        _dev(k, "k"), _dev(v, "v"), _dev(slot_mapping, "slot_mapping", torch.int64), _dev(q, "q"),
+        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), float(scale), hk, _dev(out, "out"), s, h, d, bs, nb, mb, dt,
+        _dev(seq_start, "seq_start", torch.int32), int(num_groups), _dev(group_offsets, "group_offsets", torch.int32),
+        _dev(group_members, "group_members", torch.int32), int(max_group_size), int(max_shared_tokens),
+        int(partition_tokens), _dev(workspace, "workspace"), ws_bytes, _dev(err_word, "err_word", torch.int32),
+        _stream(stream, q))
+    _check(st, "pa_decode_step_shared_prefix")
+    return out
+
+
 def pa_selftest_bounded_wait(err_word, outcome=None, stream=None) -> None:
     """Run the bounded-wait check (a wait nothing completes must time out and report)."""
     import torch
@@ -602,12 +641,15 @@ class BlockAllocator:
     """Owning wrapper over a pa_allocator handle."""
 
     def __init__(self, num_blocks: int, initial_order=None):
+        # the C function is held here: at interpreter exit the module's globals
+        # may already be gone when __del__ runs
+        self._destroy = _lib.pa_allocator_destroy
         self.handle = pa_allocator_create(num_blocks, initial_order)
 
     def __del__(self):
         h = getattr(self, "handle", None)
         if h:
-            pa_allocator_destroy(h)
+            self._destroy(h)
             self.handle = None
 
     def alloc(self) -> int:

@@ -156,6 +156,9 @@ struct SharedPrefixLaunch {
     int32_t* sched;
     int32_t* merge_cnt;
     int32_t* merge_queue;
+    // nonzero: launched as a programmatic dependent of the step's cache write,
+    // which the kernel waits for before the decode engine may launch
+    int after_write;
 };
 int launch_shared_prefix(const SharedPrefixLaunch& l, cudaStream_t stream);
 

@@ -535,27 +535,38 @@ extern "C" int pa_decode_fp8(const void* q, const void* k_cache, const void* v_c
                            : launch_decode_fp8<BF16Tag>(args, k_cache, v_cache, num_kv_heads, st);
 }
 
-extern "C" int pa_decode_shared_prefix(const void* q, const void* k_cache, const void* v_cache,
-                                       const int32_t* block_tables, const int32_t* context_lens, float scale,
-                                       int num_kv_heads, void* out, int num_seqs, int num_heads, int head_dim,
-                                       int block_size, int num_blocks, int max_blocks_per_seq, int dtype,
-                                       const int32_t* seq_start, int num_groups, const int32_t* group_offsets,
-                                       const int32_t* group_members, int max_group_size, int max_shared_tokens,
-                                       int partition_tokens, void* workspace, size_t workspace_bytes,
-                                       int32_t* err_word, void* stream) {
-    using namespace pa;
-    if (num_groups < 0 || max_group_size < 0 || max_shared_tokens < 0) return PA_ERR_INVALID_ARG;
-    DecodeArgs args;
-    const int rc = prepare_decode(args, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out,
-                                  num_seqs, num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype,
-                                  partition_tokens, workspace, workspace_bytes, err_word);
-    if (rc >= 0) return rc;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool shared = num_groups > 0 && max_shared_tokens > 0 && args.num_partitions > 1;
+namespace pa {
+namespace {
+
+// The checks of pa_decode_shared_prefix's group arguments, after prepare_decode
+// filled args.  Sets *shared when the prefix kernel runs; returns -1 when the call
+// may go on, else the status to return.
+int check_shared_prefix(const DecodeArgs& args, const int32_t* seq_start, int num_groups,
+                        const int32_t* group_offsets, const int32_t* group_members, int max_group_size,
+                        int max_shared_tokens, bool* shared) {
+    *shared = num_groups > 0 && max_shared_tokens > 0 && args.num_partitions > 1;
+    if (*shared && (!seq_start || !group_offsets || !group_members || !aligned4(seq_start) ||
+                    !aligned4(group_offsets) || !aligned4(group_members) || max_group_size <= 0 ||
+                    max_shared_tokens % args.partition_tokens != 0))
+        return PA_ERR_INVALID_ARG;
+    if (*shared && ((int64_t)(max_shared_tokens / args.partition_tokens) * num_groups > 65535 ||
+                    args.num_heads / args.group > 65535))
+        return PA_ERR_UNSUPPORTED;  // the prefix kernel's grid (groups x shared partitions, kv heads)
+    return -1;
+}
+
+// The prefix kernel (when *shared) and then the decode engine and merge.
+// after_write: the cache write of the same step was launched just before; the
+// prefix kernel runs as its programmatic dependent and holds the engine's launch
+// until the write is complete, or, with no prefix kernel, the engine waits for it.
+int launch_shared_prefix_decode(DecodeArgs args, bool shared, const void* q, const void* k_cache,
+                                const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                                float scale, int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+                                int block_size, int num_blocks, int max_blocks_per_seq, int dtype,
+                                const int32_t* seq_start, int num_groups, const int32_t* group_offsets,
+                                const int32_t* group_members, int max_group_size, int max_shared_tokens,
+                                int32_t* err_word, bool after_write, cudaStream_t st) {
     if (shared) {
-        if (!seq_start || !group_offsets || !group_members || !aligned4(seq_start) || !aligned4(group_offsets) ||
-            !aligned4(group_members) || max_group_size <= 0 || max_shared_tokens % args.partition_tokens != 0)
-            return PA_ERR_INVALID_ARG;
         SharedPrefixLaunch l{};
         l.q = q;
         l.k_cache = k_cache;
@@ -590,15 +601,81 @@ extern "C" int pa_decode_shared_prefix(const void* q, const void* k_cache, const
         l.sched = args.sched;
         l.merge_cnt = args.merge_cnt;
         l.merge_queue = args.merge_queue;
+        l.after_write = after_write ? 1 : 0;
         const int r = launch_shared_prefix(l, st);
         if (r != PA_OK) return r;
         args.seq_start = seq_start;
+    } else if (after_write) {
+        args.wait_prior = 1;
     }
     if (head_dim == 128)
         return dtype == PA_F16 ? launch_decode<F16Tag, 128>(args, k_cache, v_cache, num_kv_heads, st)
                                : launch_decode<BF16Tag, 128>(args, k_cache, v_cache, num_kv_heads, st);
     return dtype == PA_F16 ? launch_decode<F16Tag, 64>(args, k_cache, v_cache, num_kv_heads, st)
                            : launch_decode<BF16Tag, 64>(args, k_cache, v_cache, num_kv_heads, st);
+}
+
+}  // namespace
+}  // namespace pa
+
+extern "C" int pa_decode_shared_prefix(const void* q, const void* k_cache, const void* v_cache,
+                                       const int32_t* block_tables, const int32_t* context_lens, float scale,
+                                       int num_kv_heads, void* out, int num_seqs, int num_heads, int head_dim,
+                                       int block_size, int num_blocks, int max_blocks_per_seq, int dtype,
+                                       const int32_t* seq_start, int num_groups, const int32_t* group_offsets,
+                                       const int32_t* group_members, int max_group_size, int max_shared_tokens,
+                                       int partition_tokens, void* workspace, size_t workspace_bytes,
+                                       int32_t* err_word, void* stream) {
+    using namespace pa;
+    if (num_groups < 0 || max_group_size < 0 || max_shared_tokens < 0) return PA_ERR_INVALID_ARG;
+    DecodeArgs args;
+    const int rc = prepare_decode(args, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out,
+                                  num_seqs, num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype,
+                                  partition_tokens, workspace, workspace_bytes, err_word);
+    if (rc >= 0) return rc;
+    bool shared = false;
+    const int rs = check_shared_prefix(args, seq_start, num_groups, group_offsets, group_members, max_group_size,
+                                       max_shared_tokens, &shared);
+    if (rs >= 0) return rs;
+    return launch_shared_prefix_decode(args, shared, q, k_cache, v_cache, block_tables, context_lens, scale,
+                                       num_kv_heads, num_seqs, num_heads, head_dim, block_size, num_blocks,
+                                       max_blocks_per_seq, dtype, seq_start, num_groups, group_offsets,
+                                       group_members, max_group_size, max_shared_tokens, err_word, false,
+                                       static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int pa_decode_step_shared_prefix(const void* k, const void* v, const int64_t* slot_mapping, const void* q,
+                                            void* k_cache, void* v_cache, const int32_t* block_tables,
+                                            const int32_t* context_lens, float scale, int num_kv_heads, void* out,
+                                            int num_seqs, int num_heads, int head_dim, int block_size,
+                                            int num_blocks, int max_blocks_per_seq, int dtype,
+                                            const int32_t* seq_start, int num_groups, const int32_t* group_offsets,
+                                            const int32_t* group_members, int max_group_size,
+                                            int max_shared_tokens, int partition_tokens, void* workspace,
+                                            size_t workspace_bytes, int32_t* err_word, void* stream) {
+    using namespace pa;
+    // every check of both calls before anything is launched
+    if (num_groups < 0 || max_group_size < 0 || max_shared_tokens < 0) return PA_ERR_INVALID_ARG;
+    const int rk = check_reshape_and_cache(k, v, slot_mapping, k_cache, v_cache, num_seqs, num_kv_heads, head_dim,
+                                           block_size, num_blocks, dtype, err_word);
+    if (rk > 0) return rk;
+    DecodeArgs args;
+    const int rc = prepare_decode(args, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, out,
+                                  num_seqs, num_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, dtype,
+                                  partition_tokens, workspace, workspace_bytes, err_word);
+    if (rc >= 0) return rc;  // an error, or an empty batch (num_seqs == 0: nothing to write either)
+    bool shared = false;
+    const int rs = check_shared_prefix(args, seq_start, num_groups, group_offsets, group_members, max_group_size,
+                                       max_shared_tokens, &shared);
+    if (rs >= 0) return rs;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int r1 = launch_reshape_and_cache(k, v, slot_mapping, k_cache, v_cache, num_seqs, num_kv_heads, head_dim,
+                                            block_size, num_blocks, err_word, st);
+    if (r1 != PA_OK) return r1;
+    return launch_shared_prefix_decode(args, shared, q, k_cache, v_cache, block_tables, context_lens, scale,
+                                       num_kv_heads, num_seqs, num_heads, head_dim, block_size, num_blocks,
+                                       max_blocks_per_seq, dtype, seq_start, num_groups, group_offsets,
+                                       group_members, max_group_size, max_shared_tokens, err_word, true, st);
 }
 
 extern "C" int pa_decode_step(const void* k, const void* v, const int64_t* slot_mapping, const void* q,

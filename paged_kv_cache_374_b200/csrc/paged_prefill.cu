@@ -298,6 +298,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
         kv_head = h / a.group;
         tab = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
     } else {
+        // Launched as a programmatic dependent of the decode step's cache write, the
+        // grid lets the decode engine launch only once that write is complete, so
+        // the engine reads the step's new K/V with no wait of its own (this grid's
+        // own reads are of shared blocks, which the write never touches).  Launched
+        // plainly, the wait returns at once.
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         // the decode engine that follows may start on the SMs this grid leaves free
         asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
         const int g = blockIdx.z / a.max_shared_partitions;
@@ -816,7 +822,7 @@ int launch_prefill(PrefillArgs args, const void* k_cache, const void* v_cache, i
 
 template <class Tag, int D>
 int launch_shared(PrefillArgs args, const void* k_cache, const void* v_cache, int num_kv_heads, int num_groups,
-                  int max_group_size, cudaStream_t stream) {
+                  int max_group_size, bool after_write, cudaStream_t stream) {
     using Lay = PfLayout<D>;
     static std::atomic<uint64_t> smem_done{0};
     auto kernel = paged_prefill_kernel<Tag, D, true>;
@@ -830,6 +836,19 @@ int launch_shared(PrefillArgs args, const void* k_cache, const void* v_cache, in
     const int64_t rows = (int64_t)max_group_size * args.group;
     dim3 grid((unsigned)((rows + kPfCtaRows - 1) / kPfCtaRows), (unsigned)num_kv_heads,
               (unsigned)(num_groups * args.max_shared_partitions));
+    if (after_write) {  // a programmatic dependent of the cache write launched just before
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(kPfThreads);
+        cfg.dynamicSmemBytes = Lay::kAlloc;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kernel, args, kmap, vmap, kmap) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    }
     kernel<<<grid, kPfThreads, Lay::kAlloc, stream>>>(args, kmap, vmap, kmap);  // (no q map in this mode)
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -866,15 +885,16 @@ int launch_shared_prefix(const SharedPrefixLaunch& l, cudaStream_t stream) {
     args.sched = l.sched;
     args.merge_cnt = l.merge_cnt;
     args.merge_queue = l.merge_queue;
+    const bool after = l.after_write != 0;
     if (l.head_dim == 128)
         return l.dtype == PA_F16 ? launch_shared<F16Tag, 128>(args, l.k_cache, l.v_cache, l.num_kv_heads, l.num_groups,
-                                                              l.max_group_size, stream)
+                                                              l.max_group_size, after, stream)
                                  : launch_shared<BF16Tag, 128>(args, l.k_cache, l.v_cache, l.num_kv_heads,
-                                                               l.num_groups, l.max_group_size, stream);
+                                                               l.num_groups, l.max_group_size, after, stream);
     return l.dtype == PA_F16 ? launch_shared<F16Tag, 64>(args, l.k_cache, l.v_cache, l.num_kv_heads, l.num_groups,
-                                                         l.max_group_size, stream)
+                                                         l.max_group_size, after, stream)
                              : launch_shared<BF16Tag, 64>(args, l.k_cache, l.v_cache, l.num_kv_heads, l.num_groups,
-                                                          l.max_group_size, stream);
+                                                          l.max_group_size, after, stream);
 }
 
 }  // namespace pa

@@ -201,3 +201,109 @@ def test_group_arrays_out_of_range_are_skipped(bad):
     ref = oracle_pkg.get().decode(c.q, c.k_cache, c.v_cache, c.tables, c.lens, c.scale, F16, pairs=pairs)
     got = out[torch.from_numpy(pairs[:, 0]).long(), torch.from_numpy(pairs[:, 1]).long()]
     assert_close(got, ref, "f16", f"groups beside a bad one ({bad})")
+
+
+def same_bits(a, b):
+    """Bit-for-bit equality (unused cache rows hold NaN, which compares unequal)."""
+    return torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def _new_tokens(c, rng):
+    """Each sequence's new K/V row [S, Hk, d] and its slot: position L-1, which lies
+    past every shared prefix (in a block private to the sequence)."""
+    slots = np.array([c.tables[s, (n - 1) // c.bs] * c.bs + (n - 1) % c.bs for s, n in enumerate(c.lens)],
+                     dtype=np.int64)
+    shape = (len(c.lens), c.Hk, c.d)
+    k = torch.from_numpy(rng.standard_normal(shape).astype(np.float32)).to(TDT[c.dtype]).cuda()
+    v = torch.from_numpy(rng.standard_normal(shape).astype(np.float32)).to(TDT[c.dtype]).cuda()
+    return k, v, torch.from_numpy(slots).cuda()
+
+
+@pytest.mark.parametrize("dtype", [F16, BF16])
+def test_decode_step_shared_prefix_is_write_then_decode(dtype):
+    """pa_decode_step_shared_prefix (the prefix kernel a programmatic dependent of the
+    cache write) equals pa_reshape_and_cache then pa_decode_shared_prefix bit for bit,
+    caches and output, over nested groups and three back-to-back steps; the output
+    is the oracle's decode over the written caches."""
+    rng = np.random.default_rng(80)
+    P = 64
+    c = PagedCase(rng, [300, 200, 193, 257, 140, 129, 130, 400, 90, 1], 8, 2, 128, 16, dtype, 1 / math.sqrt(128),
+                  extra_blocks=4)
+    share(c, [0, 1, 2, 3], 192)
+    share(c, [0, 4], 64)
+    share(c, [5, 6, 7], 128)
+    grp = pa.pa_find_shared_prefixes(c.tables, c.lens, c.bs, P)
+    assert grp.num_groups == 2
+    start, offs, mem = grp.to("cuda")
+    q = dev(c.q, dtype)
+    tb, ln = torch.from_numpy(c.tables).cuda(), torch.from_numpy(c.lens).cuda()
+    k, v, slots = _new_tokens(c, rng)
+    kc_a, vc_a = dev(c.k_cache, dtype), dev(c.v_cache, dtype)
+    kc_b, vc_b = kc_a.clone(), vc_a.clone()
+    err_a = torch.zeros(1, dtype=torch.int32, device="cuda")
+    err_b = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out_a, out_b = torch.empty_like(q), torch.empty_like(q)
+    pa.pa_reshape_and_cache(k, v, slots, kc_a, vc_a, err_word=err_a)
+    pa.pa_decode_shared_prefix(q, kc_a, vc_a, tb, ln, c.scale, c.Hk, out_a, start, offs, mem, grp.num_groups,
+                               grp.max_group_size, grp.max_shared_tokens, partition_tokens=P, err_word=err_a)
+    for _ in range(3):
+        pa.pa_decode_step_shared_prefix(k, v, slots, q, kc_b, vc_b, tb, ln, c.scale, c.Hk, out_b, start, offs, mem,
+                                        grp.num_groups, grp.max_group_size, grp.max_shared_tokens,
+                                        partition_tokens=P, err_word=err_b)
+    torch.cuda.synchronize()
+    assert err_a.item() == 0 and err_b.item() == 0
+    assert same_bits(kc_a, kc_b) and same_bits(vc_a, vc_b)
+    assert same_bits(out_a, out_b)
+    kh, vh = bits(kc_b), bits(vc_b)
+    ref = oracle_pkg.get().decode(c.q, kh, vh, c.tables, c.lens, c.scale, dtype, nthreads=8)
+    assert_close(out_b, ref, WK[dtype], "fused shared-prefix step")
+
+
+def test_decode_step_shared_prefix_without_groups_is_decode_step():
+    """With no groups the call is pa_decode_step, bit for bit."""
+    rng = np.random.default_rng(81)
+    c = PagedCase(rng, [100, 300, 64], 4, 4, 128, 16, F16, 0.1)
+    grp = pa.pa_find_shared_prefixes(c.tables, c.lens, c.bs, 64)
+    assert grp.num_groups == 0
+    start, offs, mem = grp.to("cuda")
+    q = dev(c.q, F16)
+    tb, ln = torch.from_numpy(c.tables).cuda(), torch.from_numpy(c.lens).cuda()
+    k, v, slots = _new_tokens(c, rng)
+    kc_a, vc_a = dev(c.k_cache, F16), dev(c.v_cache, F16)
+    kc_b, vc_b = kc_a.clone(), vc_a.clone()
+    out_a, out_b = torch.empty_like(q), torch.empty_like(q)
+    pa.pa_decode_step(k, v, slots, q, kc_a, vc_a, tb, ln, c.scale, c.Hk, out_a, partition_tokens=64)
+    pa.pa_decode_step_shared_prefix(k, v, slots, q, kc_b, vc_b, tb, ln, c.scale, c.Hk, out_b, start, offs, mem,
+                                    grp.num_groups, grp.max_group_size, grp.max_shared_tokens, partition_tokens=64)
+    torch.cuda.synchronize()
+    assert same_bits(kc_a, kc_b) and same_bits(vc_a, vc_b) and same_bits(out_a, out_b)
+
+
+def test_beam_decode_step_shared_prefix():
+    """The beam workload's step through pa_decode_step_shared_prefix: bitwise the
+    two-call step, and the oracle's decode on sampled (sequence, head) pairs."""
+    step = Step("beam")
+    t = step.tensors()
+    grp = pa.pa_find_shared_prefixes(step.tables, step.lens, step.bs, 256)
+    start, offs, mem = grp.to("cuda")
+    tb, ln = torch.from_numpy(step.tables).cuda(), torch.from_numpy(step.lens).cuda()
+    slots = torch.from_numpy(step.slots).cuda()
+    kc_b, vc_b = t["k_cache"].clone(), t["v_cache"].clone()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out_a, out_b = torch.empty_like(t["q"]), torch.empty_like(t["q"])
+    pa.pa_reshape_and_cache(t["k"], t["v"], slots, t["k_cache"], t["v_cache"], err_word=err)
+    pa.pa_decode_shared_prefix(t["q"], t["k_cache"], t["v_cache"], tb, ln, step.spec.scale, 32, out_a, start, offs,
+                               mem, grp.num_groups, grp.max_group_size, grp.max_shared_tokens, err_word=err)
+    pa.pa_decode_step_shared_prefix(t["k"], t["v"], slots, t["q"], kc_b, vc_b, tb, ln, step.spec.scale, 32, out_b,
+                                    start, offs, mem, grp.num_groups, grp.max_group_size, grp.max_shared_tokens,
+                                    err_word=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert same_bits(t["k_cache"], kc_b) and same_bits(t["v_cache"], vc_b) and same_bits(out_a, out_b)
+    rng = np.random.default_rng(82)
+    pairs = np.array([(int(rng.integers(0, step.spec.num_seqs)), int(rng.integers(0, 32))) for _ in range(32)],
+                     dtype=np.int32)
+    ref = oracle_pkg.get().decode(bits(t["q"]), bits(kc_b), bits(vc_b), step.tables, step.lens, step.spec.scale, F16,
+                                  pairs=pairs, nthreads=8)
+    got = out_b[torch.from_numpy(pairs[:, 0]).long(), torch.from_numpy(pairs[:, 1]).long()]
+    assert_close(got, ref, "f16", "beam fused step")
