@@ -307,3 +307,34 @@ def test_beam_decode_step_shared_prefix():
                                   pairs=pairs, nthreads=8)
     got = out_b[torch.from_numpy(pairs[:, 0]).long(), torch.from_numpy(pairs[:, 1]).long()]
     assert_close(got, ref, "f16", "beam fused step")
+
+
+def test_decode_step_shared_prefix_more_sequences_than_one_launch():
+    """The fused step with 1100 sequences in four groups (two engine launches, which
+    start only once the cache write is complete): bit for bit the two calls."""
+    rng = np.random.default_rng(83)
+    S, P, bs = 1100, 64, 16
+    lens = rng.integers(65, 400, size=S).astype(np.int32)
+    c = PagedCase(rng, lens, 2, 2, 64, bs, F16, 0.125, extra_blocks=2)
+    for g in [list(range(0, 300)), list(range(300, 700)), list(range(700, 1050, 2)), [1098, 1099]]:
+        share(c, g, 64 * int(min(-(-int(min(lens[g])) // 64) - 1, 3)))
+    grp = pa.pa_find_shared_prefixes(c.tables, c.lens, c.bs, P)
+    assert grp.num_groups >= 4
+    start, offs, mem = grp.to("cuda")
+    q = dev(c.q, F16)
+    tb, ln = torch.from_numpy(c.tables).cuda(), torch.from_numpy(c.lens).cuda()
+    k, v, slots = _new_tokens(c, rng)
+    kc_a, vc_a = dev(c.k_cache, F16), dev(c.v_cache, F16)
+    kc_b, vc_b = kc_a.clone(), vc_a.clone()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out_a, out_b = torch.empty_like(q), torch.empty_like(q)
+    pa.pa_reshape_and_cache(k, v, slots, kc_a, vc_a, err_word=err)
+    pa.pa_decode_shared_prefix(q, kc_a, vc_a, tb, ln, c.scale, c.Hk, out_a, start, offs, mem, grp.num_groups,
+                               grp.max_group_size, grp.max_shared_tokens, partition_tokens=P, err_word=err)
+    for _ in range(2):
+        pa.pa_decode_step_shared_prefix(k, v, slots, q, kc_b, vc_b, tb, ln, c.scale, c.Hk, out_b, start, offs, mem,
+                                        grp.num_groups, grp.max_group_size, grp.max_shared_tokens,
+                                        partition_tokens=P, err_word=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert same_bits(kc_a, kc_b) and same_bits(vc_a, vc_b) and same_bits(out_a, out_b)
