@@ -61,7 +61,7 @@ _sig("pa_decode_shared_prefix", _i32, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _
      _i32, _i32, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
 _sig("pa_decode_step_shared_prefix", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _i32,
      _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp, _vp)
-_sig("pa_find_shared_prefixes", _i32, _i32p, _i32p, _i32, _i32, _i32, _i32, _i32p, _i32p, _i32p,
+_sig("pa_find_shared_prefixes", _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
      ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int))
 _sig("pa_selftest_bounded_wait", _i32, _vp, _vp, _vp)
 _sig("pa_allocator_create", _vp, _i32, _i32p)
@@ -130,6 +130,13 @@ def _h32(a: np.ndarray):
     return a.ctypes.data_as(_i32p)
 
 
+def _h32_addr(a: np.ndarray) -> int:
+    """Address of a C-contiguous int32 numpy array, for a void* argument (cheaper per
+    call than building a typed pointer: the grouping runs every decode step)."""
+    assert a.dtype == np.int32 and a.flags.c_contiguous
+    return a.ctypes.data
+
+
 def _stream(stream, like):
     import torch
     if stream is None:
@@ -185,8 +192,8 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_hea
     for t in (k_cache, v_cache, out):
         if t.dtype != q.dtype:
             raise TypeError("q, the caches and out must share one dtype")
-    need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
     if workspace is None:
+        need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
         workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
     ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
@@ -217,8 +224,8 @@ def pa_decode_step(k, v, slot_mapping, q, k_cache, v_cache, block_tables, contex
     for t in (k, v, k_cache, v_cache, out):
         if t.dtype != q.dtype:
             raise TypeError("q, k, v, the caches and out must share one dtype")
-    need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
     if workspace is None:
+        need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
         workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
     st = _lib.pa_decode_step(_dev(k, "k"), _dev(v, "v"), _dev(slot_mapping, "slot_mapping", torch.int64),
                              _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
@@ -250,8 +257,8 @@ def pa_decode_step_fp8(k, v, slot_mapping, q, k_cache, v_cache, block_tables, co
         if t.dtype != q.dtype:
             raise TypeError("q, k, v and out must share one dtype")
     mb = block_tables.shape[1]
-    need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
     if workspace is None:
+        need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
         workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
     st = _lib.pa_decode_step_fp8(_dev(k, "k"), _dev(v, "v"), _dev(slot_mapping, "slot_mapping", torch.int64),
                                  _dev(q, "q"), _dev(k_cache, "k_cache", torch.uint8),
@@ -294,9 +301,9 @@ def pa_find_shared_prefixes(block_tables: np.ndarray, context_lens: np.ndarray, 
     offs = np.zeros(s + 1, dtype=np.int32)
     members = np.zeros(max(s, 1), dtype=np.int32)
     ng, mg, mt = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
-    st = _lib.pa_find_shared_prefixes(_h32(tb), _h32(ln), s, mb, block_size, partition_tokens, _h32(start),
-                                      _h32(offs), _h32(members), ctypes.byref(ng), ctypes.byref(mg),
-                                      ctypes.byref(mt))
+    st = _lib.pa_find_shared_prefixes(_h32_addr(tb), _h32_addr(ln), s, mb, block_size, partition_tokens,
+                                      _h32_addr(start), _h32_addr(offs), _h32_addr(members), ctypes.byref(ng),
+                                      ctypes.byref(mg), ctypes.byref(mt))
     _check(st, "pa_find_shared_prefixes")
     n = int(ng.value)
     return SharedPrefixes(start, offs[: n + 1].copy(), members[: int(offs[n])].copy(), n, int(mg.value),
@@ -321,8 +328,8 @@ def pa_decode_shared_prefix(q, k_cache, v_cache, block_tables, context_lens, sca
     for t in (k_cache, v_cache, out):
         if t.dtype != q.dtype:
             raise TypeError("q, the caches and out must share one dtype")
-    need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
     if workspace is None:
+        need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
         workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
     st = _lib.pa_decode_shared_prefix(
@@ -358,8 +365,8 @@ def pa_decode_step_shared_prefix(k, v, slot_mapping, q, k_cache, v_cache, block_
     for t in (k, v, k_cache, v_cache, out):
         if t.dtype != q.dtype:
             raise TypeError("q, k, v, the caches and out must share one dtype")
-    need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
     if workspace is None:
+        need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
         workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
     st = _lib.pa_decode_step_shared_prefix(
@@ -437,8 +444,8 @@ def pa_decode_fp8(q, k_cache, v_cache, block_tables, context_lens, scale, k_scal
         raise TypeError("q and out must share one dtype")
     mb = block_tables.shape[1]
     dt = _dtype_code(q)
-    need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
     if workspace is None:
+        need = pa_decode_workspace_size(s, h, hk, d, bs, mb, partition_tokens)
         workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=q.device)
     st = _lib.pa_decode_fp8(_dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
                             _dev(block_tables, "block_tables", torch.int32),
