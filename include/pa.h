@@ -256,12 +256,10 @@ int pa_decode_shared_prefix(const void* q, const void* k_cache, const void* v_ca
  * in one call (P2 §2.1: the step's new K/V enter their slots, then the step's
  * query attends over the whole context; P3 §四: the beams share the prompt).
  * The shared-prefix kernel is launched as a programmatic dependent of the cache
- * write and lets the decode engine launch only after that write has completed:
- * the write's launch and the prefix kernel's start overlap.  Arguments, layouts,
- * ownership and errors as those two calls; the checks of both run before anything
- * is launched.  The write must not touch a shared block (a block the write
- * appends to is private to its sequence, as after copy-on-write), since the
- * prefix kernel may read shared blocks before the write has completed.
+ * write: its launch and start overlap the write, it waits for the write to
+ * complete before it reads anything, and only then lets the decode engine launch.
+ * The result is exactly that of the two calls.  Arguments, layouts, ownership and
+ * errors as those two calls; the checks of both run before anything is launched.
  */
 int pa_decode_step_shared_prefix(const void* k, const void* v, const int64_t* slot_mapping, const void* q,
                                  void* k_cache, void* v_cache, const int32_t* block_tables,

@@ -299,10 +299,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
         tab = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
     } else {
         // Launched as a programmatic dependent of the decode step's cache write, the
-        // grid lets the decode engine launch only once that write is complete, so
-        // the engine reads the step's new K/V with no wait of its own (this grid's
-        // own reads are of shared blocks, which the write never touches).  Launched
-        // plainly, the wait returns at once.
+        // grid reads nothing before that write is complete, and lets the decode
+        // engine launch only then, so the engine reads the step's new K/V with no
+        // wait of its own.  Launched plainly, the wait returns at once.
         asm volatile("griddepcontrol.wait;" ::: "memory");
         // the decode engine that follows may start on the SMs this grid leaves free
         asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
