@@ -798,6 +798,9 @@ def measure_append_loop(torch, name, device, args, target_s=0.8):
            "roofline_us_first_last": [round(float(k2_ms[0]) * 1e3, 2), round(float(k2_ms[-1]) * 1e3, 2)],
            "bytes_per_pass": int(sum(step_bytes)), "kv_gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
            "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+           # DRAM bytes per step from the ncu summary, scaled to the loop's mean context tokens per step
+           "traffic": profiled_traffic(float(np.mean([np.sum(ps[1]) for ps in per_step])), spec.name,
+                                       TRAFFIC_SUMMARIES.get(spec.name, PROFILE_SUMMARY)),
            "kv_gbs_min_max_step": [round(min(gbs_steps), 1), round(max(gbs_steps), 1)],
            "a1_us_mean": round(float(np.mean(a1_us)), 1), "clocks": sampler.summary(),
            "e2e_tokens_per_s": round(S * nsteps * passes / (e2e_ms / 1e3), 1),
