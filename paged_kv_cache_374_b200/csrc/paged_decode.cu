@@ -549,9 +549,8 @@ int check_shared_prefix(const DecodeArgs& args, const int32_t* seq_start, int nu
                     !aligned4(group_offsets) || !aligned4(group_members) || max_group_size <= 0 ||
                     max_shared_tokens % args.partition_tokens != 0))
         return PA_ERR_INVALID_ARG;
-    if (*shared && ((int64_t)(max_shared_tokens / args.partition_tokens) * num_groups > 65535 ||
-                    args.num_heads / args.group > 65535))
-        return PA_ERR_UNSUPPORTED;  // the prefix kernel's grid (groups x shared partitions, kv heads)
+    if (*shared && (num_groups > 65535 || args.num_heads / args.group > 65535))
+        return PA_ERR_UNSUPPORTED;  // the prefix kernel's grid (groups, kv heads)
     return -1;
 }
 

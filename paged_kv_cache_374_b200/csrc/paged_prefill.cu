@@ -185,13 +185,13 @@ struct PrefillArgs {
     int32_t* merge_queue;
 };
 
-// One partial of (seq, head) is in the workspace (this thread's stores fenced
-// first); the write that completes the sequence's partitions queues it.
-__device__ __forceinline__ void count_partial(const PrefillArgs& a, int seq, int head) {
+// n partition slots of (seq, head) are in the workspace (this thread's stores
+// fenced first); the write that completes the sequence's partitions queues it.
+__device__ __forceinline__ void count_partial(const PrefillArgs& a, int seq, int head, int n) {
     __threadfence();
     const int sh = seq * a.num_heads + head;
     const int np = (a.context_lens[seq] + a.partition_tokens - 1) / a.partition_tokens;
-    if (atomicAdd(a.merge_cnt + sh, 1) == np - 1) {
+    if (atomicAdd(a.merge_cnt + sh, n) + n == np) {
         const int slot = atomicAdd(a.sched + 2, 1);
         asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(a.merge_queue + slot), "r"(sh + 1) : "memory");
     }
@@ -254,8 +254,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
     const int32_t* tab;
     // prefill: rows q_first .. of sequence s, head h
     int s = 0, h = 0, q0 = 0, q_first = 0;
-    // shared prefix: rows q_first .. of the group's (member, query head) list, partition p
-    int m0 = 0, p = 0;
+    // shared prefix: rows q_first .. of the group's (member, query head) list
+    int m0 = 0;
     // prefill: the load warp's table entries for its boxes of tiles 0 and 1, read
     // before the lengths arrive (entries past the sequence are ignored later)
     int pre0 = -1, pre1 = -1;
@@ -305,8 +305,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
         asm volatile("griddepcontrol.wait;" ::: "memory");
         // the decode engine that follows may start on the SMs this grid leaves free
         asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-        const int g = blockIdx.z / a.max_shared_partitions;
-        p = blockIdx.z - g * a.max_shared_partitions;
+        const int g = blockIdx.z;
         kv_head = blockIdx.y;
         m0 = a.group_offsets[g];
         const int m1 = a.group_offsets[g + 1];
@@ -319,7 +318,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
                 bad_group |= mem < 0 || mem >= a.num_seqs;
             }
         if (__syncthreads_or(bad_group)) {
-            if (tid == 0 && p == 0 && blockIdx.x == 0 && blockIdx.y == 0) report(a.err_word, PA_DEVERR_GROUP_RANGE);
+            if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0) report(a.err_word, PA_DEVERR_GROUP_RANGE);
             return;
         }
         const int rows = (m1 - m0) * a.group;
@@ -330,17 +329,20 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
         L = a.seq_start[lead];  // tokens shared by the group
         const int P = a.partition_tokens;
         if (L <= 0 || L % P != 0 || L > a.max_blocks_per_seq * bs) {  // the group's start is unusable
-            if (tid == 0 && p == 0 && blockIdx.x == 0 && blockIdx.y == 0) report(a.err_word, PA_DEVERR_LEN_RANGE);
+            if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0) report(a.err_word, PA_DEVERR_LEN_RANGE);
             return;
         }
         // the launch bounds (max_group_size, max_shared_tokens) must cover every group
-        if (tid == 0 && ((p == a.max_shared_partitions - 1 && L > a.max_shared_partitions * P) ||
+        if (tid == 0 && ((blockIdx.x == 0 && L > a.max_shared_partitions * P) ||
                          (blockIdx.x == gridDim.x - 1 && rows > (int)gridDim.x * kPfCtaRows)))
             report(a.err_word, PA_DEVERR_LEN_RANGE);
-        if ((p + 1) * P > L) return;  // past this group's prefix
-        base_pos = 1 << 29;  // no causal mask: every row sees the whole partition
-        tok0 = p * P;
-        tok_end = (p + 1) * P;
+        // One CTA covers the whole shared prefix, all L / P partitions: its result
+        // goes into the first partition's slot, and the others are marked absent
+        // (running max -inf), which the merge skips.  One CTA per partition would
+        // pay the CTA's start-up and epilogue once per partition.
+        base_pos = 1 << 29;  // no causal mask: every row sees the whole prefix
+        tok0 = 0;
+        tok_end = L;
         tab = a.block_tables + (int64_t)lead * a.max_blocks_per_seq;
     }
     // K/V tiles of each query tile: up to the one holding the last token its last row sees
@@ -447,10 +449,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
             for (int r = tid; r < nrows; r += kPfThreads) {
                 int seq, head;
                 shared_row(r, seq, head);
-                const int64_t pi = ((int64_t)seq * a.num_heads + head) * a.num_partitions + p;
+                const int64_t pi = ((int64_t)seq * a.num_heads + head) * a.num_partitions;
                 a.ws_m[pi] = __int_as_float(0x7fc00000);
                 a.ws_l[pi] = __int_as_float(0x7fc00000);
-                if (a.early_merge) count_partial(a, seq, head);  // merged, so the NaN reaches the row
+                for (int k = 1; k < L / a.partition_tokens; ++k) a.ws_m[pi + k] = -INFINITY;
+                // merged, so the NaN reaches the row
+                if (a.early_merge) count_partial(a, seq, head, L / a.partition_tokens);
             }
             if (tid == 0) report(a.err_word, PA_DEVERR_TABLE_RANGE);
             return;
@@ -717,8 +721,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
         }
         if (ok && nt > 0) ok = __all_sync(FULL, pf_wait(&bars[kBarOLast + x], 0) && !*abort_flag);
         if (ok && nt > 0 && kShared) {
-            // partial of this partition for the row's (sequence, head): running max
-            // (base-2 units, scores scaled by scale * log2 e), sum, unnormalised o
+            // partial of the whole prefix for the row's (sequence, head), in the
+            // first partition's slot: running max (base-2 units, scores scaled by
+            // scale * log2 e), sum, unnormalised o
             umma::fence_after_sync();
             bool write = r < nrows;
             int64_t pi = 0;
@@ -731,7 +736,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
                     report(a.err_word, PA_DEVERR_LEN_RANGE);
                     write = false;
                 }
-                pi = ((int64_t)seq * a.num_heads + head) * a.num_partitions + p;
+                pi = ((int64_t)seq * a.num_heads + head) * a.num_partitions;
             }
             float4* dst = reinterpret_cast<float4*>(a.ws_o + pi * D);
 #pragma unroll 1
@@ -749,7 +754,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) paged_prefill_kernel(const Pref
             if (write) {
                 a.ws_m[pi] = m_used;
                 a.ws_l[pi] = l;
-                if (a.early_merge) count_partial(a, seq, head);
+                for (int k = 1; k < L / a.partition_tokens; ++k) a.ws_m[pi + k] = -INFINITY;  // absent
+                if (a.early_merge) count_partial(a, seq, head, L / a.partition_tokens);
             }
         } else if (ok && nt > 0) {
             umma::fence_after_sync();
@@ -834,7 +840,7 @@ int launch_shared(PrefillArgs args, const void* k_cache, const void* v_cache, in
         return PA_ERR_CUDA;
     const int64_t rows = (int64_t)max_group_size * args.group;
     dim3 grid((unsigned)((rows + kPfCtaRows - 1) / kPfCtaRows), (unsigned)num_kv_heads,
-              (unsigned)(num_groups * args.max_shared_partitions));
+              (unsigned)num_groups);
     if (after_write) {  // a programmatic dependent of the cache write launched just before
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = grid;
@@ -858,7 +864,7 @@ int launch_shared_prefix(const SharedPrefixLaunch& l, cudaStream_t stream) {
     if (l.partition_tokens % 64 != 0 || l.max_shared_tokens % l.partition_tokens != 0) return PA_ERR_INVALID_ARG;
     const int64_t maxpp = l.max_shared_tokens / l.partition_tokens;
     if (maxpp == 0 || l.num_groups == 0) return PA_OK;
-    if (maxpp * l.num_groups > 65535 || l.num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    if (l.num_groups > 65535 || l.num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
     PrefillArgs args{};
     args.q = static_cast<const uint16_t*>(l.q);
     args.block_tables = l.block_tables;
