@@ -338,3 +338,22 @@ def test_decode_step_shared_prefix_more_sequences_than_one_launch():
     torch.cuda.synchronize()
     assert err.item() == 0
     assert same_bits(kc_a, kc_b) and same_bits(vc_a, vc_b) and same_bits(out_a, out_b)
+
+
+def test_bad_table_entry_in_a_shared_prefix():
+    """A table entry out of range inside a group's shared prefix: the prefix kernel
+    copies nothing from it and reports PA_DEVERR_TABLE_RANGE, and the prefix partial
+    is NaN, so every member's rows come out NaN; the sequence outside the group
+    still gets the oracle's result."""
+    rng = np.random.default_rng(84)
+    c = PagedCase(rng, [300, 280, 290, 200], 4, 4, 128, 16, F16, 1 / math.sqrt(128))
+    share(c, [0, 1, 2], 256)
+    ref = oracle_pkg.get().decode(c.q, c.k_cache, c.v_cache, c.tables, c.lens, c.scale, F16)
+    for s in (0, 1, 2):  # the members' common entry 3 (tokens 48-63) points past the pool
+        c.tables[s, 3] = c.NB + 7
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, _, grp = run_both(c, 64, err=err)
+    assert grp.num_groups == 1 and list(grp.seq_start) == [256, 256, 256, 0]
+    assert err.item() & pa.PA_DEVERR_TABLE_RANGE
+    assert torch.isnan(out[:3].float()).all()
+    assert_close(out[3:], ref[3:], "f16", "sequence outside the group")
